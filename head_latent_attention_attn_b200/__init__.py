@@ -1,0 +1,261 @@
+"""Python binding of libmla.so, the B200 (sm_100a) weight-absorbed MLA decode library.
+
+The functions here carry the C ABI's names (include/mla.h) and only marshal arguments:
+they check torch tensors' device, dtype, contiguity and shapes, take their data
+pointers and the current CUDA stream, and call the library. Every step of the decode
+path runs in the library's CUDA kernels; there is no other implementation. If the
+library is not built, every call raises ``MlaError``.
+
+Decode step, in the absorbed order of the DeepSeek-V2 MLA page ("Matrix absorption"):
+    mla_cache_append -> mla_absorb_q -> mla_decode_attn -> mla_out_up
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Optional
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libmla.so")
+
+MLA_OK = 0
+MLA_ERR_INVALID_ARG = 1
+MLA_ERR_UNSUPPORTED = 2
+MLA_ERR_WORKSPACE = 3
+MLA_ERR_CUDA = 4
+MLA_ERR_DEVICE_BOUNDS = 5
+MLA_ERR_DEVICE_TIMEOUT = 6
+STATUS_NAMES = {0: "MLA_OK", 1: "MLA_ERR_INVALID_ARG", 2: "MLA_ERR_UNSUPPORTED",
+                3: "MLA_ERR_WORKSPACE", 4: "MLA_ERR_CUDA", 5: "MLA_ERR_DEVICE_BOUNDS",
+                6: "MLA_ERR_DEVICE_TIMEOUT"}
+
+# Public C symbols (kept in sync with include/mla.h; a CPU test checks both ways).
+C_SYMBOLS = ("mla_row_width", "mla_status_string", "mla_cache_append", "mla_absorb_q",
+             "mla_decode_workspace_size", "mla_decode_attn", "mla_out_up",
+             "mla_get_device_status")
+
+
+class MlaError(RuntimeError):
+    def __init__(self, msg: str, status: int = MLA_ERR_CUDA):
+        super().__init__(msg)
+        self.status = status
+
+
+class MlaDims(ctypes.Structure):
+    _fields_ = [("num_heads", ctypes.c_int32), ("num_kv_groups", ctypes.c_int32),
+                ("kv_lora_rank", ctypes.c_int32), ("qk_nope_dim", ctypes.c_int32),
+                ("rope_dim", ctypes.c_int32), ("v_head_dim", ctypes.c_int32),
+                ("page_size", ctypes.c_int32), ("softmax_scale", ctypes.c_float)]
+
+    @property
+    def row_width(self) -> int:
+        return self.kv_lora_rank + self.num_kv_groups * self.rope_dim
+
+
+def make_dims(num_heads: int, num_kv_groups: int, kv_lora_rank: int, qk_nope_dim: int,
+              rope_dim: int, v_head_dim: int, page_size: int, softmax_scale: float) -> MlaDims:
+    return MlaDims(num_heads, num_kv_groups, kv_lora_rank, qk_nope_dim, rope_dim, v_head_dim,
+                   page_size, softmax_scale)
+
+
+_lib = None
+_P = ctypes.c_void_p
+_I32 = ctypes.c_int32
+_I64 = ctypes.c_int64
+
+
+def lib() -> ctypes.CDLL:
+    """Load libmla.so (raises MlaError when it has not been built)."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(LIB_PATH):
+        raise MlaError(f"{LIB_PATH} is missing: build it with "
+                       "`python -m head_latent_attention_attn_b200.build`")
+    L = ctypes.CDLL(LIB_PATH)
+    D = ctypes.POINTER(MlaDims)
+    L.mla_row_width.argtypes = [D]
+    L.mla_row_width.restype = _I32
+    L.mla_status_string.argtypes = [_I32]
+    L.mla_status_string.restype = ctypes.c_char_p
+    L.mla_cache_append.argtypes = [D, _P, _P, _P, _P, _P, _I32, _P, _I32, _I32, _P, _I64, _P, _P]
+    L.mla_cache_append.restype = _I32
+    L.mla_absorb_q.argtypes = [D, _P, _P, _P, _P, _P, _I64, _I32, _I32, _P, _P]
+    L.mla_absorb_q.restype = _I32
+    L.mla_decode_workspace_size.argtypes = [D, _I32, _I32, _I32, _I32]
+    L.mla_decode_workspace_size.restype = ctypes.c_size_t
+    L.mla_decode_attn.argtypes = [D, _P, _P, _I64, _P, _I32, _P, _I32, _I32, _I32, _I32, _I32,
+                                  _P, ctypes.c_size_t, _P, _P, _P]
+    L.mla_decode_attn.restype = _I32
+    L.mla_out_up.argtypes = [D, _P, _P, _I64, _P, _I32, _P, _P]
+    L.mla_out_up.restype = _I32
+    L.mla_get_device_status.argtypes = [_P, _I32, _P]
+    L.mla_get_device_status.restype = _I32
+    _lib = L
+    return L
+
+
+def _ptr(t: Optional[torch.Tensor]):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream) -> ctypes.c_void_p:
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    if isinstance(stream, torch.cuda.Stream):
+        return ctypes.c_void_p(stream.cuda_stream)
+    return ctypes.c_void_p(int(stream))
+
+
+def _check(status: int, what: str) -> None:
+    if status != MLA_OK:
+        raise MlaError(f"{what}: {STATUS_NAMES.get(status, status)}", status)
+
+
+def _need(t, name: str, dtype, shape=None, cuda: bool = True) -> None:
+    if not isinstance(t, torch.Tensor):
+        raise MlaError(f"{name} must be a torch.Tensor", MLA_ERR_INVALID_ARG)
+    if cuda and t.device.type != "cuda":
+        raise MlaError(f"{name} must be on a CUDA device", MLA_ERR_INVALID_ARG)
+    if t.dtype != dtype:
+        raise MlaError(f"{name} must be {dtype}, got {t.dtype}", MLA_ERR_INVALID_ARG)
+    if not t.is_contiguous():
+        raise MlaError(f"{name} must be contiguous", MLA_ERR_INVALID_ARG)
+    if shape is not None and tuple(t.shape) != tuple(shape):
+        raise MlaError(f"{name} has shape {tuple(t.shape)}, expected {tuple(shape)}",
+                       MLA_ERR_INVALID_ARG)
+
+
+def mla_row_width(dims: MlaDims) -> int:
+    return int(lib().mla_row_width(ctypes.byref(dims)))
+
+
+def mla_cache_append(dims: MlaDims, c_kv, k_r, rope_cos, rope_sin, block_table, start_pos,
+                     cache, dev_error=None, stream=None) -> None:
+    """Write c_kv [B, n, r] and RoPE(k_r [B, n, G, d_r]) into cache [P, ps, D] in place."""
+    B, n = c_kv.shape[0], c_kv.shape[1]
+    G, dr, r = dims.num_kv_groups, dims.rope_dim, dims.kv_lora_rank
+    _need(c_kv, "c_kv", torch.bfloat16, (B, n, r))
+    if dr > 0:
+        _need(k_r, "k_r", torch.bfloat16, (B, n, G, dr))
+        _need(rope_cos, "rope_cos", torch.float32, (B, n, G, dr // 2))
+        _need(rope_sin, "rope_sin", torch.float32, (B, n, G, dr // 2))
+    _need(block_table, "block_table", torch.int32)
+    _need(start_pos, "start_pos", torch.int32, (B,))
+    _need(cache, "cache", torch.bfloat16)
+    if cache.dim() != 3 or cache.shape[1] != dims.page_size or cache.shape[2] != dims.row_width:
+        raise MlaError(f"cache shape {tuple(cache.shape)} does not match dims", MLA_ERR_INVALID_ARG)
+    if block_table.dim() != 2 or block_table.shape[0] != B:
+        raise MlaError("block_table must be [B, max_pages]", MLA_ERR_INVALID_ARG)
+    if dev_error is not None:
+        _need(dev_error, "dev_error", torch.int32)
+    st = lib().mla_cache_append(ctypes.byref(dims), _ptr(c_kv), _ptr(k_r if dr > 0 else None),
+                                _ptr(rope_cos if dr > 0 else None),
+                                _ptr(rope_sin if dr > 0 else None), _ptr(block_table),
+                                block_table.shape[1], _ptr(start_pos), B, n, _ptr(cache),
+                                cache.shape[0], _ptr(dev_error), _stream(stream))
+    _check(st, "mla_cache_append")
+
+
+def mla_absorb_q(dims: MlaDims, q_nope, q_pe, rope_cos, rope_sin, w_uk, q_ext,
+                 w_uk_head_stride: Optional[int] = None, stream=None) -> None:
+    """q_ext [B, q, H, D] = [W_UK^T q_nope ; RoPE(q_pe) in its group's slot, zeros elsewhere]."""
+    B, q = q_nope.shape[0], q_nope.shape[1]
+    H, G, dr = dims.num_heads, dims.num_kv_groups, dims.rope_dim
+    _need(q_nope, "q_nope", torch.bfloat16, (B, q, H, dims.qk_nope_dim))
+    if dr > 0:
+        _need(q_pe, "q_pe", torch.bfloat16, (B, q, H, dr))
+        _need(rope_cos, "rope_cos", torch.float32, (B, q, G, dr // 2))
+        _need(rope_sin, "rope_sin", torch.float32, (B, q, G, dr // 2))
+    _need(q_ext, "q_ext", torch.bfloat16, (B, q, H, dims.row_width))
+    if w_uk_head_stride is None:
+        _need(w_uk, "w_uk", torch.bfloat16, (H, dims.qk_nope_dim, dims.kv_lora_rank))
+        w_uk_head_stride = dims.qk_nope_dim * dims.kv_lora_rank
+    else:
+        _need(w_uk, "w_uk", torch.bfloat16)
+    st = lib().mla_absorb_q(ctypes.byref(dims), _ptr(q_nope), _ptr(q_pe if dr > 0 else None),
+                            _ptr(rope_cos if dr > 0 else None), _ptr(rope_sin if dr > 0 else None),
+                            _ptr(w_uk), int(w_uk_head_stride), B, q, _ptr(q_ext),
+                            _stream(stream))
+    _check(st, "mla_absorb_q")
+
+
+def mla_decode_workspace_size(dims: MlaDims, batch: int, q_len: int, max_seq_len: int,
+                              num_splits: int = 0) -> int:
+    return int(lib().mla_decode_workspace_size(ctypes.byref(dims), batch, q_len, max_seq_len,
+                                               num_splits))
+
+
+def mla_decode_attn(dims: MlaDims, q_ext, cache, block_table, seq_lens, max_seq_len: int,
+                    workspace, o_latent, lse, causal: bool = True, num_splits: int = 0,
+                    stream=None) -> None:
+    """o_latent [B, q, H, r] (bf16) and lse [B, q, H] (fp32) of the absorbed attention."""
+    B, q = q_ext.shape[0], q_ext.shape[1]
+    H, r = dims.num_heads, dims.kv_lora_rank
+    _need(q_ext, "q_ext", torch.bfloat16, (B, q, H, dims.row_width))
+    _need(cache, "cache", torch.bfloat16)
+    if cache.dim() != 3 or cache.shape[1] != dims.page_size or cache.shape[2] != dims.row_width:
+        raise MlaError(f"cache shape {tuple(cache.shape)} does not match dims", MLA_ERR_INVALID_ARG)
+    _need(block_table, "block_table", torch.int32)
+    if block_table.dim() != 2 or block_table.shape[0] != B:
+        raise MlaError("block_table must be [B, max_pages]", MLA_ERR_INVALID_ARG)
+    _need(seq_lens, "seq_lens", torch.int32, (B,))
+    _need(o_latent, "o_latent", torch.bfloat16, (B, q, H, r))
+    _need(lse, "lse", torch.float32, (B, q, H))
+    _need(workspace, "workspace", torch.uint8)
+    st = lib().mla_decode_attn(ctypes.byref(dims), _ptr(q_ext), _ptr(cache), cache.shape[0],
+                               _ptr(block_table), block_table.shape[1], _ptr(seq_lens), B, q,
+                               int(max_seq_len), 1 if causal else 0, int(num_splits),
+                               _ptr(workspace), workspace.numel(), _ptr(o_latent), _ptr(lse),
+                               _stream(stream))
+    _check(st, "mla_decode_attn")
+
+
+def mla_out_up(dims: MlaDims, o_latent, w_uv, o, bias=None,
+               w_uv_head_stride: Optional[int] = None, stream=None) -> None:
+    """o [rows, H, d_v] = W_UV o_latent (+ bias); o_latent is [rows, H, r] (any leading shape)."""
+    H, r, dv = dims.num_heads, dims.kv_lora_rank, dims.v_head_dim
+    _need(o_latent, "o_latent", torch.bfloat16)
+    if o_latent.shape[-2:] != (H, r):
+        raise MlaError("o_latent must end in [H, r]", MLA_ERR_INVALID_ARG)
+    rows = o_latent.numel() // (H * r)
+    _need(o, "o", torch.bfloat16)
+    if o.numel() != rows * H * dv:
+        raise MlaError("o must hold rows * H * d_v elements", MLA_ERR_INVALID_ARG)
+    if w_uv_head_stride is None:
+        _need(w_uv, "w_uv", torch.bfloat16, (H, dv, r))
+        w_uv_head_stride = dv * r
+    else:
+        _need(w_uv, "w_uv", torch.bfloat16)
+    if bias is not None:
+        _need(bias, "bias", torch.bfloat16, (H, dv))
+    st = lib().mla_out_up(ctypes.byref(dims), _ptr(o_latent), _ptr(w_uv), int(w_uv_head_stride),
+                          _ptr(bias), rows, _ptr(o), _stream(stream))
+    _check(st, "mla_out_up")
+
+
+def mla_get_device_status(dev_error, reset: bool = False, stream=None) -> int:
+    """Synchronise and read a device error word (an int32 tensor, or a decode workspace)."""
+    if dev_error.device.type != "cuda":
+        raise MlaError("dev_error must be on a CUDA device", MLA_ERR_INVALID_ARG)
+    return int(lib().mla_get_device_status(_ptr(dev_error), 1 if reset else 0, _stream(stream)))
+
+
+def mla_decode_step(dims: MlaDims, *, c_kv_new, k_r_new, cos_new, sin_new, start_pos,
+                    q_nope, q_pe, cos_q, sin_q, w_uk, w_uv, bias, cache, block_table, seq_lens,
+                    max_seq_len: int, q_ext, workspace, o_latent, lse, o, causal: bool = True,
+                    num_splits: int = 0, stream=None) -> None:
+    """One decode step through the four library calls, on one stream, all buffers given."""
+    mla_cache_append(dims, c_kv_new, k_r_new, cos_new, sin_new, block_table, start_pos, cache,
+                     dev_error=workspace.view(torch.int32)[:1], stream=stream)
+    mla_absorb_q(dims, q_nope, q_pe, cos_q, sin_q, w_uk, q_ext, stream=stream)
+    mla_decode_attn(dims, q_ext, cache, block_table, seq_lens, max_seq_len, workspace, o_latent,
+                    lse, causal=causal, num_splits=num_splits, stream=stream)
+    mla_out_up(dims, o_latent, w_uv, o, bias=bias, stream=stream)
+
+
+__all__ = ["MlaDims", "MlaError", "make_dims", "lib", "mla_row_width", "mla_cache_append",
+           "mla_absorb_q", "mla_decode_workspace_size", "mla_decode_attn", "mla_out_up",
+           "mla_get_device_status", "mla_decode_step", "C_SYMBOLS", "STATUS_NAMES"]

@@ -1,0 +1,358 @@
+// api.cu - the extern "C" boundary of libmla.so (declared in include/mla.h): argument
+// validation, tensor-map encoding and launch planning. No allocation happens here; every
+// buffer is the caller's.
+#include <algorithm>
+#include <cstring>
+
+#include "host_common.h"
+#include "kernels.h"
+
+using namespace mla;
+
+namespace {
+
+constexpr int kMaxSmem = 232448;  // 227 KB opt-in dynamic shared memory per CTA
+
+inline cudaStream_t as_stream(void* s) { return reinterpret_cast<cudaStream_t>(s); }
+
+int num_sms() {
+  int dev = 0, n = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess ||
+      cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) {
+    cudaGetLastError();
+    return 148;
+  }
+  return n;
+}
+
+int pow2_at_least(int x, int lo) {
+  int v = lo;
+  while (v < x) v <<= 1;
+  return v;
+}
+
+// Launch geometry of one mla_decode_attn problem.
+struct DecodePlan {
+  int ncol, col_groups, nblk, nch, slot_blocks, nslot, npt, tmem_cols, splits, tiles_per_split;
+  size_t smem;
+  size_t ws_bytes;
+  size_t part_lse_off, part_o_off;
+};
+
+mla_status plan_decode(const mla_dims* d, int32_t batch, int32_t q_len, int32_t max_seq_len,
+                       int32_t num_splits, DecodePlan* P) {
+  mla_status st = check_dims(d);
+  if (st != MLA_OK) return st;
+  if (batch < 0 || q_len <= 0 || max_seq_len < q_len || num_splits < 0)
+    return MLA_ERR_INVALID_ARG;
+  if (d->page_size != kDecodeTok) return MLA_ERR_UNSUPPORTED;
+  const int r = d->kv_lora_rank;
+  const int D = row_width(d);
+  if (r > 512 || D > 64 * kDecodeMaxBlk) return MLA_ERR_UNSUPPORTED;
+  const int64_t qH = int64_t(q_len) * d->num_heads;
+  if (qH > 64 * 65535) return MLA_ERR_UNSUPPORTED;
+  P->ncol = qH <= 16 ? 16 : (qH <= 32 ? 32 : 64);
+  P->col_groups = int((qH + P->ncol - 1) / P->ncol);
+  P->nblk = (D + 63) / 64;
+  P->nch = (r + 127) / 128;
+  P->slot_blocks = std::max(P->nblk, 2 * P->nch);
+  P->tmem_cols = pow2_at_least((2 + P->nch) * P->ncol, 32);
+  if (P->tmem_cols > 512) return MLA_ERR_UNSUPPORTED;
+  // Most cache slots that fit, preferring two P^T buffers; at least two slots.
+  P->nslot = 0;
+  for (int npt = 2; npt >= 1 && P->nslot == 0; --npt) {
+    for (int ns = kDecodeMaxSlots; ns >= 2; --ns) {
+      if (decode_smem_bytes(P->ncol, P->nblk, P->slot_blocks, ns, npt) <= size_t(kMaxSmem)) {
+        P->nslot = ns;
+        P->npt = npt;
+        break;
+      }
+    }
+  }
+  if (P->nslot < 2) return MLA_ERR_UNSUPPORTED;
+  P->smem = decode_smem_bytes(P->ncol, P->nblk, P->slot_blocks, P->nslot, P->npt);
+  const int max_tiles = (max_seq_len + kDecodeTok - 1) / kDecodeTok;
+  const int64_t units = int64_t(std::max(batch, 1)) * P->col_groups;
+  int S = num_splits;
+  if (S == 0) {
+    const int sms = num_sms();
+    S = units >= sms ? 1 : int(sms / units);
+  }
+  S = std::max(1, std::min(S, max_tiles));
+  P->tiles_per_split = (max_tiles + S - 1) / S;
+  S = (max_tiles + P->tiles_per_split - 1) / P->tiles_per_split;  // drop empty splits
+  if (S > 65535) return MLA_ERR_UNSUPPORTED;
+  P->splits = S;
+  size_t off = 256;  // device error word + padding
+  P->part_lse_off = off;
+  P->part_o_off = off;
+  if (S > 1) {
+    const size_t rows = size_t(std::max(batch, 1)) * P->col_groups * S * P->ncol;
+    off += (rows * sizeof(float) + 255) / 256 * 256;
+    P->part_o_off = off;
+    off += rows * size_t(r) * sizeof(float);
+  }
+  P->ws_bytes = off;
+  return MLA_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+int32_t mla_row_width(const mla_dims* dims) {
+  if (check_dims(dims) != MLA_OK) return -1;
+  return row_width(dims);
+}
+
+const char* mla_status_string(mla_status s) {
+  switch (s) {
+    case MLA_OK: return "MLA_OK";
+    case MLA_ERR_INVALID_ARG: return "MLA_ERR_INVALID_ARG";
+    case MLA_ERR_UNSUPPORTED: return "MLA_ERR_UNSUPPORTED";
+    case MLA_ERR_WORKSPACE: return "MLA_ERR_WORKSPACE";
+    case MLA_ERR_CUDA: return "MLA_ERR_CUDA";
+    case MLA_ERR_DEVICE_BOUNDS: return "MLA_ERR_DEVICE_BOUNDS";
+    case MLA_ERR_DEVICE_TIMEOUT: return "MLA_ERR_DEVICE_TIMEOUT";
+  }
+  return "MLA_ERR_UNKNOWN";
+}
+
+mla_status mla_cache_append(const mla_dims* dims, const void* c_kv, const void* k_r,
+                            const float* rope_cos, const float* rope_sin,
+                            const int32_t* block_table, int32_t max_pages_per_seq,
+                            const int32_t* start_pos, int32_t batch, int32_t n_new, void* cache,
+                            int64_t num_pages, int32_t* dev_error, void* stream) {
+  mla_status st = check_dims(dims);
+  if (st != MLA_OK) return st;
+  if (batch < 0 || n_new < 0 || max_pages_per_seq <= 0 || num_pages <= 0 ||
+      num_pages > INT32_MAX)
+    return MLA_ERR_INVALID_ARG;
+  if (batch == 0 || n_new == 0) return MLA_OK;
+  if (!c_kv || !block_table || !start_pos || !cache) return MLA_ERR_INVALID_ARG;
+  if (dims->rope_dim > 0 && (!k_r || !rope_cos || !rope_sin)) return MLA_ERR_INVALID_ARG;
+  if (!aligned(c_kv, 16) || !aligned(cache, 16)) return MLA_ERR_INVALID_ARG;
+  AppendParams p{};
+  p.c_kv = static_cast<const uint16_t*>(c_kv);
+  p.k_r = static_cast<const uint16_t*>(k_r);
+  p.rope_cos = rope_cos;
+  p.rope_sin = rope_sin;
+  p.block_table = block_table;
+  p.start_pos = start_pos;
+  p.cache = static_cast<uint16_t*>(cache);
+  p.dev_error = dev_error;
+  p.num_pages = num_pages;
+  p.max_pages = max_pages_per_seq;
+  p.batch = batch;
+  p.n_new = n_new;
+  p.r = dims->kv_lora_rank;
+  p.groups = dims->num_kv_groups;
+  p.rope_dim = dims->rope_dim;
+  p.page_size = dims->page_size;
+  return launch_cache_append(p, as_stream(stream)) == cudaSuccess ? MLA_OK : MLA_ERR_CUDA;
+}
+
+static int pick_nr(int64_t rows) {
+  return rows <= 16 ? 16 : rows <= 32 ? 32 : rows <= 64 ? 64 : 128;
+}
+
+mla_status mla_absorb_q(const mla_dims* dims, const void* q_nope, const void* q_pe,
+                        const float* rope_cos, const float* rope_sin, const void* w_uk,
+                        int64_t w_uk_head_stride, int32_t batch, int32_t q_len, void* q_ext,
+                        void* stream) {
+  mla_status st = check_dims(dims);
+  if (st != MLA_OK) return st;
+  if (batch < 0 || q_len <= 0) return MLA_ERR_INVALID_ARG;
+  if (batch == 0) return MLA_OK;
+  const int H = dims->num_heads, r = dims->kv_lora_rank, dn = dims->qk_nope_dim;
+  if (!q_nope || !w_uk || !q_ext) return MLA_ERR_INVALID_ARG;
+  if (dims->rope_dim > 0 && (!q_pe || !rope_cos || !rope_sin)) return MLA_ERR_INVALID_ARG;
+  if (w_uk_head_stride < int64_t(dn) * r || w_uk_head_stride % 8 != 0) return MLA_ERR_INVALID_ARG;
+  if (!aligned(q_nope, 16) || !aligned(w_uk, 16) || !aligned(q_ext, 16)) return MLA_ERR_INVALID_ARG;
+  const int64_t rows = int64_t(batch) * q_len;
+  if (rows > int64_t(65535) * 128) return MLA_ERR_UNSUPPORTED;
+  const int D = row_width(dims);
+  WGemmParams p{};
+  {
+    const uint64_t dims3[3] = {uint64_t(r), uint64_t(dn), uint64_t(H)};
+    const uint64_t str[2] = {uint64_t(r) * 2, uint64_t(w_uk_head_stride) * 2};
+    const uint32_t box[3] = {64, 64, 1};
+    if (!encode_bf16_map(&p.tm_w, w_uk, 3, dims3, str, box, CU_TENSOR_MAP_SWIZZLE_128B))
+      return MLA_ERR_CUDA;
+  }
+  const int nr = pick_nr(rows);
+  {
+    const uint64_t dims3[3] = {uint64_t(dn), uint64_t(H), uint64_t(rows)};
+    const uint64_t str[2] = {uint64_t(dn) * 2, uint64_t(H) * dn * 2};
+    const uint32_t box[3] = {64, 1, uint32_t(nr)};
+    if (!encode_bf16_map(&p.tm_x, q_nope, 3, dims3, str, box, CU_TENSOR_MAP_SWIZZLE_128B))
+      return MLA_ERR_CUDA;
+  }
+  p.out = static_cast<uint16_t*>(q_ext);
+  p.out_row_stride = int64_t(H) * D;
+  p.out_head_stride = D;
+  p.bias = nullptr;
+  p.dev_error = nullptr;
+  p.M = r;
+  p.K = dn;
+  p.rows = int32_t(rows);
+  p.heads = H;
+  p.a_mn = 1;
+  p.q_pe = dims->rope_dim > 0 ? static_cast<const uint16_t*>(q_pe) : nullptr;
+  p.rope_cos = rope_cos;
+  p.rope_sin = rope_sin;
+  p.groups = dims->num_kv_groups;
+  p.rope_dim = dims->rope_dim;
+  return launch_wgemm(p, nr, as_stream(stream)) == cudaSuccess ? MLA_OK : MLA_ERR_CUDA;
+}
+
+mla_status mla_out_up(const mla_dims* dims, const void* o_latent, const void* w_uv,
+                      int64_t w_uv_head_stride, const void* bias, int32_t rows, void* o,
+                      void* stream) {
+  mla_status st = check_dims(dims);
+  if (st != MLA_OK) return st;
+  if (rows < 0) return MLA_ERR_INVALID_ARG;
+  if (rows == 0) return MLA_OK;
+  const int H = dims->num_heads, r = dims->kv_lora_rank, dv = dims->v_head_dim;
+  if (!o_latent || !w_uv || !o) return MLA_ERR_INVALID_ARG;
+  if (w_uv_head_stride < int64_t(dv) * r || w_uv_head_stride % 8 != 0) return MLA_ERR_INVALID_ARG;
+  if (!aligned(o_latent, 16) || !aligned(w_uv, 16) || !aligned(o, 16)) return MLA_ERR_INVALID_ARG;
+  if (int64_t(rows) > int64_t(65535) * 128) return MLA_ERR_UNSUPPORTED;
+  WGemmParams p{};
+  {
+    const uint64_t dims3[3] = {uint64_t(r), uint64_t(dv), uint64_t(H)};
+    const uint64_t str[2] = {uint64_t(r) * 2, uint64_t(w_uv_head_stride) * 2};
+    const uint32_t box[3] = {64, 128, 1};
+    if (!encode_bf16_map(&p.tm_w, w_uv, 3, dims3, str, box, CU_TENSOR_MAP_SWIZZLE_128B))
+      return MLA_ERR_CUDA;
+  }
+  const int nr = pick_nr(rows);
+  {
+    const uint64_t dims3[3] = {uint64_t(r), uint64_t(H), uint64_t(rows)};
+    const uint64_t str[2] = {uint64_t(r) * 2, uint64_t(H) * r * 2};
+    const uint32_t box[3] = {64, 1, uint32_t(nr)};
+    if (!encode_bf16_map(&p.tm_x, o_latent, 3, dims3, str, box, CU_TENSOR_MAP_SWIZZLE_128B))
+      return MLA_ERR_CUDA;
+  }
+  p.out = static_cast<uint16_t*>(o);
+  p.out_row_stride = int64_t(H) * dv;
+  p.out_head_stride = dv;
+  p.bias = static_cast<const uint16_t*>(bias);
+  p.dev_error = nullptr;
+  p.M = dv;
+  p.K = r;
+  p.rows = rows;
+  p.heads = H;
+  p.a_mn = 0;
+  p.q_pe = nullptr;
+  return launch_wgemm(p, nr, as_stream(stream)) == cudaSuccess ? MLA_OK : MLA_ERR_CUDA;
+}
+
+size_t mla_decode_workspace_size(const mla_dims* dims, int32_t batch, int32_t q_len,
+                                 int32_t max_seq_len, int32_t num_splits) {
+  DecodePlan P;
+  if (plan_decode(dims, batch, q_len, max_seq_len, num_splits, &P) != MLA_OK) return 0;
+  return P.ws_bytes;
+}
+
+mla_status mla_decode_attn(const mla_dims* dims, const void* q_ext, const void* cache,
+                           int64_t num_pages, const int32_t* block_table,
+                           int32_t max_pages_per_seq, const int32_t* seq_lens, int32_t batch,
+                           int32_t q_len, int32_t max_seq_len, int32_t causal,
+                           int32_t num_splits, void* workspace, size_t workspace_bytes,
+                           void* o_latent, float* lse, void* stream) {
+  DecodePlan P;
+  mla_status st = plan_decode(dims, batch, q_len, max_seq_len, num_splits, &P);
+  if (st != MLA_OK) return st;
+  if (num_pages <= 0 || num_pages * kDecodeTok > (int64_t(1) << 31) || max_pages_per_seq <= 0 ||
+      (causal != 0 && causal != 1))
+    return MLA_ERR_INVALID_ARG;
+  if (batch == 0) return MLA_OK;
+  if (!q_ext || !cache || !block_table || !seq_lens || !o_latent || !lse)
+    return MLA_ERR_INVALID_ARG;
+  if (!aligned(q_ext, 16) || !aligned(cache, 16)) return MLA_ERR_INVALID_ARG;
+  if (!workspace || !aligned(workspace, 256)) return MLA_ERR_WORKSPACE;
+  if (workspace_bytes < P.ws_bytes) return MLA_ERR_WORKSPACE;
+  const int D = row_width(dims);
+  const int64_t qH = int64_t(q_len) * dims->num_heads;
+  DecodeParams p{};
+  {
+    const uint64_t d2[2] = {uint64_t(D), uint64_t(num_pages) * kDecodeTok};
+    const uint64_t s2[1] = {uint64_t(D) * 2};
+    const uint32_t box[2] = {64, uint32_t(kDecodeTok)};
+    if (!encode_bf16_map(&p.tm_cache, cache, 2, d2, s2, box, CU_TENSOR_MAP_SWIZZLE_128B))
+      return MLA_ERR_CUDA;
+  }
+  {
+    const uint64_t d3[3] = {uint64_t(D), uint64_t(qH), uint64_t(batch)};
+    const uint64_t s3[2] = {uint64_t(D) * 2, uint64_t(qH) * D * 2};
+    const uint32_t box[3] = {64, uint32_t(P.ncol), 1};
+    if (!encode_bf16_map(&p.tm_q, q_ext, 3, d3, s3, box, CU_TENSOR_MAP_SWIZZLE_128B))
+      return MLA_ERR_CUDA;
+  }
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  p.block_table = block_table;
+  p.seq_lens = seq_lens;
+  p.o_latent = static_cast<uint16_t*>(o_latent);
+  p.lse = lse;
+  p.part_lse = reinterpret_cast<float*>(ws + P.part_lse_off);
+  p.part_o = reinterpret_cast<float*>(ws + P.part_o_off);
+  p.dev_error = reinterpret_cast<int32_t*>(ws);
+  p.num_pages = num_pages;
+  p.max_pages = max_pages_per_seq;
+  p.batch = batch;
+  p.q_len = q_len;
+  p.num_heads = dims->num_heads;
+  p.qH = int32_t(qH);
+  p.r = dims->kv_lora_rank;
+  p.D = D;
+  p.nblk = P.nblk;
+  p.nch = P.nch;
+  p.col_groups = P.col_groups;
+  p.splits = P.splits;
+  p.tiles_per_split = P.tiles_per_split;
+  p.max_seq_len = max_seq_len;
+  p.causal = causal;
+  p.nslot = P.nslot;
+  p.slot_blocks = P.slot_blocks;
+  p.tmem_cols = P.tmem_cols;
+  p.npt = P.npt;
+  p.scale_log2 = dims->softmax_scale * 1.4426950408889634f;
+  const dim3 grid(P.splits, P.col_groups, batch);
+  cudaStream_t s = as_stream(stream);
+  if (launch_decode(p, P.ncol, grid, P.smem, s) != cudaSuccess) return MLA_ERR_CUDA;
+  if (P.splits > 1) {
+    CombineParams c{};
+    c.part_o = p.part_o;
+    c.part_lse = p.part_lse;
+    c.o_latent = p.o_latent;
+    c.lse = lse;
+    c.batch = batch;
+    c.qH = int32_t(qH);
+    c.r = p.r;
+    c.ncol = P.ncol;
+    c.col_groups = P.col_groups;
+    c.splits = P.splits;
+    if (launch_combine(c, s) != cudaSuccess) return MLA_ERR_CUDA;
+  }
+  return MLA_OK;
+}
+
+mla_status mla_get_device_status(const int32_t* dev_error, int32_t reset, void* stream) {
+  if (!dev_error) return MLA_ERR_INVALID_ARG;
+  cudaStream_t s = as_stream(stream);
+  int32_t v = 0;
+  if (cudaMemcpyAsync(&v, dev_error, sizeof(v), cudaMemcpyDeviceToHost, s) != cudaSuccess ||
+      cudaStreamSynchronize(s) != cudaSuccess)
+    return MLA_ERR_CUDA;
+  if (reset) {
+    if (cudaMemsetAsync(const_cast<int32_t*>(dev_error), 0, sizeof(int32_t), s) != cudaSuccess ||
+        cudaStreamSynchronize(s) != cudaSuccess)
+      return MLA_ERR_CUDA;
+  }
+  if (v & MLA_DEVERR_TIMEOUT) return MLA_ERR_DEVICE_TIMEOUT;
+  if (v & MLA_DEVERR_BOUNDS) return MLA_ERR_DEVICE_BOUNDS;
+  return MLA_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,78 @@
+// kernels.h - parameter blocks and launchers of the sm_100a kernels behind the C ABI.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace mla {
+
+// ---- mla_cache_append -------------------------------------------------------------------
+struct AppendParams {
+  const uint16_t* c_kv;      // [B, n_new, r]
+  const uint16_t* k_r;       // [B, n_new, G, d_r]
+  const float* rope_cos;     // [B, n_new, G, d_r/2]
+  const float* rope_sin;
+  const int32_t* block_table;
+  const int32_t* start_pos;
+  uint16_t* cache;           // [num_pages, ps, D]
+  int32_t* dev_error;
+  int64_t num_pages;
+  int32_t max_pages, batch, n_new, r, groups, rope_dim, page_size;
+};
+cudaError_t launch_cache_append(const AppendParams& p, cudaStream_t stream);
+
+// ---- per-head weight GEMM (mla_absorb_q, mla_out_up) --------------------------------------
+// For every head h and activation row n: out[n, h, m] = sum_k W_h[m, k] * x[n, h, k] (+ bias).
+// The weight tile is the UMMA A operand (M = output features), the activation rows are B.
+struct WGemmParams {
+  CUtensorMap tm_w;          // 3D weight map, box 128 x 64 (see launcher)
+  CUtensorMap tm_x;          // 3D activations {K, H, rows}, box {64, 1, NR}
+  uint16_t* out;             // element (n, h, m) at n*out_row_stride + h*out_head_stride + m
+  int64_t out_row_stride, out_head_stride;
+  const uint16_t* bias;      // [H, M] or null
+  int32_t* dev_error;
+  int32_t M, K, rows, heads;
+  int32_t a_mn;              // 1: weight stored [K][M] (W_UK), 0: stored [M][K] (W_UV)
+  // rotary part of q_ext (mla_absorb_q only; q_pe == nullptr otherwise)
+  const uint16_t* q_pe;      // [rows, H, d_r]
+  const float* rope_cos;     // [rows, G, d_r/2]
+  const float* rope_sin;
+  int32_t groups, rope_dim;
+};
+cudaError_t launch_wgemm(const WGemmParams& p, int nr, cudaStream_t stream);
+
+// ---- mla_decode_attn -----------------------------------------------------------------------
+constexpr int kDecodeTok = 64;        // tokens per tile = one cache page
+constexpr int kDecodeMaxBlk = 10;     // D <= 640 -> at most 10 64-column blocks
+constexpr int kDecodeMaxSlots = 8;
+
+struct DecodeParams {
+  CUtensorMap tm_cache;      // 2D {D, num_pages*64}, box {64, 64}, 128B swizzle
+  CUtensorMap tm_q;          // 3D {D, q*H, B}, box {64, NCOL, 1}, 128B swizzle
+  const int32_t* block_table;
+  const int32_t* seq_lens;
+  uint16_t* o_latent;        // [B, q, H, r]
+  float* lse;                // [B, q, H]
+  float* part_o;             // [B, CG, S, NCOL, r]  (splits > 1)
+  float* part_lse;           // [B, CG, S, NCOL]
+  int32_t* dev_error;
+  int64_t num_pages;
+  int32_t max_pages, batch, q_len, num_heads, qH, r, D, nblk, nch, col_groups, splits,
+      tiles_per_split, max_seq_len, causal, nslot, slot_blocks, tmem_cols, npt;
+  float scale_log2;          // softmax_scale * log2(e)
+};
+size_t decode_smem_bytes(int ncol, int nblk, int slot_blocks, int nslot, int npt);
+cudaError_t launch_decode(const DecodeParams& p, int ncol, dim3 grid, size_t smem,
+                          cudaStream_t stream);
+
+struct CombineParams {
+  const float* part_o;
+  const float* part_lse;
+  uint16_t* o_latent;
+  float* lse;
+  int32_t batch, qH, r, ncol, col_groups, splits;
+};
+cudaError_t launch_combine(const CombineParams& p, cudaStream_t stream);
+
+}  // namespace mla

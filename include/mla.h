@@ -1,0 +1,193 @@
+/*
+ * mla.h - C ABI of the B200 (sm_100a) weight-absorbed MLA decode library (libmla.so).
+ *
+ * The library computes one decode step of Multi-head Latent Attention over a paged
+ * cache that holds, per token, only the rank-r latent c_kv and the rotated RoPE key
+ * of every key group. The four compute calls follow the absorbed order of the
+ * DeepSeek-V2 MLA page (dtcms.com, "Matrix absorption" section):
+ *
+ *   mla_cache_append  write c_kv and RoPE(k_r) of new tokens into the paged cache
+ *   mla_absorb_q      q_c = einsum('hdc,bhqd->bhqc', W_UK, q_nope), RoPE(q_pe) -> q_ext
+ *   mla_decode_attn   scores = q_pe.k_pe + q_c.c_kv, scaled, softmaxed;
+ *                     o_ = einsum('bhql,blc->bhqc', attn, c_kv)   (einsum 4) and lse
+ *   mla_out_up        o = einsum('bhqc,hdc->bhqd', o_, W_UV) (+ bias)  (einsum 5)
+ *
+ * Conventions shared by every call
+ *   - Every data pointer is DEVICE memory owned by the caller; the library allocates
+ *     nothing and keeps no state between calls, so concurrent calls on different
+ *     streams are safe as long as their output buffers differ.
+ *   - bf16 tensors are passed as void* (uint16 storage), contiguous, row-major, in the
+ *     shapes given below; fp32 and int32 tensors likewise.
+ *   - Calls are asynchronous on `stream` (a cudaStream_t / CUstream; NULL = the legacy
+ *     default stream). The returned status covers host-side argument validation and
+ *     launch errors only; nothing is launched when validation fails.
+ *   - Faults the device detects (a page id outside [0, num_pages), a context length
+ *     outside the bounds the call was planned for, a pipeline wait that ran out) set
+ *     bits in a caller-owned int32 "device error word"; read it with
+ *     mla_get_device_status. Kernels only OR bits into the word, never clear it.
+ *
+ * Shapes use: B batch, q query tokens per sequence, H query heads, G key groups
+ * (1 = one k_pe shared by all heads), r = kv_lora_rank, d_n = qk_nope_dim,
+ * d_r = rope_dim per group, d_v = v_head_dim, ps = page_size, D = r + G*d_r the
+ * cache row width. Head h uses key group g(h) = h / (H / G).
+ */
+#ifndef MLA_H_
+#define MLA_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum mla_status {
+  MLA_OK = 0,
+  MLA_ERR_INVALID_ARG = 1,    /* null pointer, bad size, inconsistent dims          */
+  MLA_ERR_UNSUPPORTED = 2,    /* valid but not implemented shape (never a fallback) */
+  MLA_ERR_WORKSPACE = 3,      /* workspace missing or smaller than required         */
+  MLA_ERR_CUDA = 4,           /* a CUDA runtime/driver call failed                   */
+  MLA_ERR_DEVICE_BOUNDS = 5,  /* device saw an out-of-range page id or length        */
+  MLA_ERR_DEVICE_TIMEOUT = 6  /* a device pipeline wait exceeded its limit           */
+} mla_status;
+
+/* Bits a kernel ORs into the device error word. */
+#define MLA_DEVERR_BOUNDS (1 << 0)
+#define MLA_DEVERR_TIMEOUT (1 << 1)
+
+typedef struct mla_dims {
+  int32_t num_heads;     /* H                                                    */
+  int32_t num_kv_groups; /* G, divides H                                         */
+  int32_t kv_lora_rank;  /* r, multiple of 8                                     */
+  int32_t qk_nope_dim;   /* d_n, multiple of 8                                   */
+  int32_t rope_dim;      /* d_r per group, even (0 allowed)                      */
+  int32_t v_head_dim;    /* d_v, multiple of 8                                   */
+  int32_t page_size;     /* tokens per cache page                                */
+  float softmax_scale;   /* multiplies q.k before the softmax                    */
+} mla_dims;
+
+/* Cache row width D = r + G*d_r, or -1 when `dims` is null or inconsistent. */
+int32_t mla_row_width(const mla_dims* dims);
+
+/* Human-readable name of a status code (static string). */
+const char* mla_status_string(mla_status status);
+
+/*
+ * mla_cache_append - write n_new tokens per sequence into the paged latent cache.
+ *
+ * Defined by the MLAfication data flow (wzjinhao.cn page: the KV cache stores only
+ * c_kv plus the low-dimensional rotary key) and the row layout
+ * torch.split(compressed_kv, [kv_lora_rank, qk_rope_head_dim]) of the DeepSeek-V2 page;
+ * the cached key is post-RoPE, as only q_pe is rotated at attention time there.
+ *
+ *   c_kv        bf16 [B, n_new, r]          latent of each new token (copied bit-exactly)
+ *   k_r         bf16 [B, n_new, G, d_r]     unrotated rotary key of each new token
+ *   rope_cos/sin fp32 [B, n_new, G, d_r/2]  cos/sin of each pair's angle at the token's
+ *                                           position; pair j is (x_j, x_{j+d_r/2})
+ *   block_table int32 [B, max_pages_per_seq] physical page of each logical page
+ *   start_pos   int32 [B]                   position of the first new token
+ *   cache       bf16 [num_pages, ps, D]     updated in place
+ *   dev_error   int32 device error word (may be NULL: faults are then only skipped)
+ *
+ * Token t of sequence b at position p = start_pos[b] + t goes to page
+ * block_table[b][p / ps], row p % ps: cache[.., 0:r] = c_kv and, for each group g,
+ * cache[.., r + g*d_r ...] = bf16_rne(x0*c - x1*s | x1*c + x0*s) with every product
+ * and sum rounded to fp32 separately. A page id outside [0, num_pages) or a logical
+ * page outside the table sets MLA_DEVERR_BOUNDS and that token is skipped.
+ */
+mla_status mla_cache_append(const mla_dims* dims, const void* c_kv, const void* k_r,
+                            const float* rope_cos, const float* rope_sin,
+                            const int32_t* block_table, int32_t max_pages_per_seq,
+                            const int32_t* start_pos, int32_t batch, int32_t n_new,
+                            void* cache, int64_t num_pages, int32_t* dev_error,
+                            void* stream);
+
+/*
+ * mla_absorb_q - fold W_UK into the query and rotate its RoPE part.
+ *
+ * The "W^{UK} is absorbed by q_nope" step of the DeepSeek-V2 page:
+ * q_c = einsum('hdc,bhqd->bhqc', q_absorb, q_nope), and q_pe = apply_rotary_pos_emb
+ * at the query positions.
+ *
+ *   q_nope      bf16 [B, q, H, d_n]
+ *   q_pe        bf16 [B, q, H, d_r]         unrotated
+ *   rope_cos/sin fp32 [B, q, G, d_r/2]      angles at each query row's position
+ *   w_uk        bf16, head h at w_uk + h*w_uk_head_stride (elements), each [d_n, r]
+ *               row-major; w_uk_head_stride >= d_n*r, multiple of 8 (a packed
+ *               kv_b_proj view [H, d_n + d_v, r] passes stride (d_n + d_v)*r)
+ *   q_ext       bf16 [B, q, H, D] output:   [0:r) = q_c (fp32 accumulate, bf16 round),
+ *               [r + g(h)*d_r, +d_r) = RoPE(q_pe) (fp32, bf16 round), other groups 0
+ */
+mla_status mla_absorb_q(const mla_dims* dims, const void* q_nope, const void* q_pe,
+                        const float* rope_cos, const float* rope_sin, const void* w_uk,
+                        int64_t w_uk_head_stride, int32_t batch, int32_t q_len, void* q_ext,
+                        void* stream);
+
+/*
+ * Bytes of workspace mla_decode_attn needs for this problem (0 on invalid input).
+ * num_splits: KV splits per sequence, 0 = let the library choose. The first 256 bytes
+ * of the workspace hold the device error word (int32 at offset 0): zero them once
+ * after allocating. The rest is scratch the library overwrites on every call.
+ */
+size_t mla_decode_workspace_size(const mla_dims* dims, int32_t batch, int32_t q_len,
+                                 int32_t max_seq_len, int32_t num_splits);
+
+/*
+ * mla_decode_attn - paged, split-KV absorbed attention over the latent cache.
+ *
+ * For sequence b with context length L = seq_lens[b] (after the append) and query row
+ * i at position L - q + i, every head h scores each visible token l (l <= L - q + i
+ * when causal != 0, else every l < L):
+ *     s = softmax_scale * (q_ext[b,i,h,:] . cache_row(b, l))
+ * (the q_pe.k_pe + q_c.c_kv of the DeepSeek-V2 page, since q_ext zero-pads the other
+ * groups' rotary slots), p = softmax over l, and writes
+ *     o_latent[b,i,h,:] = sum_l p * c_kv[l]      (einsum 4, bf16)
+ *     lse[b,i,h]        = ln sum_l exp(s)        (fp32)
+ * Long contexts are split across CTAs; the per-split results are merged with the
+ * log-sum-exp identity.
+ *
+ *   q_ext       bf16 [B, q, H, D]   from mla_absorb_q
+ *   cache       bf16 [num_pages, ps, D]
+ *   block_table int32 [B, max_pages_per_seq]
+ *   seq_lens    int32 [B], each in [q, max_seq_len] and <= max_pages_per_seq*ps
+ *   max_seq_len host-side upper bound of seq_lens, used to plan the splits
+ *   o_latent    bf16 [B, q, H, r] output; lse fp32 [B, q, H] output
+ *   workspace   >= mla_decode_workspace_size(...) bytes, 256-byte aligned
+ * Supported: ps == 64, H*q rows split in groups of <= 64 per CTA, r <= 512,
+ * D <= 640. Others return MLA_ERR_UNSUPPORTED.
+ */
+mla_status mla_decode_attn(const mla_dims* dims, const void* q_ext, const void* cache,
+                           int64_t num_pages, const int32_t* block_table,
+                           int32_t max_pages_per_seq, const int32_t* seq_lens, int32_t batch,
+                           int32_t q_len, int32_t max_seq_len, int32_t causal,
+                           int32_t num_splits, void* workspace, size_t workspace_bytes,
+                           void* o_latent, float* lse, void* stream);
+
+/*
+ * mla_out_up - apply the value up-projection to the attention output (einsum 5 of the
+ * DeepSeek-V2 page, o = einsum('bhqc,hdc->bhqd', o_, W_UV)), plus the optional up_v
+ * bias of the MLAfied checkpoints (wzjinhao.cn page). Exact under absorption because
+ * softmax weights sum to one.
+ *
+ *   o_latent  bf16 [rows, H, r]   rows = B*q
+ *   w_uv      bf16, head h at w_uv + h*w_uv_head_stride (elements), each [d_v, r]
+ *   bias      bf16 [H, d_v] or NULL
+ *   o         bf16 [rows, H, d_v] output (fp32 accumulate)
+ */
+mla_status mla_out_up(const mla_dims* dims, const void* o_latent, const void* w_uv,
+                      int64_t w_uv_head_stride, const void* bias, int32_t rows, void* o,
+                      void* stream);
+
+/*
+ * Synchronise `stream`, read the device error word at `dev_error` and, if reset != 0,
+ * clear it. Returns MLA_ERR_DEVICE_TIMEOUT, MLA_ERR_DEVICE_BOUNDS or MLA_OK (or
+ * MLA_ERR_CUDA if the read fails). For mla_decode_attn the word is the first int32
+ * of its workspace.
+ */
+mla_status mla_get_device_status(const int32_t* dev_error, int32_t reset, void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MLA_H_ */

@@ -14,6 +14,8 @@ What it computes, and where the pages define it
   section). The absorbed kernels reach the same result by associativity (einsums (4)-(5)
   of that section), so this plain definition is the reference for them.
   It also returns o_latent = sum_l p_l c_kv[l], the intermediate of einsum (4).
+* ``absorb_reference`` / ``out_up_reference``: the absorb einsum and einsum (5) on their
+  own, for checking the two projection steps separately.
 * ``rope_rotate``: RoPE on a rotary slice, pairs (x_j, x_{j+d/2}) rotated by theta_j * pos
   (the rotate-half convention of ``apply_rotary_pos_emb`` used on that page), angles in fp64.
 * ``cache_append_emulate``: the byte-exact result of writing new tokens into the paged
@@ -137,6 +139,29 @@ def mla_decode_reference(q_nope, q_pe, c_kv, k_r, w_uk, w_uv, bias, theta, q_pos
     if want_p:
         out["p"] = p_all
     return out
+
+
+def absorb_reference(q_nope, q_pe, w_uk, theta, q_pos, num_groups: int):
+    """Absorb step in fp64: q_c = einsum('hdc,ihd->ihc', W_UK, q_nope) (the q_absorb einsum
+    of the "Matrix absorption" listing) and the rotated q_pe of each head at its row's
+    position. q_nope [q, H, d_n], q_pe [q, H, d_r] -> (q_c [q, H, r], q_rot [q, H, d_r])."""
+    q_nope, q_pe, w_uk = as_f64(q_nope), as_f64(q_pe), as_f64(w_uk)
+    H = w_uk.shape[0]
+    g_of = group_of_head(H, num_groups)
+    q_c = np.einsum("hdc,ihd->ihc", w_uk, q_nope)
+    q_rot = np.empty_like(q_pe)
+    for h in range(H):
+        q_rot[:, h, :] = rope_rotate(q_pe[:, h, :], np.asarray(theta)[g_of[h]], np.asarray(q_pos))
+    return q_c, q_rot
+
+
+def out_up_reference(o_latent, w_uv, bias=None):
+    """Einsum (5) of the "Matrix absorption" section, o = einsum('ihc,hdc->ihd', o_, W_UV),
+    plus the optional up_v bias. o_latent [..., H, r] -> [..., H, d_v]."""
+    o = np.einsum("...hc,hdc->...hd", as_f64(o_latent), as_f64(w_uv))
+    if bias is not None:
+        o = o + as_f64(bias)
+    return o
 
 
 # ----------------------------------------------------------------------------------------

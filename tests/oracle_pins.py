@@ -355,6 +355,26 @@ def pin_append_slots(O):
                         "rotated key within bf16 rounding"
 
 
-ALL_PINS = [pin_bruteforce, pin_associativity, pin_sdpa_identity_weights, pin_zero_query_uniform,
+def pin_absorb_single_token(O):
+    """With one cached token lse = s_0; the absorbed score from absorb_reference must equal it."""
+    P = _problem(101, nq=2, H=4, G=2, r=6, dn=3, dr=4, dv=2, L=1)
+    P["q_pos"] = np.array([0, 0])
+    got = O.mla_decode_reference(**P, causal=False)
+    q_c, q_rot = O.absorb_reference(P["q_nope"], P["q_pe"], P["w_uk"], P["theta"], P["q_pos"], 2)
+    g_of = np.arange(4) // 2
+    k_rot = np.stack([O.rope_rotate(P["k_r"][:, g, :], P["theta"][g], np.arange(1)) for g in range(2)], 1)
+    s0 = P["softmax_scale"] * (np.einsum("ihc,c->ih", q_c, P["c_kv"][0]) +
+                               np.einsum("ihe,he->ih", q_rot, k_rot[0, g_of, :]))
+    _close(got["lse"], s0, 1e-12, "absorbed score vs single-token lse")
+
+
+def pin_out_up_associativity(O):
+    """o = W_UV o_latent + bias (einsum 5) equals the unabsorbed o, since weights sum to 1."""
+    P = _problem(102, nq=3, H=4, G=1, r=7, dn=3, dr=2, dv=5, L=19)
+    got = O.mla_decode_reference(**P)
+    _close(O.out_up_reference(got["o_latent"], P["w_uv"], P["bias"]), got["o"], 1e-12, "einsum 5")
+
+
+ALL_PINS = [pin_absorb_single_token, pin_out_up_associativity, pin_bruteforce, pin_associativity, pin_sdpa_identity_weights, pin_zero_query_uniform,
             pin_single_token, pin_rows_sum_to_one, pin_causal_prefix, pin_rope_complex,
             pin_rope_norm_and_relative, pin_bf16_rounding, pin_rotate_fp32, pin_append_slots]

@@ -1,0 +1,134 @@
+"""The C ABI without a GPU: every declared symbol is exported, and host-side argument
+validation returns the documented status before any CUDA call."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import head_latent_attention_attn_b200 as mla
+from mla_inputs import CONFIGS
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _declared_symbols():
+    names = set()
+    inc = os.path.join(ROOT, "include")
+    for fn in os.listdir(inc):
+        if fn.endswith(".h"):
+            src = open(os.path.join(inc, fn)).read()
+            src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+            names |= set(re.findall(r"^[A-Za-z_][\w\s\*]*?\b(mla_\w+)\s*\(", src, flags=re.M))
+    return names
+
+
+def _dims(cfg=None, **kw):
+    c = cfg or CONFIGS["deepseek_v2"]
+    d = dict(num_heads=c.num_heads, num_kv_groups=c.num_kv_groups, kv_lora_rank=c.kv_lora_rank,
+             qk_nope_dim=c.qk_nope_dim, rope_dim=c.rope_dim, v_head_dim=c.v_head_dim,
+             page_size=c.page_size, softmax_scale=c.softmax_scale)
+    d.update(kw)
+    return mla.make_dims(**d)
+
+
+def test_every_declared_symbol_is_exported(mla_lib):
+    declared = _declared_symbols()
+    assert declared == set(mla.C_SYMBOLS), declared ^ set(mla.C_SYMBOLS)
+    for name in declared:
+        assert hasattr(mla_lib, name), name
+
+
+def test_row_width(mla_lib):
+    for c in CONFIGS.values():
+        assert mla.mla_row_width(_dims(c)) == c.row_width
+    assert mla.mla_row_width(_dims(num_kv_groups=3)) == -1       # 128 % 3 != 0
+    assert mla.mla_row_width(_dims(kv_lora_rank=100)) == -1      # not a multiple of 8
+    assert mla.mla_row_width(_dims(rope_dim=7)) == -1            # odd rotary dims
+    assert mla.mla_row_width(_dims(softmax_scale=0.0)) == -1
+
+
+def test_status_strings(mla_lib):
+    for code, name in mla.STATUS_NAMES.items():
+        assert mla_lib.mla_status_string(code).decode() == name
+
+
+P = ctypes.c_void_p
+FAKE = P(0x10000)  # 16-byte-aligned, never dereferenced: validation fails before use
+
+
+def _append(d, **kw):
+    a = dict(c_kv=FAKE, k_r=FAKE, cos=FAKE, sin=FAKE, table=FAKE, maxp=4, start=FAKE, batch=2,
+             n=1, cache=FAKE, npages=8, err=None)
+    a.update(kw)
+    return mla.lib().mla_cache_append(ctypes.byref(d), a["c_kv"], a["k_r"], a["cos"], a["sin"],
+                                      a["table"], a["maxp"], a["start"], a["batch"], a["n"],
+                                      a["cache"], a["npages"], a["err"], None)
+
+
+def test_append_validation(mla_lib):
+    assert _append(_dims(num_kv_groups=3)) == mla.MLA_ERR_INVALID_ARG
+    assert _append(_dims(), c_kv=None) == mla.MLA_ERR_INVALID_ARG
+    assert _append(_dims(), k_r=None) == mla.MLA_ERR_INVALID_ARG
+    assert _append(_dims(), cache=P(0x10008)) == mla.MLA_ERR_INVALID_ARG   # misaligned
+    assert _append(_dims(), batch=-1) == mla.MLA_ERR_INVALID_ARG
+    assert _append(_dims(), npages=0) == mla.MLA_ERR_INVALID_ARG
+    assert _append(_dims(), batch=0) == mla.MLA_OK                          # nothing to do
+    assert _append(_dims(), n=0) == mla.MLA_OK
+
+
+def _decode(d, **kw):
+    a = dict(q=FAKE, cache=FAKE, npages=100, table=FAKE, maxp=4, lens=FAKE, batch=2, qlen=1,
+             maxlen=256, causal=1, splits=1, ws=P(0x10000), wsb=1 << 20, o=FAKE, lse=FAKE)
+    a.update(kw)
+    return mla.lib().mla_decode_attn(ctypes.byref(d), a["q"], a["cache"], a["npages"], a["table"],
+                                     a["maxp"], a["lens"], a["batch"], a["qlen"], a["maxlen"],
+                                     a["causal"], a["splits"], a["ws"], a["wsb"], a["o"],
+                                     a["lse"], None)
+
+
+def test_decode_validation(mla_lib):
+    assert _decode(_dims(page_size=32)) == mla.MLA_ERR_UNSUPPORTED
+    assert _decode(_dims(kv_lora_rank=1024)) == mla.MLA_ERR_UNSUPPORTED
+    assert _decode(_dims(), qlen=0) == mla.MLA_ERR_INVALID_ARG
+    assert _decode(_dims(), maxlen=0) == mla.MLA_ERR_INVALID_ARG
+    assert _decode(_dims(), causal=2) == mla.MLA_ERR_INVALID_ARG
+    assert _decode(_dims(), lens=None) == mla.MLA_ERR_INVALID_ARG
+    assert _decode(_dims(), ws=None) == mla.MLA_ERR_WORKSPACE
+    assert _decode(_dims(), ws=P(0x10010)) == mla.MLA_ERR_WORKSPACE          # not 256-aligned
+    assert _decode(_dims(), splits=4, wsb=256) == mla.MLA_ERR_WORKSPACE       # partials need room
+    assert _decode(_dims(), batch=0) == mla.MLA_OK
+
+
+def test_workspace_size(mla_lib):
+    d = _dims()
+    ws = lambda *a: mla.mla_decode_workspace_size(d, *a)  # noqa: E731
+    assert ws(64, 1, 8192, 1) == 256                    # one split: only the error word
+    # 4 splits, 2 column groups of 64 rows, 64 sequences: lse + fp32 partial outputs
+    rows = 64 * 2 * 4 * 64
+    assert ws(64, 1, 8192, 4) == 256 + (rows * 4 + 255) // 256 * 256 + rows * 512 * 4
+    assert ws(64, 0, 8192, 1) == 0                      # invalid q_len
+    assert mla.mla_decode_workspace_size(_dims(page_size=16), 1, 1, 64, 1) == 0
+
+
+def test_absorb_and_out_up_validation(mla_lib):
+    L = mla.lib()
+    d = _dims()
+    st = L.mla_absorb_q(ctypes.byref(d), FAKE, FAKE, FAKE, FAKE, FAKE, 100, 4, 1, FAKE, None)
+    assert st == mla.MLA_ERR_INVALID_ARG                # head stride < d_n * r
+    st = L.mla_absorb_q(ctypes.byref(d), None, FAKE, FAKE, FAKE, FAKE, 128 * 512, 4, 1, FAKE, None)
+    assert st == mla.MLA_ERR_INVALID_ARG
+    st = L.mla_absorb_q(ctypes.byref(d), FAKE, FAKE, FAKE, FAKE, FAKE, 128 * 512, 0, 1, FAKE, None)
+    assert st == mla.MLA_OK
+    st = L.mla_out_up(ctypes.byref(d), FAKE, FAKE, 128 * 512 + 4, None, 4, FAKE, None)
+    assert st == mla.MLA_ERR_INVALID_ARG                # head stride not a multiple of 8
+    st = L.mla_out_up(ctypes.byref(d), FAKE, FAKE, 128 * 512, None, 0, FAKE, None)
+    assert st == mla.MLA_OK
+    assert L.mla_get_device_status(None, 0, None) == mla.MLA_ERR_INVALID_ARG
+
+
+def test_binding_fails_loudly_without_library(monkeypatch, tmp_path):
+    monkeypatch.setattr(mla, "_lib", None)
+    monkeypatch.setattr(mla, "LIB_PATH", str(tmp_path / "libmla.so"))
+    with pytest.raises(mla.MlaError):
+        mla.lib()

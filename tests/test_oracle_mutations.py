@@ -33,6 +33,8 @@ MUTATIONS = {
     "fp32_rotation_sign": ("y1 = np.add(", "y1 = np.subtract("),
     "append_row_shift": ("rows = pos % page_size", "rows = (pos + 1) % page_size"),
     "append_page_index": ("pages = block_table[b, pos // page_size]", "pages = block_table[b, pos // page_size * 0]"),
+    "absorb_wrong_contraction": ('np.einsum("hdc,ihd->ihc", w_uk, q_nope)', 'np.einsum("hdc,ihd->ihc", w_uk, q_nope[:, ::-1])'),
+    "out_up_bias_dropped": ("        o = o + as_f64(bias)", "        o = o + 0.0"),
     "append_groups_swapped": ("out[pages, rows, r:] = f32_to_bf16_bits(y).reshape(n, G * dr)",
                               "out[pages, rows, r:] = f32_to_bf16_bits(y[:, ::-1]).reshape(n, G * dr)"),
 }
