@@ -1,0 +1,410 @@
+#!/usr/bin/env python
+"""Benchmark of one MLA decode step on B200: append -> absorb -> decode -> out_up.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--config NAME] [--impl reference]
+
+A step is one pass of the whole decode path over one batch of synthetic input already
+resident in HBM: mla_cache_append of the q new tokens, mla_absorb_q, mla_decode_attn
+(paged, split-KV, combine) and mla_out_up. ``value`` is decode tokens per second (B*q per
+step) over all ranks; ``roofline`` describes mla_decode_attn (the dominant kernel),
+timed with CUDA events around its launches inside the timed region; ``e2e`` repeats the
+step through the same public API from pinned HOST buffers, with the host->device copy of
+the step's inputs and the device->host read of its output inside the timed region.
+Under torchrun every rank runs an independent replica on its own GPU (the path has no
+exchange step); time is the max over ranks.
+
+``--impl reference`` times the fp64 CPU oracle (the unabsorbed form) on the host cores on
+a bounded sample of the same workload.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "MLA decode attn: tokens/s, latent-cache HBM GB/s, TFLOP/s, % of roofline"
+DEFAULT_CONFIG = "deepseek_v2"
+L2_BYTES = 126 * 1024 * 1024
+
+
+def _peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        d = json.load(open(path))
+        return {"hbm_gbs": float(d["hbm_gbs"]), "bf16_tflops": float(d["bf16_tflops"]),
+                "bf16_tflops_sustained": float(d.get("bf16_tflops_sustained", d["bf16_tflops"])),
+                "source": "measured"}
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0,
+            "source": "fallback"}
+
+
+def algorithmic_work(cfg, seq_lens):
+    """Latent-cache bytes read and FLOPs of one mla_decode_attn launch.
+
+    Bytes: every cached row (D bf16) of every sequence, read once for all heads and query
+    rows. FLOPs: 2*H*(r + d_r) for the scores and 2*H*r for o_ per query row and visible
+    cached token (padding of the rotary slots and of the UMMA tiles not counted)."""
+    D = cfg.row_width
+    tokens = int(np.sum(seq_lens, dtype=np.int64))
+    nbytes = tokens * D * 2
+    q, H, r, dr = cfg.q_len, cfg.num_heads, cfg.kv_lora_rank, cfg.rope_dim
+    vis = 0
+    for L in seq_lens:
+        for i in range(q):
+            vis += int(L) - q + i + 1 if cfg.causal else int(L)
+    flops = vis * (2 * H * (r + dr) + 2 * H * r)
+    return nbytes, flops
+
+
+class ClockSampler:
+    """nvidia-smi clocks and throttle reasons sampled every 200 ms while running."""
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_id: str):
+        self.gpu = gpu_id  # nvidia-smi -i accepts an index or a UUID
+        self.proc = None
+        self.path = None
+
+    def __enter__(self):
+        try:
+            out_dir = os.path.join(ROOT, "gpurun_out")
+            os.makedirs(out_dir, exist_ok=True)
+            self.path = os.path.join(out_dir, f"clocks_rank{os.environ.get('RANK', '0')}.csv")
+            self.fh = open(self.path, "w")
+            self.proc = subprocess.Popen(["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.Q}",
+                                          "--format=csv,noheader,nounits", "-lms", "200"],
+                                         stdout=self.fh, stderr=subprocess.DEVNULL)
+            time.sleep(0.3)
+        except Exception:
+            self.proc = None
+        return self
+
+    def __exit__(self, *a):
+        if self.proc is not None:
+            time.sleep(0.25)
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except Exception:
+                self.proc.kill()
+            self.fh.close()
+
+    def summary(self):
+        if self.proc is None or self.path is None or not os.path.exists(self.path):
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"]}
+        sms, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in open(self.path):
+            f = [x.strip() for x in line.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm, mx = float(f[1]), float(f[2])
+            except ValueError:
+                continue
+            sms.append(sm)
+            for n, v in zip(names, f[5:9]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        if not sms:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"]}
+        loaded = [s for s in sms if s > 0.5 * (mx or max(sms))] or sms
+        return {"sm_mhz": statistics.median(loaded), "sm_max_mhz": mx, "samples": len(sms),
+                "reasons": sorted(reasons)}
+
+
+def _source_hash():
+    h = hashlib.sha256()
+    for f in ("decode.cu", "ptx.cuh", "kernels.h"):
+        h.update(open(os.path.join(ROOT, "head_latent_attention_attn_b200", "csrc", f), "rb").read())
+    return h.hexdigest()[:16]
+
+
+def _traffic(config_name):
+    """Per-launch DRAM bytes of mla_decode_attn from a committed ncu summary, if it was taken
+    on the current kernel source; else None."""
+    path = os.path.join(ROOT, "profiles", "decode_traffic.json")
+    if not os.path.exists(path):
+        return None
+    d = json.load(open(path))
+    e = d.get(config_name)
+    if not e or e.get("source_hash") != _source_hash():
+        return None
+    return e.get("dram_bytes_per_launch")
+
+
+def cpu_oracle_sample(cfg, wl, budget_s=12.0, max_seqs=None):
+    """Time the fp64 oracle on whole sequences of the workload until ``budget_s`` is spent."""
+    import oracle.mla_oracle as O
+    try:
+        from threadpoolctl import threadpool_info
+        cores = max([i.get("num_threads", 1) for i in threadpool_info()] + [1])
+    except Exception:
+        cores = os.cpu_count()
+    order = list(np.argsort(-wl.seq_lens)) if cfg.lens_range else list(range(cfg.batch))
+    done, tok_ctx, t0 = [], 0, time.perf_counter()
+    for b in order:
+        c_kv, k_r = wl.context(int(b))
+        O.mla_decode_reference(wl.q_nope[b], wl.q_pe[b], c_kv, k_r, wl.w_uk, wl.w_uv, wl.bias,
+                               wl.theta, wl.query_positions()[b], cfg.softmax_scale, causal=cfg.causal)
+        done.append(int(b))
+        tok_ctx += int(wl.seq_lens[b])
+        if time.perf_counter() - t0 >= budget_s or (max_seqs and len(done) >= max_seqs):
+            break
+    el = time.perf_counter() - t0
+    return {"value": len(done) * cfg.q_len / el, "unit": "tokens/s", "cores": int(cores),
+            "kind": "oracle",
+            "sample": f"{len(done)} of {cfg.batch} sequences ({tok_ctx} cached tokens, all "
+                      f"{cfg.num_heads} heads), fp64 unabsorbed form, {el:.1f} s"}
+
+
+def run_reference(args, cfg, rank, world):
+    from mla_inputs import make_workload
+    if rank != 0:
+        return
+    wl = make_workload(cfg)
+    per_step = []
+    for it in range(args.warmup + args.steps):
+        s = cpu_oracle_sample(cfg, wl, budget_s=0.0, max_seqs=1)
+        if it >= args.warmup:
+            per_step.append(s)
+    v = statistics.mean(x["value"] for x in per_step)
+    line = {"impl": "reference", "metric": METRIC, "value": v, "unit": "tokens/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1000.0 * cfg.q_len / v,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic", "config": _config_json(cfg),
+            "cpu_baseline": {"value": v, "unit": "tokens/s", "cores": per_step[0]["cores"],
+                             "kind": "oracle", "sample": "each step: " + per_step[0]["sample"]},
+            "e2e": {"value": v, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def _config_json(cfg):
+    return {"workload": cfg.name, "batch": cfg.batch, "q_len": cfg.q_len, "heads": cfg.num_heads,
+            "kv_groups": cfg.num_kv_groups, "kv_lora_rank": cfg.kv_lora_rank,
+            "rope_dim_per_group": cfg.rope_dim, "qk_nope_dim": cfg.qk_nope_dim,
+            "v_head_dim": cfg.v_head_dim, "page_size": cfg.page_size,
+            "context": cfg.context if cfg.lens_range is None else f"U{list(cfg.lens_range)}",
+            "parallelism": "replicas"}
+
+
+def run_gpu(args, cfg, rank, world, dist):
+    import torch
+
+    import head_latent_attention_attn_b200 as mla
+    from mla_inputs import make_workload
+    sys.path.insert(0, os.path.join(ROOT, "tests"))
+    from tests.gpu_harness import GpuProblem
+
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    mla.lib()
+    wl = make_workload(cfg)
+    prob = GpuProblem(wl, num_splits=args.splits, device=str(dev))
+    stream = torch.cuda.current_stream()
+    nbytes, flops = algorithmic_work(cfg, wl.seq_lens)
+    cache_bytes = nbytes
+    flush = None
+    if cache_bytes < 2 * L2_BYTES:
+        flush = torch.empty(4 * L2_BYTES // 4, dtype=torch.float32, device=dev)
+    plan_splits_ws = prob.workspace.numel()
+
+    def barrier():
+        if dist is not None:
+            dist.barrier()
+        torch.cuda.synchronize()
+
+    def one_step(ev):
+        # ev = (step_start, dec_start, dec_end, step_end)
+        ev[0].record(stream)
+        mla.mla_cache_append(prob.dims, prob.c_new, prob.k_new, prob.cos_q, prob.sin_q,
+                             prob.block_table, prob.start_pos, prob.cache,
+                             dev_error=prob.workspace.view(torch.int32)[:1], stream=stream)
+        mla.mla_absorb_q(prob.dims, prob.q_nope, prob.q_pe, prob.cos_q, prob.sin_q, prob.w_uk,
+                         prob.q_ext, stream=stream)
+        ev[1].record(stream)
+        mla.mla_decode_attn(prob.dims, prob.q_ext, prob.cache, prob.block_table, prob.seq_lens,
+                            prob.max_seq_len, prob.workspace, prob.o_latent, prob.lse,
+                            causal=cfg.causal, num_splits=args.splits, stream=stream)
+        ev[2].record(stream)
+        mla.mla_out_up(prob.dims, prob.o_latent, prob.w_uv, prob.o, bias=prob.bias, stream=stream)
+        ev[3].record(stream)
+
+    mk = lambda: [torch.cuda.Event(enable_timing=True) for _ in range(4)]  # noqa: E731
+    for _ in range(args.warmup):
+        if flush is not None:
+            flush.zero_()
+        one_step(mk())
+    barrier()
+    evs = []
+    with ClockSampler(_gpu_id(local)) as clk:
+        barrier()
+        for _ in range(args.steps):
+            if flush is not None:
+                flush.zero_()
+            e = mk()
+            one_step(e)
+            evs.append(e)
+        barrier()
+    step_ms = [e[0].elapsed_time(e[3]) for e in evs]
+    dec_ms = [e[1].elapsed_time(e[2]) for e in evs]
+    t_step = sum(step_ms) / len(step_ms)
+    t_dec = sum(dec_ms) / len(dec_ms)
+    status = mla.mla_get_device_status(prob.workspace.view(torch.int32)[:1])
+    if status != mla.MLA_OK:
+        raise RuntimeError(f"device error word set: {mla.STATUS_NAMES[status]}")
+
+    # ---- end to end through the public API with pinned host buffers ------------------------
+    host_in = {k: getattr(prob, k).detach().cpu().pin_memory()
+               for k in ("c_new", "k_new", "cos_q", "sin_q", "start_pos", "q_nope", "q_pe")}
+    host_o = torch.empty(prob.o.shape, dtype=prob.o.dtype).pin_memory()
+    host_lse = torch.empty(prob.lse.shape, dtype=prob.lse.dtype).pin_memory()
+    h2d = sum(t.numel() * t.element_size() for t in host_in.values())
+    d2h = host_o.numel() * host_o.element_size() + host_lse.numel() * host_lse.element_size()
+
+    def e2e_step():
+        for k, t in host_in.items():
+            getattr(prob, k).copy_(t, non_blocking=True)
+        mla.mla_decode_step(prob.dims, c_kv_new=prob.c_new, k_r_new=prob.k_new,
+                            cos_new=prob.cos_q, sin_new=prob.sin_q, start_pos=prob.start_pos,
+                            q_nope=prob.q_nope, q_pe=prob.q_pe, cos_q=prob.cos_q, sin_q=prob.sin_q,
+                            w_uk=prob.w_uk, w_uv=prob.w_uv, bias=prob.bias, cache=prob.cache,
+                            block_table=prob.block_table, seq_lens=prob.seq_lens,
+                            max_seq_len=prob.max_seq_len, q_ext=prob.q_ext,
+                            workspace=prob.workspace, o_latent=prob.o_latent, lse=prob.lse,
+                            o=prob.o, causal=cfg.causal, num_splits=args.splits, stream=stream)
+        host_o.copy_(prob.o, non_blocking=True)
+        host_lse.copy_(prob.lse, non_blocking=True)
+
+    for _ in range(args.warmup):
+        e2e_step()
+    barrier()
+    e2e_ms = []
+    for _ in range(args.steps):
+        if flush is not None:
+            flush.zero_()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        e2e_step()
+        b.record(stream)
+        b.synchronize()
+        e2e_ms.append(a.elapsed_time(b))
+    barrier()
+    t_e2e = sum(e2e_ms) / len(e2e_ms)
+
+    # ---- max over ranks -------------------------------------------------------------------
+    vec = torch.tensor([t_step, t_dec, t_e2e], dtype=torch.float64, device=dev)
+    if dist is not None:
+        dist.all_reduce(vec, op=dist.ReduceOp.MAX)
+    t_step, t_dec, t_e2e = [float(x) for x in vec.tolist()]
+    if rank != 0:
+        return
+    peaks = _peaks()
+    tokens = cfg.batch * cfg.q_len
+    value = world * tokens / (t_step * 1e-3)
+    gbs = nbytes / (t_dec * 1e-3) / 1e9
+    tfl = flops / (t_dec * 1e-3) / 1e12
+    t_hbm = nbytes / (peaks["hbm_gbs"] * 1e9)
+    t_tc = flops / (peaks["bf16_tflops"] * 1e12)
+    bound = "hbm" if t_hbm >= t_tc else "tensor"
+    if bound == "hbm":
+        roof = {"bound": "hbm", "achieved": gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                "frac": gbs / peaks["hbm_gbs"]}
+    else:
+        roof = {"bound": "tensor", "achieved": tfl, "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
+                "frac": tfl / peaks["bf16_tflops"]}
+    roof["traffic"] = _traffic(cfg.name)
+    roof["peak_source"] = peaks["source"]
+    roof["kernel"] = "mla_decode_attn (decode kernel + split combine when splits > 1)"
+    roof["algorithmic_bytes_per_launch"] = nbytes
+    roof["algorithmic_flops_per_launch"] = flops
+    roof["roofline_time_us"] = 1e6 * max(t_hbm, t_tc)
+    roof["pct_of_roofline"] = 100.0 * max(t_hbm, t_tc) / (t_dec * 1e-3)
+    # append, absorb, decode, out_up (+ the split combine when the plan has > 1 split;
+    # a one-split plan needs only the 256-byte error-word workspace)
+    launches_per_step = 4 + (1 if plan_splits_ws > 256 else 0)
+    line = {
+        "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": t_step,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic",
+        "config": dict(_config_json(cfg), l2=("cache > L2, no flush" if flush is None
+                                              else "L2 flushed between steps (512 MB write)")),
+        "decode_us": 1e3 * t_dec, "decode_gbs": gbs, "decode_tflops": tfl,
+        "roofline": roof,
+        "e2e": {"value": world * tokens / (t_e2e * 1e-3), "unit": "tokens/s",
+                "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
+                "ms_per_step": t_e2e},
+        "gpu_launches": launches_per_step * args.steps,
+        "clocks": clk.summary(),
+    }
+    if world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_oracle_sample(cfg, wl, budget_s=args.cpu_budget)
+    print(json.dumps(line), flush=True)
+
+
+def _gpu_id(local: int) -> str:
+    import torch
+    try:
+        u = str(torch.cuda.get_device_properties(local).uuid)
+        return u if u.startswith("GPU-") else "GPU-" + u
+    except Exception:
+        return str(local)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--config", default=DEFAULT_CONFIG)
+    ap.add_argument("--impl", default="b200", choices=["b200", "reference"])
+    ap.add_argument("--splits", type=int, default=0, help="KV splits per sequence (0 = auto)")
+    ap.add_argument("--cpu-budget", type=float, default=12.0)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    args.warmup = max(args.warmup, 3)
+
+    from mla_inputs import CONFIGS
+    cfg = CONFIGS[args.config]
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    dist = None
+    if world > 1:
+        import datetime
+
+        import torch
+        import torch.distributed as tdist
+        if args.impl == "reference":
+            if rank == 0:
+                run_reference(args, cfg, rank, world)
+            return
+        torch.cuda.set_device(int(os.environ.get("LOCAL_RANK", "0")))
+        tdist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300))
+        dist = tdist
+    try:
+        if args.impl == "reference":
+            run_reference(args, cfg, rank, world)
+        else:
+            run_gpu(args, cfg, rank, world, dist)
+    finally:
+        if dist is not None:
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

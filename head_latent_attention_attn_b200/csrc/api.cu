@@ -13,6 +13,8 @@ namespace {
 
 constexpr int kMaxSmem = 232448;  // 227 KB opt-in dynamic shared memory per CTA
 
+
+
 inline cudaStream_t as_stream(void* s) { return reinterpret_cast<cudaStream_t>(s); }
 
 int num_sms() {
@@ -33,11 +35,13 @@ int pow2_at_least(int x, int lo) {
 
 // Launch geometry of one mla_decode_attn problem.
 struct DecodePlan {
-  int ncol, col_groups, nblk, nch, slot_blocks, nslot, npt, tmem_cols, splits, tiles_per_split;
+  int ncol, col_groups, units, nblk, nch, slot_blocks, nslot, npt, tmem_cols, grid;
   size_t smem;
   size_t ws_bytes;
-  size_t part_lse_off, part_o_off;
+  size_t range_off, unit_start_off, part_lse_off, part_o_off;
 };
+
+size_t align256(size_t x) { return (x + 255) / 256 * 256; }
 
 mla_status plan_decode(const mla_dims* d, int32_t batch, int32_t q_len, int32_t max_seq_len,
                        int32_t num_splits, DecodePlan* P) {
@@ -50,9 +54,11 @@ mla_status plan_decode(const mla_dims* d, int32_t batch, int32_t q_len, int32_t 
   const int D = row_width(d);
   if (r > 512 || D > 64 * kDecodeMaxBlk) return MLA_ERR_UNSUPPORTED;
   const int64_t qH = int64_t(q_len) * d->num_heads;
-  if (qH > 64 * 65535) return MLA_ERR_UNSUPPORTED;
   P->ncol = qH <= 16 ? 16 : (qH <= 32 ? 32 : 64);
   P->col_groups = int((qH + P->ncol - 1) / P->ncol);
+  const int64_t units = int64_t(std::max(batch, 1)) * P->col_groups;
+  if (units > (int64_t(1) << 24)) return MLA_ERR_UNSUPPORTED;
+  P->units = int(units);
   P->nblk = (D + 63) / 64;
   P->nch = (r + 127) / 128;
   P->slot_blocks = std::max(P->nblk, 2 * P->nch);
@@ -71,27 +77,25 @@ mla_status plan_decode(const mla_dims* d, int32_t batch, int32_t q_len, int32_t 
   }
   if (P->nslot < 2) return MLA_ERR_UNSUPPORTED;
   P->smem = decode_smem_bytes(P->ncol, P->nblk, P->slot_blocks, P->nslot, P->npt);
-  const int max_tiles = (max_seq_len + kDecodeTok - 1) / kDecodeTok;
-  const int64_t units = int64_t(std::max(batch, 1)) * P->col_groups;
-  int S = num_splits;
-  if (S == 0) {
-    const int sms = num_sms();
-    S = units >= sms ? 1 : int(sms / units);
-  }
-  S = std::max(1, std::min(S, max_tiles));
-  P->tiles_per_split = (max_tiles + S - 1) / S;
-  S = (max_tiles + P->tiles_per_split - 1) / P->tiles_per_split;  // drop empty splits
-  if (S > 65535) return MLA_ERR_UNSUPPORTED;
-  P->splits = S;
-  size_t off = 256;  // device error word + padding
+  // Persistent grid: the units' page tiles are cut into `grid` equal ranges. By default
+  // one CTA per SM; num_splits > 0 asks for num_splits ranges per unit on average.
+  const int64_t max_tiles = (int64_t(max_seq_len) + kDecodeTok - 1) / kDecodeTok;
+  // The grid is a multiple of the number of row blocks: CTA c works on row block
+  // c % col_groups, so the blocks of a sequence are read in lockstep.
+  const int cgs = P->col_groups;
+  int64_t g = num_splits > 0 ? units * num_splits : num_sms();
+  g = std::min<int64_t>(g, units * max_tiles);
+  g = std::max<int64_t>(cgs, std::min<int64_t>(g, 1 << 20) / cgs * cgs);
+  P->grid = int(g);
+  size_t off = 256;                              // device error word + padding
+  P->range_off = off;                            // int32: tiles per CTA range
+  off += 256;
+  P->unit_start_off = off;                       // int32 per unit: its first global tile
+  off = align256(off + size_t(units) * sizeof(int32_t));
   P->part_lse_off = off;
+  off = align256(off + size_t(g) * 2 * P->ncol * sizeof(float));
   P->part_o_off = off;
-  if (S > 1) {
-    const size_t rows = size_t(std::max(batch, 1)) * P->col_groups * S * P->ncol;
-    off += (rows * sizeof(float) + 255) / 256 * 256;
-    P->part_o_off = off;
-    off += rows * size_t(r) * sizeof(float);
-  }
+  off += size_t(g) * 2 * P->ncol * size_t(r) * sizeof(float);
   P->ws_bytes = off;
   return MLA_OK;
 }
@@ -297,6 +301,8 @@ mla_status mla_decode_attn(const mla_dims* dims, const void* q_ext, const void* 
   p.lse = lse;
   p.part_lse = reinterpret_cast<float*>(ws + P.part_lse_off);
   p.part_o = reinterpret_cast<float*>(ws + P.part_o_off);
+  p.unit_start = reinterpret_cast<int32_t*>(ws + P.unit_start_off);
+  p.range_len = reinterpret_cast<int32_t*>(ws + P.range_off);
   p.dev_error = reinterpret_cast<int32_t*>(ws);
   p.num_pages = num_pages;
   p.max_pages = max_pages_per_seq;
@@ -309,8 +315,7 @@ mla_status mla_decode_attn(const mla_dims* dims, const void* q_ext, const void* 
   p.nblk = P.nblk;
   p.nch = P.nch;
   p.col_groups = P.col_groups;
-  p.splits = P.splits;
-  p.tiles_per_split = P.tiles_per_split;
+  p.units = P.units;
   p.max_seq_len = max_seq_len;
   p.causal = causal;
   p.nslot = P.nslot;
@@ -318,22 +323,29 @@ mla_status mla_decode_attn(const mla_dims* dims, const void* q_ext, const void* 
   p.tmem_cols = P.tmem_cols;
   p.npt = P.npt;
   p.scale_log2 = dims->softmax_scale * 1.4426950408889634f;
-  const dim3 grid(P.splits, P.col_groups, batch);
   cudaStream_t s = as_stream(stream);
-  if (launch_decode(p, P.ncol, grid, P.smem, s) != cudaSuccess) return MLA_ERR_CUDA;
-  if (P.splits > 1) {
+  if (launch_decode(p, P.ncol, dim3(P.grid), P.smem, s) != cudaSuccess) return MLA_ERR_CUDA;
+  if (P.grid > 1) {
+    // merge the pieces of units cut between CTAs (units held whole are skipped)
     CombineParams c{};
     c.part_o = p.part_o;
     c.part_lse = p.part_lse;
+    c.unit_start = p.unit_start;
+    c.range_len = p.range_len;
+    c.seq_lens = seq_lens;
     c.o_latent = p.o_latent;
     c.lse = lse;
-    c.batch = batch;
-    c.qH = int32_t(qH);
+    c.q_len = q_len;
+    c.max_seq_len = max_seq_len;
+    c.max_pages = max_pages_per_seq;
+    c.qH = p.qH;
     c.r = p.r;
     c.ncol = P.ncol;
     c.col_groups = P.col_groups;
-    c.splits = P.splits;
-    if (launch_combine(c, s) != cudaSuccess) return MLA_ERR_CUDA;
+    c.units = P.units;
+    const int64_t items = int64_t(P.units) * P.ncol * ((p.r + 127) / 128);
+    const int cgrid = int(std::min<int64_t>(items, int64_t(num_sms()) * 8));
+    if (launch_combine(c, cgrid, s) != cudaSuccess) return MLA_ERR_CUDA;
   }
   return MLA_OK;
 }

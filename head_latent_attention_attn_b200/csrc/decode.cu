@@ -1,24 +1,31 @@
 // decode.cu - mla_decode_attn on sm_100a: paged, split-KV absorbed attention over the
-// latent cache, plus the log-sum-exp combine of the splits.
+// latent cache, with the split merge fused into the same launch.
 //
 // Formulation. Every query row (i, h) of a sequence scores the SAME cache rows, so the
-// CTA keeps the query block resident and streams the cache once:
+// CTA keeps a block of NCOL query rows resident and streams the cache pages once:
 //   S^T[tok, n] = C[tok, :] . Q[n, :]          UMMA M=64 tokens, N=NCOL rows, K = D
 //   O^T[c, n]  += C[tok, c]^T P^T[tok, n]      UMMA M=128 latent, N=NCOL, K = 64 tokens
-// with C a 64-token page of the cache (row = [c_kv | rotated keys]), Q = q_ext rows, and
-// P^T the softmax weights written by the softmax warps. Putting tokens on M keeps N (the
-// query rows, 4..64) free of padding and puts O^T's latent on TMEM lanes, so O^T needs
-// only ceil(r/128) * NCOL TMEM columns. The same TMA-loaded, 128B-swizzled page is read
+// with C one 64-token page of the cache (row = [c_kv | rotated keys]), Q the q_ext rows
+// and P^T the softmax weights written by the softmax warps. Tokens on M keep N (4..64
+// query rows) free of padding and put O^T's latent on TMEM lanes, so O^T needs only
+// ceil(r/128) * NCOL TMEM columns. The same TMA-loaded, 128B-swizzled page is read
 // K-major for S^T and MN-major for O^T.
 //
-// Roles (192 threads): warp 0 TMA producer, warp 1 UMMA issuer + TMEM owner, warps 2-5
-// softmax (one token per lane in lanes 0-15 of each TMEM sub-partition, as the M=64
-// accumulator layout places rows 16*sp..16*sp+15 in lanes 32*sp..32*sp+15) and epilogue.
+// Schedule. A "unit" is (sequence b, block cg of NCOL query rows); its work is
+// ceil(L_b / 64) page tiles. The units' tiles are laid end to end and cut into gridDim.x
+// equal ranges, one per CTA, so ragged lengths balance. A CTA walks the units its range
+// touches; a unit it holds whole is written straight to o_latent / lse, a unit cut
+// between CTAs leaves one normalised fp32 partial (o, lse) per piece, merged afterwards
+// by mla_combine_kernel with the log-sum-exp identity.
 //
-// Online softmax in the log2 domain with a lazily updated per-row reference max: the
-// reference only moves when some score exceeds it by more than 8 (so unnormalised
-// weights stay <= 256); then the new tile max is reduced across the CTA and O^T and the
-// running sums are rescaled. Per-thread partial row sums are reduced once at the end.
+// Roles (192 threads): warp 0 TMA producer, warp 1 UMMA issuer and TMEM owner, warps 2-5
+// softmax and epilogue. In the M=64 accumulator layout rows 16*sp..16*sp+15 sit in lanes
+// 32*sp..32*sp+15 of TMEM sub-partition sp; the 16x32bx2 load gives each of those 16
+// tokens to two threads, one per half of the NCOL columns.
+//
+// Online softmax in the log2 domain with a lazily moved reference max per query row:
+// it moves only when a score exceeds it by more than 8 (unnormalised weights stay <= 256);
+// then the tile max is reduced over the CTA and O^T and the running sums are rescaled.
 #include <math.h>
 
 #include "kernels.h"
@@ -26,18 +33,43 @@
 
 namespace mla {
 
+// Optional per-tile timeline of CTA 0 (compile with -DMLA_TRACE; read with mla_trace_read).
+// Events: 0 producer starts a tile, 1 S issued (all blocks landed), 2 S committed, 3 PV
+// committed, 4 softmax sees S, 5 after the vote barrier, 6 P buffer free, 7 P written
+// and PV about to be issued, 8 producer finished issuing the tile, 9 first block landed.
+#ifdef MLA_TRACE
+constexpr int kTraceTiles = 512;
+__device__ unsigned long long g_mla_trace[10 * kTraceTiles + 1];
+#define MLA_TRACE_AT(ev, idx)                                                         \
+  do {                                                                                \
+    if (blockIdx.x == 0 && (idx) < kTraceTiles) g_mla_trace[(ev) * kTraceTiles + (idx)] = clock64(); \
+  } while (0)
+#else
+#define MLA_TRACE_AT(ev, idx) \
+  do {                       \
+  } while (0)
+#endif
+
 namespace {
 
 constexpr int kThreads = 192;
 constexpr int kBlkBytes = kDecodeTok * 128;   // one 64 x 64 bf16 block, 8 KB
 constexpr float kLazyThreshold = 8.0f;        // log2 units
+// Initial reference max: finite, so a masked score (-inf) minus it is exactly -inf (weight
+// 0) and any finite score exceeds it, forcing the first real reference to be computed.
+constexpr float kRefInit = -3.0e38f;
 constexpr float kLn2 = 0.69314718055994530942f;
+// misc ints: [0,8) vote flags, 8 TMEM base, 9 abort flag, [10,16) schedule, [16,22) warp
+// sums, [23,25) reference-moved flags; 32 reserved.
+constexpr int kMiscInts = 32;
 
 struct DecodeLayout {
-  uint32_t q_off, slot_off, pt_off, red_off, m_off, flag_off, misc_off, bar_off, total;
+  uint32_t q_off, slot_off, pt_off, red_off, alpha_off, mref_off, misc_off, bar_off, total;
 };
 
 __host__ __device__ inline uint32_t round_up(uint32_t x, uint32_t a) { return (x + a - 1) / a * a; }
+
+__host__ __device__ constexpr int num_bars(int nslot, int nblk) { return nslot * nblk + nslot + 8; }
 
 __host__ __device__ inline DecodeLayout decode_layout(int ncol, int nblk, int slot_blocks,
                                                       int nslot, int npt) {
@@ -49,16 +81,16 @@ __host__ __device__ inline DecodeLayout decode_layout(int ncol, int nblk, int sl
   off += uint32_t(nslot) * slot_blocks * kBlkBytes;
   L.pt_off = off;
   off += uint32_t(npt) * round_up(uint32_t(kDecodeTok) * ncol * 2, 1024);
-  L.red_off = off;                 // float red[4][64]
+  L.red_off = off;                 // float red[4][64]: per-warp column partials
   off += 4 * 64 * 4;
-  L.m_off = off;                   // float m_ref[64]
+  L.alpha_off = off;               // float alpha[64]: O^T rescale factor per column
   off += 64 * 4;
-  L.flag_off = off;                // int flags[2][4]
-  off += 2 * 4 * 4;
-  L.misc_off = off;                // uint32 tmem base, int abort flag
-  off += 16;
-  L.bar_off = round_up(off, 8);    // mbarriers
-  off = L.bar_off + 8 * (nslot * nblk + nslot + 1 + 2 * 4);
+  L.mref_off = off;                // float mref[64]: reference max per column
+  off += 64 * 4;
+  L.misc_off = off;                // int misc[kMiscInts], index map in the kernel
+  off += 4 * kMiscInts;
+  L.bar_off = round_up(off, 8);
+  off = L.bar_off + 8 * num_bars(nslot, nblk);
   L.total = off + 1024;            // slack for 1024-byte alignment of the base
   return L;
 }
@@ -67,20 +99,85 @@ MLA_DEVICE uint8_t* align1024(uint8_t* p) {
   return reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(p) + 1023) & ~uintptr_t(1023));
 }
 
-template <int NCOL>
-MLA_DEVICE void tmem_ld_cols(uint32_t taddr, float* v) {
-#pragma unroll
-  for (int c = 0; c < NCOL; c += 16) tmem_ld16(taddr + c, v + c);
+// 16x32bx2 TMEM load of the M=64 S^T accumulator: threads 0-15 read lanes 0-15 of the
+// warp's sub-partition at columns [c, c+HALF), threads 16-31 the same lanes at
+// [c+HALF, c+2*HALF).
+template <int HALF>
+MLA_DEVICE void tmem_ld_s(uint32_t taddr, float* v);
+
+template <>
+MLA_DEVICE void tmem_ld_s<8>(uint32_t taddr, float* v) {
+  uint32_t* r = reinterpret_cast<uint32_t*>(v);
+  asm volatile("tcgen05.ld.sync.aligned.16x32bx2.x8.b32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8], 8;"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]),
+                 "=r"(r[6]), "=r"(r[7])
+               : "r"(taddr)
+               : "memory");
 }
 
-template <int NCOL>
-MLA_DEVICE void tmem_st_cols(uint32_t taddr, const float* v) {
-#pragma unroll
-  for (int c = 0; c < NCOL; c += 16) tmem_st16(taddr + c, v + c);
+template <>
+MLA_DEVICE void tmem_ld_s<16>(uint32_t taddr, float* v) {
+  uint32_t* r = reinterpret_cast<uint32_t*>(v);
+  asm volatile(
+      "tcgen05.ld.sync.aligned.16x32bx2.x16.b32 "
+      "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16], 16;"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+        "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]),
+        "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
+      : "r"(taddr)
+      : "memory");
+}
+
+template <>
+MLA_DEVICE void tmem_ld_s<32>(uint32_t taddr, float* v) {
+  uint32_t* r = reinterpret_cast<uint32_t*>(v);
+  asm volatile(
+      "tcgen05.ld.sync.aligned.16x32bx2.x32.b32 "
+      "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
+      "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32], 32;"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+        "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]),
+        "=r"(r[13]), "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]),
+        "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]),
+        "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]),
+        "=r"(r[31])
+      : "r"(taddr)
+      : "memory");
 }
 
 __host__ __device__ constexpr SmemSwizzle pt_swizzle(int ncol) {
   return ncol == 64 ? kSw128 : (ncol == 32 ? kSw64 : kSw32);
+}
+
+MLA_DEVICE int unit_tiles(int L) { return L > 0 ? (L + kDecodeTok - 1) / kDecodeTok : 1; }
+
+// Context length of sequence b if it is within the bounds the launch was planned for,
+// else 0 (the unit then produces zeros and lse = -inf, and the error word is set).
+MLA_DEVICE int valid_len(const DecodeParams& p, int L) {
+  const bool ok = L >= p.q_len && L <= p.max_seq_len &&
+                  int64_t(L) <= int64_t(p.max_pages) * kDecodeTok;
+  return ok ? L : 0;
+}
+
+// The walk over the sequences a CTA's tile range touches; every role runs the same walk.
+// A CTA works on one block cg of query rows: unit u = b * col_groups + cg.
+struct UnitWalk {
+  int b, s;       // sequence and the index of its first tile in this row block's tile space
+  int tiles, L, u;
+  MLA_DEVICE void load(const DecodeParams& p, int cg) {
+    L = valid_len(p, p.seq_lens[b]);
+    tiles = unit_tiles(L);
+    u = b * p.col_groups + cg;
+  }
+};
+
+// Partial-result slot of virtual CTA i (of row block cg) holding a piece of a unit whose
+// first tile is s, when ranges are `per` tiles long: slot 0 holds a CTA's first piece,
+// slot 1 its last. A unit is the first piece of every CTA it reaches except possibly the
+// one where it starts.
+MLA_DEVICE int piece_slot(int i, int s, int per, int col_groups, int cg) {
+  const int i0 = s / per;
+  return 2 * (i * col_groups + cg) + ((i == i0 && s != i0 * per) ? 1 : 0);
 }
 
 }  // namespace
@@ -92,6 +189,7 @@ size_t decode_smem_bytes(int ncol, int nblk, int slot_blocks, int nslot, int npt
 template <int NCOL>
 __global__ void __launch_bounds__(kThreads, 1)
     mla_decode_kernel(const __grid_constant__ DecodeParams p) {
+  constexpr int HALF = NCOL / 2;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* base = align1024(smem_raw);
   const DecodeLayout lay = decode_layout(NCOL, p.nblk, p.slot_blocks, p.nslot, p.npt);
@@ -99,26 +197,33 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint8_t* slots = base + lay.slot_off;
   uint8_t* pt = base + lay.pt_off;
   float* red = reinterpret_cast<float*>(base + lay.red_off);
-  float* m_ref = reinterpret_cast<float*>(base + lay.m_off);
-  int* flags = reinterpret_cast<int*>(base + lay.flag_off);
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(base + lay.misc_off);
-  volatile int* abort_flag = reinterpret_cast<volatile int*>(base + lay.misc_off + 4);
+  float* alpha_s = reinterpret_cast<float*>(base + lay.alpha_off);
+  float* mref_s = reinterpret_cast<float*>(base + lay.mref_off);
+  int* misc = reinterpret_cast<int*>(base + lay.misc_off);
+  int* flags = misc;                                   // [2][4]
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(misc + 8);
+  volatile int* abort_flag = misc + 9;
+  int* sched = misc + 10;                              // b_a, s_a, r0, r1, per, scan carry
+  int* warp_sum = misc + 16;                           // [6]
+  int* chg_flag = misc + 23;                           // [2] reference moved, per half
+  static_assert(23 + 2 <= kMiscInts, "misc ints overflow into the mbarriers");
   uint64_t* bars = reinterpret_cast<uint64_t*>(base + lay.bar_off);
-  uint64_t* full = bars;                                        // [slot][blk]
-  uint64_t* empty = full + p.nslot * p.nblk;                    // [slot]
-  uint64_t* q_full = empty + kDecodeMaxSlots;
-  uint64_t* s_full = q_full + 1;                                // [2]
-  uint64_t* s_free = s_full + 2;                                // [2]
-  uint64_t* p_full = s_free + 2;                                // [2]
-  uint64_t* pv_done = p_full + 2;                               // [2]
+  uint64_t* full = bars;                               // [slot][blk]
+  uint64_t* empty = full + p.nslot * p.nblk;           // [slot]
+  uint64_t* q_full = empty + p.nslot;
+  uint64_t* q_empty = q_full + 1;
+  uint64_t* s_full = q_empty + 1;                      // [2]
+  uint64_t* s_free = s_full + 2;                       // [2]
+  uint64_t* pv_done = s_free + 2;                      // [2]
 
   constexpr uint32_t kPtBytes = ((kDecodeTok * NCOL * 2) + 1023) / 1024 * 1024;
   constexpr uint32_t kQBlk = NCOL * 128;
+  const uint32_t slot_bytes = uint32_t(p.slot_blocks) * kBlkBytes;
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-  const int split = blockIdx.x;
-  const int cg = blockIdx.y;
-  const int b = blockIdx.z;
+  const int cg = int(blockIdx.x) % p.col_groups;       // row block of this CTA
+  const int vc = int(blockIdx.x) / p.col_groups;       // index among the CTAs of that block
+  const int vgrid = int(gridDim.x) / p.col_groups;
   const WaitCtx wc{abort_flag, p.dev_error};
 
   if (threadIdx.x == 0) {
@@ -127,10 +232,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&empty[s], 1);
     }
     mbar_init(q_full, 1);
+    mbar_init(q_empty, 1);
     for (int i = 0; i < 2; ++i) {
       mbar_init(&s_full[i], 1);
-      mbar_init(&s_free[i], 128);
-      mbar_init(&p_full[i], 128);
+      mbar_init(&s_free[i], 4);
       mbar_init(&pv_done[i], 1);
     }
     *abort_flag = 0;
@@ -140,313 +245,419 @@ __global__ void __launch_bounds__(kThreads, 1)
     tmem_alloc(tmem_slot, p.tmem_cols);
     tmem_relinquish();
   }
+
+  // ---- schedule: this CTA's tile range [r0, r1) in its row block, first sequence -------
+  // The row blocks of a sequence are worked on in lockstep by neighbouring CTAs, so the
+  // second read of every page is served from L2.
+  {
+    int total = 0;
+    for (int b = threadIdx.x; b < p.batch; b += kThreads) {
+      const int Lv = valid_len(p, p.seq_lens[b]);
+      if (Lv == 0 && blockIdx.x == 0 && p.dev_error) atomicOr(p.dev_error, MLA_DEVERR_BOUNDS);
+      total += unit_tiles(Lv);
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) total += __shfl_xor_sync(0xffffffffu, total, o);
+    if (lane == 0) warp_sum[warp] = total;
+    __syncthreads();
+    total = 0;
+#pragma unroll
+    for (int w = 0; w < kThreads / 32; ++w) total += warp_sum[w];
+    const int per = max(1, (total + vgrid - 1) / vgrid);
+    const int r0 = min(total, vc * per);
+    const int r1 = min(total, r0 + per);
+    __syncthreads();
+    if (threadIdx.x == 0) {
+      sched[0] = -1;
+      sched[2] = r0;
+      sched[3] = r1;
+      sched[4] = per;
+      sched[5] = 0;   // running tile count before the current chunk of sequences
+    }
+    __syncthreads();
+    // chunked exclusive scan over the sequences until the one holding tile r0 is found
+    for (int b0 = 0; b0 < p.batch && r0 < r1; b0 += kThreads) {
+      const int b = b0 + threadIdx.x;
+      const int t = b < p.batch ? unit_tiles(valid_len(p, p.seq_lens[b])) : 0;
+      int incl = t;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int y = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += y;
+      }
+      if (lane == 31) warp_sum[warp] = incl;
+      __syncthreads();
+      int before = sched[5];
+      for (int w = 0; w < warp; ++w) before += warp_sum[w];
+      const int start = before + incl - t;
+      if (b < p.batch && start <= r0 && r0 < start + t) {
+        sched[0] = b;
+        sched[1] = start;
+      }
+      __syncthreads();
+      if (threadIdx.x == kThreads - 1) sched[5] = before + incl;
+      __syncthreads();
+      if (sched[0] >= 0) break;
+    }
+  }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
-
-  // ---- work of this CTA: tiles [t0, t0 + ntl) of sequence b --------------------------
-  int L = p.seq_lens[b];
-  const bool len_ok = L >= p.q_len && L <= p.max_seq_len &&
-                      int64_t(L) <= int64_t(p.max_pages) * kDecodeTok;
-  if (!len_ok) {
-    if (threadIdx.x == 0 && p.dev_error) atomicOr(p.dev_error, MLA_DEVERR_BOUNDS);
-    L = 0;
-  }
-  const int n_tiles = (L + kDecodeTok - 1) / kDecodeTok;
-  const int t0 = split * p.tiles_per_split;
-  const int t1 = min(n_tiles, t0 + p.tiles_per_split);
-  const int ntl = t1 > t0 ? t1 - t0 : 0;
+  const int r0 = sched[2], r1 = sched[3], per = sched[4];
+  const bool has_work = sched[0] >= 0 && r0 < r1;
 
   if (warp == 0) {
     // ===================================== TMA producer ==================================
-    if (ntl > 0 && elect_one()) {
+    if (has_work && elect_one()) {
       prefetch_tensormap(&p.tm_cache);
       prefetch_tensormap(&p.tm_q);
-      mbar_arrive_expect_tx(q_full, p.nblk * kQBlk);
-      for (int k = 0; k < p.nblk; ++k)
-        tma_load_3d(q_smem + k * kQBlk, &p.tm_q, k * 64, cg * NCOL, b, q_full);
-      const int32_t* bt = p.block_table + int64_t(b) * p.max_pages;
-      int jj = 0;
-      for (; jj < ntl; ++jj) {
-        const int slot = jj % p.nslot;
-        if (jj >= p.nslot && !mbar_wait(&empty[slot], ((jj / p.nslot) - 1) & 1, wc)) break;
-        int32_t page = bt[t0 + jj];
-        if (page < 0 || page >= p.num_pages) {
-          if (p.dev_error) atomicOr(p.dev_error, MLA_DEVERR_BOUNDS);
-          page = 0;
-        }
-        uint8_t* sbase = slots + slot * p.slot_blocks * kBlkBytes;
-        for (int k = 0; k < p.nblk; ++k) {
-          uint64_t* fb = &full[slot * p.nblk + k];
-          mbar_arrive_expect_tx(fb, kBlkBytes);
-          tma_load_2d(sbase + k * kBlkBytes, &p.tm_cache, k * 64, page * kDecodeTok, fb);
+      if (blockIdx.x == 0) *p.range_len = per;
+      UnitWalk w{sched[0], sched[1]};
+      int jj = 0, pc = 0;
+      bool ok = true;
+      for (; ok && w.s < r1; w.s += w.tiles, ++w.b, ++pc) {
+        w.load(p, cg);
+        p.unit_start[w.u] = w.s;   // same value from every CTA that touches the unit
+        const int tb = max(w.s, r0), te = min(w.s + w.tiles, r1);
+        if (pc > 0 && !mbar_wait(q_empty, (pc - 1) & 1, wc)) { ok = false; break; }
+        mbar_arrive_expect_tx(q_full, p.nblk * kQBlk);
+        for (int k = 0; k < p.nblk; ++k)
+          tma_load_3d(q_smem + k * kQBlk, &p.tm_q, k * 64, cg * NCOL, w.b, q_full);
+        const int32_t* bt = p.block_table + int64_t(w.b) * p.max_pages;
+        for (int t = tb; t < te; ++t, ++jj) {
+          const int slot = jj % p.nslot;
+          if (jj >= p.nslot && !mbar_wait(&empty[slot], ((jj / p.nslot) - 1) & 1, wc)) {
+            ok = false;
+            break;
+          }
+          MLA_TRACE_AT(0, jj);
+          int32_t page = bt[t - w.s];
+          if (page < 0 || page >= p.num_pages) {
+            if (p.dev_error) atomicOr(p.dev_error, MLA_DEVERR_BOUNDS);
+            page = 0;
+          }
+          uint8_t* sbase = slots + slot * slot_bytes;
+          for (int k = 0; k < p.nblk; ++k) {
+            uint64_t* fb = &full[slot * p.nblk + k];
+            mbar_arrive_expect_tx(fb, kBlkBytes);
+            tma_load_2d(sbase + k * kBlkBytes, &p.tm_cache, k * 64, page * kDecodeTok, fb);
+          }
+          MLA_TRACE_AT(8, jj);
         }
       }
       // Drain: never leave while copies into this CTA's shared memory are in flight.
-      mbar_wait_bounded(q_full, 0, 200000000ull);
+      if (pc > 0) mbar_wait_bounded(q_full, (pc - 1) & 1, 200000000ull);
       for (int j = (jj > p.nslot ? jj - p.nslot : 0); j < jj; ++j)
         for (int k = 0; k < p.nblk; ++k)
-          mbar_wait_bounded(&full[(j % p.nslot) * p.nblk + k], (j / p.nslot) & 1,
-                            200000000ull);
+          mbar_wait_bounded(&full[(j % p.nslot) * p.nblk + k], (j / p.nslot) & 1, 200000000ull);
     }
     __syncwarp();
   } else if (warp == 1) {
-    // ===================================== UMMA issuer ===================================
-    if (ntl > 0 && elect_one()) {
+    // ================================ UMMA issuer for S^T ================================
+    // S^T(j) is issued one 64-column block at a time as the blocks land. The PV products
+    // are issued by the softmax warps themselves, the moment P(j) is written.
+    if (has_work && elect_one()) {
       const uint32_t idesc_s = make_idesc_bf16(64, NCOL, 0, 0);
-      const uint32_t idesc_o = make_idesc_bf16(128, NCOL, 1, 1);
-      const uint32_t q_addr = smem_u32(q_smem);
-      const uint32_t slot_addr0 = smem_u32(slots);
-      const uint32_t pt_addr0 = smem_u32(pt);
-      const uint32_t pt_sbo = 8 * NCOL * 2;
-      const SmemSwizzle pt_sw = pt_swizzle(NCOL);
-      bool ok = mbar_wait(q_full, 0, wc);
-
-      auto issue_pv = [&](int t) -> bool {
-        const int pb = t & 1;
-        const int slot = t % p.nslot;
-        if (!mbar_wait(&p_full[pb], (t >> 1) & 1, wc)) return false;
-        tc_fence_after();
-        const uint32_t sa = slot_addr0 + slot * p.slot_blocks * kBlkBytes;
-        const uint32_t pa = pt_addr0 + (t % p.npt) * kPtBytes;
-        for (int c = 0; c < p.nch; ++c) {
-#pragma unroll
-          for (int kk = 0; kk < 4; ++kk) {
-            const uint64_t ad = make_sdesc(sa + 2 * c * kBlkBytes + kk * 2048, kBlkBytes, 1024, kSw128);
-            const uint64_t bd = make_sdesc(pa + kk * 16 * NCOL * 2, kPtBytes, pt_sbo, pt_sw);
-            umma_bf16(tmem + (2 + c) * NCOL, ad, bd, idesc_o, (t > 0 || kk > 0) ? 1u : 0u);
-          }
-        }
-        umma_commit(&pv_done[pb]);
-        umma_commit(&empty[slot]);
-        return true;
-      };
-
-      for (int jj = 0; ok && jj < ntl; ++jj) {
-        const int slot = jj % p.nslot;
-        const int sb = jj & 1;
-        if (jj >= 2 && !mbar_wait(&s_free[sb], ((jj - 2) >> 1) & 1, wc)) { ok = false; break; }
-        tc_fence_after();
-        const uint32_t sa = slot_addr0 + slot * p.slot_blocks * kBlkBytes;
-        for (int k = 0; k < p.nblk; ++k) {
-          if (!mbar_wait(&full[slot * p.nblk + k], (jj / p.nslot) & 1, wc)) { ok = false; break; }
+      const uint64_t a0 = make_sdesc(smem_u32(slots), 16, 1024, kSw128);
+      const uint64_t b0 = make_sdesc(smem_u32(q_smem), 16, 1024, kSw128);
+      UnitWalk w{sched[0], sched[1]};
+      int jj = 0, pc = 0;
+      bool ok = true;
+      for (; ok && w.s < r1; w.s += w.tiles, ++w.b, ++pc) {
+        w.load(p, cg);
+        const int tb = max(w.s, r0), te = min(w.s + w.tiles, r1);
+        if (!mbar_wait(q_full, pc & 1, wc)) { ok = false; break; }
+        for (int t = tb; ok && t < te; ++t, ++jj) {
+          const int slot = jj % p.nslot;
+          const int sb = jj & 1;
+          if (jj >= 2 && !mbar_wait(&s_free[sb], ((jj - 2) >> 1) & 1, wc)) { ok = false; break; }
           tc_fence_after();
-          const int rem = p.D - k * 64;
-          const int nkk = rem >= 64 ? 4 : (rem + 15) / 16;
-          for (int kk = 0; kk < nkk; ++kk) {
-            const uint64_t ad = make_sdesc(sa + k * kBlkBytes + kk * 32, 16, 1024, kSw128);
-            const uint64_t bd = make_sdesc(q_addr + k * kQBlk + kk * 32, 16, 1024, kSw128);
-            umma_bf16(tmem + sb * NCOL, ad, bd, idesc_s, (k | kk) != 0 ? 1u : 0u);
+          const uint32_t soff = slot * slot_bytes;
+          for (int k = 0; k < p.nblk; ++k) {
+            if (!mbar_wait(&full[slot * p.nblk + k], (jj / p.nslot) & 1, wc)) { ok = false; break; }
+            tc_fence_after();
+            if (k == 0) MLA_TRACE_AT(9, jj);
+            const int rem = p.D - k * 64;
+            const int nkk = rem >= 64 ? 4 : (rem + 15) / 16;
+            for (int kk = 0; kk < nkk; ++kk) {
+              const uint64_t ad = a0 + ((soff + k * kBlkBytes + kk * 32) >> 4);
+              const uint64_t bd = b0 + ((k * kQBlk + kk * 32) >> 4);
+              umma_bf16(tmem + sb * NCOL, ad, bd, idesc_s, (k | kk) != 0 ? 1u : 0u);
+            }
           }
+          if (!ok) break;
+          MLA_TRACE_AT(1, jj);
+          umma_commit(&s_full[sb]);
+          MLA_TRACE_AT(2, jj);
+          if (t == te - 1) umma_commit(q_empty);   // this piece's Q is no longer read
         }
-        if (!ok) break;
-        umma_commit(&s_full[sb]);
-        if (jj >= 1 && !issue_pv(jj - 1)) { ok = false; break; }
       }
-      if (ok) issue_pv(ntl - 1);
     }
     __syncwarp();
-  } else {
-    // ================================ softmax + epilogue =================================
+  } else if (has_work) {
+    // ============================ softmax, PV issue, epilogue ============================
     const int sp = warp & 3;                  // TMEM sub-partition this warp may access
     const int wi = warp - 2;                  // index among the 4 softmax warps
+    const int tid = threadIdx.x - 64;         // 0..127
     const uint32_t lane_base = uint32_t(sp * 32) << 16;
-    const bool has_tok = lane < 16;
-    const int tok = 16 * sp + lane;           // token of this lane inside the tile
-    const int qH = p.qH;
-    const int last_pos = L - p.q_len;         // position of query row 0
-    float l_part[NCOL];
-#pragma unroll
-    for (int n = 0; n < NCOL; ++n) l_part[n] = 0.0f;
-    if (threadIdx.x - 64 < NCOL) m_ref[threadIdx.x - 64] = -INFINITY;
-    named_bar_sync(1, 128);
+    const int tok = 16 * sp + (lane & 15);    // token of this thread inside the tile
+    const int hf = lane >> 4;                 // which half of the columns
+    const int c0 = hf * HALF;                 // first column of this thread
+    const bool col_owner = (lane & 15) == 0;  // publishes its half-warp's column values
+    const float c_log2 = p.scale_log2;
+    // PV operands: C^T of the tile (MN-major) and P^T (MN-major), advanced by offsets
+    const uint32_t idesc_o = make_idesc_bf16(128, NCOL, 1, 1);
+    const uint64_t pa0 = make_sdesc(smem_u32(slots), kBlkBytes, 1024, kSw128);
+    const uint64_t pb0 = make_sdesc(smem_u32(pt), kPtBytes, 8 * NCOL * 2, pt_swizzle(NCOL));
 
-    for (int jj = 0; jj < ntl; ++jj) {
-      const int sb = jj & 1;
-      const int tile = t0 + jj;
-      // warp-uniform: the TMEM load below is a warp-collective instruction
-      const bool got = __all_sync(0xffffffffu, mbar_wait(&s_full[sb], (jj >> 1) & 1, wc));
-      float s[NCOL];
-      if (got) {
-        tc_fence_after();
-        tmem_ld_cols<NCOL>(tmem + lane_base + sb * NCOL, s);
-        tmem_wait_ld();
+    UnitWalk w{sched[0], sched[1]};
+    int jj = 0;
+    for (; w.s < r1; w.s += w.tiles, ++w.b) {
+      w.load(p, cg);
+      const int tb = max(w.s, r0), te = min(w.s + w.tiles, r1);
+      const int L = w.L;
+      const int last_full = p.causal ? L - p.q_len : L - 1;  // last position every row sees
+      float m[HALF], l[HALF];
+#pragma unroll
+      for (int j = 0; j < HALF; ++j) {
+        m[j] = kRefInit;
+        l[j] = 0.0f;
       }
-      tc_fence_before();
-      mbar_arrive(&s_free[sb]);
-
-      const int pos = tile * kDecodeTok + tok;
-      const bool tok_ok = got && has_tok && pos < L;
-      bool exceed = false;
-#pragma unroll
-      for (int n = 0; n < NCOL; ++n) {
-        const int f = cg * NCOL + n;
-        const int qi = f / p.num_heads;
-        const bool vis = tok_ok && f < qH && (!p.causal || pos <= last_pos + qi);
-        s[n] = vis ? s[n] * p.scale_log2 : -INFINITY;
-        exceed |= s[n] > m_ref[n] + kLazyThreshold;
-      }
-      exceed = __any_sync(0xffffffffu, exceed);
-      if (lane == 0) flags[(jj & 1) * 4 + wi] = exceed ? 1 : 0;
-      named_bar_sync(1, 128);
-      const bool upd = (flags[(jj & 1) * 4 + 0] | flags[(jj & 1) * 4 + 1] |
-                        flags[(jj & 1) * 4 + 2] | flags[(jj & 1) * 4 + 3]) != 0;
-      if (upd) {
-        // tile max per query row across the 64 tokens (16 lanes x 4 warps)
-        float tmax[NCOL];
-#pragma unroll
-        for (int n = 0; n < NCOL; ++n) {
-          float v = s[n];
-          v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, 8));
-          v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, 4));
-          v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, 2));
-          v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, 1));
-          tmax[n] = v;
+      for (int t = tb; t < te; ++t, ++jj) {
+        const int sb = jj & 1;
+        const uint32_t s_addr = tmem + lane_base + sb * NCOL;
+        const bool got = __all_sync(0xffffffffu, mbar_wait(&s_full[sb], (jj >> 1) & 1, wc));
+        if (threadIdx.x == 64) MLA_TRACE_AT(4, jj);
+        const int tile_pos0 = (t - w.s) * kDecodeTok;
+        const int pos = tile_pos0 + tok;
+        const bool ragged = !got || tile_pos0 + kDecodeTok - 1 > last_full;
+        // tt = s * c - m: the scaled score against the current reference (in place)
+        float tt[HALF];
+        if (got) {
+          tc_fence_after();
+          tmem_ld_s<HALF>(s_addr, tt);
+          tmem_wait_ld();
         }
-        if (lane == 0) {
+        if (ragged) {
+          // row (i, h) sees token pos iff pos < L and (causal) pos <= L - q + i
 #pragma unroll
-          for (int n = 0; n < NCOL; ++n) red[wi * 64 + n] = tmax[n];
-        }
-        named_bar_sync(1, 128);
-        float alpha[NCOL];
-        bool rescale = false;
-#pragma unroll
-        for (int n = 0; n < NCOL; ++n) {
-          const float mo = m_ref[n];
-          const float mn = fmaxf(fmaxf(mo, red[n]),
-                                 fmaxf(fmaxf(red[64 + n], red[128 + n]), red[192 + n]));
-          alpha[n] = (mo == -INFINITY) ? 0.0f : ex2_approx(mo - mn);
-          rescale |= (mo != -INFINITY) && (mn != mo);
-          tmax[n] = mn;
-          l_part[n] *= alpha[n];
-        }
-        if (rescale && jj > 0) {
-          // O^T holds tiles < jj: wait for the last of them, then scale its columns
-          if (__all_sync(0xffffffffu, mbar_wait(&pv_done[(jj - 1) & 1], ((jj - 1) >> 1) & 1, wc))) {
-            tc_fence_after();
-            for (int c = 0; c < p.nch; ++c) {
-              float o[NCOL];
-              const uint32_t ta = tmem + lane_base + (2 + c) * NCOL;
-              tmem_ld_cols<NCOL>(ta, o);
-              tmem_wait_ld();
-#pragma unroll
-              for (int n = 0; n < NCOL; ++n) o[n] *= alpha[n];
-              tmem_st_cols<NCOL>(ta, o);
-            }
-            tmem_wait_st();
+          for (int j = 0; j < HALF; ++j) {
+            const int qi = (cg * NCOL + c0 + j) / p.num_heads;
+            const bool vis = got && pos < L && (!p.causal || pos <= L - p.q_len + qi);
+            tt[j] = vis ? tt[j] : -INFINITY;
           }
         }
-        named_bar_sync(1, 128);
-        if (threadIdx.x - 64 < NCOL) {
-          float v = -INFINITY;
+        float tmax = -INFINITY;
 #pragma unroll
-          for (int n = 0; n < NCOL; ++n) v = (n == int(threadIdx.x) - 64) ? tmax[n] : v;
-          m_ref[threadIdx.x - 64] = v;
+        for (int j = 0; j < HALF; ++j) {
+          tt[j] = fmaf(tt[j], c_log2, -m[j]);
+          tmax = fmaxf(tmax, tt[j]);
         }
+        const bool exceed = __any_sync(0xffffffffu, tmax > kLazyThreshold);
+        if (lane == 0) flags[(jj & 1) * 4 + wi] = exceed ? 1 : 0;
         named_bar_sync(1, 128);
-      }
+        if (threadIdx.x == 64) MLA_TRACE_AT(5, jj);
+        const int* fl = flags + (jj & 1) * 4;
+        if ((fl[0] | fl[1] | fl[2] | fl[3]) != 0) {
+          // Move the reference to the running column max of the scaled scores; the raw
+          // scores are read again from TMEM (the S buffer is released only below).
+          float s[HALF];
+          if (got) {
+            tmem_ld_s<HALF>(s_addr, s);
+            tmem_wait_ld();
+          }
+#pragma unroll
+          for (int j = 0; j < HALF; ++j) {
+            if (ragged) {
+              const int qi = (cg * NCOL + c0 + j) / p.num_heads;
+              const bool vis = got && pos < L && (!p.causal || pos <= L - p.q_len + qi);
+              s[j] = vis ? s[j] : -INFINITY;
+            }
+            float v = s[j] * c_log2;   // -inf stays -inf
+            v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, 8));
+            v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, 4));
+            v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, 2));
+            v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, 1));
+            if (col_owner) red[wi * 64 + c0 + j] = v;
+          }
+          named_bar_sync(1, 128);
+          bool chg = false;
+#pragma unroll
+          for (int j = 0; j < HALF; ++j) {
+            const int n = c0 + j;
+            const float tm = fmaxf(fmaxf(red[n], red[64 + n]), fmaxf(red[128 + n], red[192 + n]));
+            const float mn = fmaxf(m[j], tm);
+            const float a = ex2_approx(m[j] - mn);   // 0 while m is still kRefInit
+            l[j] *= a;
+            m[j] = mn;
+            tt[j] = fmaf(s[j], c_log2, -mn);
+            chg |= a != 1.0f;
+            if (col_owner && wi == 0) alpha_s[n] = a;
+          }
+          if (col_owner && wi == 0) chg_flag[hf] = chg ? 1 : 0;
+          named_bar_sync(1, 128);
+          if (t > tb && (chg_flag[0] | chg_flag[1]) != 0) {
+            // O^T already holds this piece's earlier tiles: scale every column of the
+            // latent rows this thread owns (all threads see the same factors)
+            const bool okw = __all_sync(0xffffffffu,
+                                        mbar_wait(&pv_done[(jj - 1) & 1], ((jj - 1) >> 1) & 1, wc));
+            if (okw) {
+              tc_fence_after();
+#pragma unroll 1
+              for (int n0 = 0; n0 < NCOL; n0 += 16) {
+                float a16[16];
+#pragma unroll
+                for (int n = 0; n < 16; ++n) a16[n] = alpha_s[n0 + n];
+                for (int c = 0; c < p.nch; ++c) {
+                  const uint32_t ta = tmem + lane_base + (2 + c) * NCOL + n0;
+                  float o[16];
+                  tmem_ld16(ta, o);
+                  tmem_wait_ld();
+#pragma unroll
+                  for (int n = 0; n < 16; ++n) o[n] *= a16[n];
+                  tmem_st16(ta, o);
+                }
+              }
+              tmem_wait_st();
+            }
+          }
+        }
 
-      // unnormalised weights p = 2^(s - m_ref), bf16, into the P^T buffer of this tile;
-      // the buffer is free once the PV product that last read it has completed
-      if (jj >= p.npt) mbar_wait(&pv_done[(jj - p.npt) & 1], ((jj - p.npt) >> 1) & 1, wc);
-      uint32_t packed[NCOL / 2];
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&s_free[sb]);   // S buffer may be overwritten now
+
+        // unnormalised weights p = 2^(s*c - m) into this tile's P^T buffer (bf16)
+        if (jj >= p.npt) mbar_wait(&pv_done[(jj - p.npt) & 1], ((jj - p.npt) >> 1) & 1, wc);
+        if (threadIdx.x == 64) MLA_TRACE_AT(6, jj);
+        uint32_t packed[HALF / 2];
 #pragma unroll
-      for (int n = 0; n < NCOL; n += 2) {
-        const float p0 = s[n] == -INFINITY ? 0.0f : ex2_approx(s[n] - m_ref[n]);
-        const float p1 = s[n + 1] == -INFINITY ? 0.0f : ex2_approx(s[n + 1] - m_ref[n + 1]);
-        l_part[n] += p0;
-        l_part[n + 1] += p1;
-        packed[n / 2] = cvt_bf16x2(p0, p1);
-      }
-      if (has_tok) {
-        uint8_t* row = pt + (jj % p.npt) * kPtBytes;
-        constexpr uint32_t kRowBytes = NCOL * 2;
-        constexpr uint32_t kChunkMask = kRowBytes / 16 - 1;
+        for (int j = 0; j < HALF; j += 2) {
+          const float p0 = ex2_approx(tt[j]);
+          const float p1 = ex2_approx(tt[j + 1]);
+          l[j] += p0;
+          l[j + 1] += p1;
+          packed[j / 2] = cvt_bf16x2(p0, p1);
+        }
+        const int slot = jj % p.nslot;
+        const int pbuf = jj % p.npt;
+        {
+          uint8_t* buf = pt + pbuf * kPtBytes;
+          constexpr uint32_t kRowBytes = NCOL * 2;
+          constexpr uint32_t kChunkMask = kRowBytes / 16 - 1;
 #pragma unroll
-        for (int ch = 0; ch < NCOL / 8; ++ch) {
-          const uint32_t off = tok * kRowBytes + ch * 16;
-          const uint32_t phys = off ^ (((off >> 7) & kChunkMask) << 4);
-          *reinterpret_cast<uint4*>(row + phys) =
-              make_uint4(packed[ch * 4 + 0], packed[ch * 4 + 1], packed[ch * 4 + 2], packed[ch * 4 + 3]);
+          for (int ch = 0; ch < HALF / 8; ++ch) {
+            const uint32_t off = tok * kRowBytes + (hf * (HALF / 8) + ch) * 16;
+            const uint32_t phys = off ^ (((off >> 7) & kChunkMask) << 4);
+            *reinterpret_cast<uint4*>(buf + phys) = make_uint4(
+                packed[ch * 4 + 0], packed[ch * 4 + 1], packed[ch * 4 + 2], packed[ch * 4 + 3]);
+          }
         }
         // cache rows past the context may hold anything (even NaN): zero them so that
         // 0-weight x garbage cannot reach O^T
-        if (tile == n_tiles - 1 && pos >= L) {
-          uint8_t* sbase = slots + (jj % p.nslot) * p.slot_blocks * kBlkBytes;
-          for (int k = 0; k < 2 * p.nch; ++k) {
+        if (pos >= L) {
+          uint8_t* sbase = slots + slot * slot_bytes;
+          for (int k = hf; k < 2 * p.nch; k += 2) {
             uint4* rowp = reinterpret_cast<uint4*>(sbase + k * kBlkBytes + tok * 128);
 #pragma unroll
             for (int ch = 0; ch < 8; ++ch) rowp[ch] = make_uint4(0, 0, 0, 0);
           }
         }
-      }
-      fence_proxy_async_smem();
-      tc_fence_before();
-      mbar_arrive(&p_full[sb]);
-    }
-
-    // ---------------------------------- epilogue ------------------------------------------
-    bool fin = true;
-    if (ntl > 0) {
-      fin = __all_sync(0xffffffffu, mbar_wait(&pv_done[(ntl - 1) & 1], ((ntl - 1) >> 1) & 1, wc));
-      tc_fence_after();
-    }
+        fence_proxy_async_smem();
+        tc_fence_before();
+        named_bar_sync(1, 128);
+        if (threadIdx.x == 64) {
+          // O^T += C^T P^T for this tile; the first tile of a piece overwrites O^T (the
+          // previous piece's epilogue reads finished before the barrier above)
+          MLA_TRACE_AT(7, jj);
+          tc_fence_after();
+          const bool first = (t == tb);
+          const uint32_t soff = slot * slot_bytes;
+          const uint32_t poff = pbuf * kPtBytes;
+          // K-step outer, latent chunk inner: consecutive MMAs feed different accumulators
 #pragma unroll
-    for (int n = 0; n < NCOL; ++n) {
-      float v = l_part[n];
-      v += __shfl_xor_sync(0xffffffffu, v, 8);
-      v += __shfl_xor_sync(0xffffffffu, v, 4);
-      v += __shfl_xor_sync(0xffffffffu, v, 2);
-      v += __shfl_xor_sync(0xffffffffu, v, 1);
-      l_part[n] = v;
-    }
-    if (lane == 0) {
-#pragma unroll
-      for (int n = 0; n < NCOL; ++n) red[wi * 64 + n] = l_part[n];
-    }
-    named_bar_sync(1, 128);
-    float inv_l[NCOL];
-#pragma unroll
-    for (int n = 0; n < NCOL; ++n) {
-      const float l = red[n] + red[64 + n] + red[128 + n] + red[192 + n];
-      inv_l[n] = l > 0.0f ? 1.0f / l : 0.0f;
-    }
-    const bool aborted = __any_sync(0xffffffffu, !fin || *abort_flag != 0);
-    const int cols_here = min(NCOL, qH - cg * NCOL);
-    const int64_t part_base = (int64_t(b) * p.col_groups + cg) * p.splits + split;
-    // lse (natural log) of each query row
-    const int tid = threadIdx.x - 64;
-    if (tid < cols_here) {
-      const float l = red[tid] + red[64 + tid] + red[128 + tid] + red[192 + tid];
-      const float v = (l > 0.0f && !aborted) ? (m_ref[tid] + __log2f(l)) * kLn2 : -INFINITY;
-      if (p.splits == 1) p.lse[int64_t(b) * qH + cg * NCOL + tid] = v;
-      else p.part_lse[part_base * NCOL + tid] = v;
-    }
-    // O^T: this thread owns latent row 128*c + 32*sp + lane of every chunk c
-    for (int c = 0; c < p.nch; ++c) {
-      float o[NCOL];
-      if (ntl > 0 && !aborted) {
-        tmem_ld_cols<NCOL>(tmem + lane_base + (2 + c) * NCOL, o);
-        tmem_wait_ld();
-      } else {
-#pragma unroll
-        for (int n = 0; n < NCOL; ++n) o[n] = 0.0f;
-      }
-      const int lat = 128 * c + 32 * sp + lane;
-      if (lat < p.r) {
-        if (p.splits == 1) {
-          uint16_t* dst = p.o_latent + (int64_t(b) * qH + cg * NCOL) * p.r + lat;
-#pragma unroll
-          for (int n = 0; n < NCOL; ++n)
-            if (n < cols_here) dst[int64_t(n) * p.r] = f32_to_bf16_rne(o[n] * inv_l[n]);
-        } else {
-          float* dst = p.part_o + part_base * NCOL * p.r + lat;
-#pragma unroll
-          for (int n = 0; n < NCOL; ++n)
-            if (n < cols_here) dst[int64_t(n) * p.r] = o[n] * inv_l[n];
+          for (int kk = 0; kk < 4; ++kk) {
+            const uint64_t bd = pb0 + ((poff + kk * 16 * NCOL * 2) >> 4);
+            for (int c = 0; c < p.nch; ++c) {
+              const uint64_t ad = pa0 + ((soff + 2 * c * kBlkBytes + kk * 2048) >> 4);
+              umma_bf16(tmem + (2 + c) * NCOL, ad, bd, idesc_o, (!first || kk > 0) ? 1u : 0u);
+            }
+          }
+          umma_commit(&pv_done[jj & 1]);
+          umma_commit(&empty[slot]);
+          MLA_TRACE_AT(3, jj);
         }
       }
+
+      // ---------------------------- epilogue of this piece --------------------------------
+      const bool fin = __all_sync(0xffffffffu,
+                                  mbar_wait(&pv_done[(jj - 1) & 1], ((jj - 1) >> 1) & 1, wc));
+      tc_fence_after();
+#pragma unroll
+      for (int j = 0; j < HALF; ++j) {
+        float v = l[j];
+        v += __shfl_xor_sync(0xffffffffu, v, 8);
+        v += __shfl_xor_sync(0xffffffffu, v, 4);
+        v += __shfl_xor_sync(0xffffffffu, v, 2);
+        v += __shfl_xor_sync(0xffffffffu, v, 1);
+        l[j] = v;
+      }
+      named_bar_sync(1, 128);   // every earlier reader of red / mref_s is done
+      if (col_owner) {
+#pragma unroll
+        for (int j = 0; j < HALF; ++j) red[wi * 64 + c0 + j] = l[j];
+      }
+      if (col_owner && wi == 0) {
+#pragma unroll
+        for (int j = 0; j < HALF; ++j) mref_s[c0 + j] = m[j];
+      }
+      named_bar_sync(1, 128);
+      const bool aborted = __any_sync(0xffffffffu, !fin || *abort_flag != 0);
+      const bool whole = (tb == w.s) && (te == w.s + w.tiles);
+      const int cols_here = min(NCOL, p.qH - cg * NCOL);
+      const int64_t row0 = int64_t(w.b) * p.qH + int64_t(cg) * NCOL;   // first (b, i, h) row
+      const int pslot = piece_slot(vc, w.s, per, p.col_groups, cg);
+      if (tid < cols_here) {
+        const float sum = red[tid] + red[64 + tid] + red[128 + tid] + red[192 + tid];
+        const float lse = (sum > 0.0f && !aborted) ? (mref_s[tid] + __log2f(sum)) * kLn2 : -INFINITY;
+        if (whole) p.lse[row0 + tid] = lse;
+        else p.part_lse[int64_t(pslot) * NCOL + tid] = lse;
+      }
+      // O^T: this thread owns latent row 128*c + 32*sp + lane of every chunk c
+#pragma unroll 1
+      for (int n0 = 0; n0 < NCOL; n0 += 16) {
+        float inv[16];
+#pragma unroll
+        for (int n = 0; n < 16; ++n) {
+          const int col = n0 + n;
+          const float sum = red[col] + red[64 + col] + red[128 + col] + red[192 + col];
+          inv[n] = sum > 0.0f ? 1.0f / sum : 0.0f;
+        }
+        for (int c = 0; c < p.nch; ++c) {
+          const int lat = 128 * c + 32 * sp + lane;
+          float o[16];
+          if (!aborted) {
+            tmem_ld16(tmem + lane_base + (2 + c) * NCOL + n0, o);
+            tmem_wait_ld();
+          } else {
+#pragma unroll
+            for (int n = 0; n < 16; ++n) o[n] = 0.0f;
+          }
+          if (lat < p.r) {
+#pragma unroll
+            for (int n = 0; n < 16; ++n) {
+              const int col = n0 + n;
+              if (col < cols_here) {
+                const float v = o[n] * inv[n];
+                if (whole) p.o_latent[(row0 + col) * p.r + lat] = f32_to_bf16_rne(v);
+                else p.part_o[(int64_t(pslot) * NCOL + col) * p.r + lat] = v;
+              }
+            }
+          }
+        }
+      }
+      tc_fence_before();
     }
   }
 
@@ -455,31 +666,81 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (warp == 1) tmem_dealloc(tmem, p.tmem_cols);
 }
 
-// ---- split merge: lse = log sum_s e^{lse_s}, o = sum_s e^{lse_s - lse} o_s ---------------
-__global__ void __launch_bounds__(128) mla_combine_kernel(CombineParams p) {
-  const int f = blockIdx.x;   // query row (i, h) of sequence b
-  const int b = blockIdx.y;
-  const int cg = f / p.ncol;
-  const int n = f % p.ncol;
-  const int64_t base = (int64_t(b) * p.col_groups + cg) * p.splits;
-  float mx = -INFINITY;
-  for (int s = 0; s < p.splits; ++s) mx = fmaxf(mx, p.part_lse[(base + s) * p.ncol + n]);
-  float wsum = 0.0f;
-  for (int s = 0; s < p.splits; ++s) {
-    const float ls = p.part_lse[(base + s) * p.ncol + n];
-    wsum += ls == -INFINITY ? 0.0f : expf(ls - mx);
-  }
-  const float lse = mx == -INFINITY ? -INFINITY : mx + logf(wsum);
-  if (threadIdx.x == 0) p.lse[int64_t(b) * p.qH + f] = lse;
-  for (int c = threadIdx.x; c < p.r; c += blockDim.x) {
-    float acc = 0.0f;
-    for (int s = 0; s < p.splits; ++s) {
-      const float ls = p.part_lse[(base + s) * p.ncol + n];
-      if (ls == -INFINITY) continue;
-      acc += expf(ls - lse) * p.part_o[((base + s) * p.ncol + n) * p.r + c];
+// ---- merge of cut units: lse = log sum_i e^{lse_i}, o = sum_i e^{lse_i - lse} o_i ------
+// Grid-stride over items (unit, query row, 128-latent chunk); 4 warps split the pieces,
+// each lane owns 4 latents of the chunk, and the warps' sums meet in shared memory.
+__global__ void __launch_bounds__(128) mla_combine_kernel(const CombineParams p) {
+  __shared__ float part[4][128];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int per = *p.range_len;
+  const int nchunk = (p.r + 127) / 128;
+  const int64_t items = int64_t(p.units) * p.ncol * nchunk;
+  for (int64_t it = blockIdx.x; it < items; it += gridDim.x) {
+    const int u = int(it / (p.ncol * nchunk));
+    const int rem = int(it - int64_t(u) * p.ncol * nchunk);
+    const int n = rem / nchunk, ch = rem - n * nchunk;
+    const int b = u / p.col_groups, cg = u - b * p.col_groups;
+    const int f = cg * p.ncol + n;
+    const int G = p.col_groups;
+    if (f >= p.qH) continue;
+    int L = p.seq_lens[b];
+    const bool ok = L >= p.q_len && L <= p.max_seq_len && int64_t(L) <= int64_t(p.max_pages) * kDecodeTok;
+    if (!ok) L = 0;
+    const int tiles = L > 0 ? (L + kDecodeTok - 1) / kDecodeTok : 1;
+    const int s = p.unit_start[u];
+    const int i0 = s / per, i1 = (s + tiles - 1) / per;
+    if (i0 == i1) continue;   // held whole by one CTA: already written
+    float mx = -INFINITY;
+    for (int i = i0 + lane; i <= i1; i += 32)
+      mx = fmaxf(mx, p.part_lse[int64_t(piece_slot(i, s, per, G, cg)) * p.ncol + n]);
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+    float den = 0.0f;
+    for (int i = i0 + lane; i <= i1; i += 32) {
+      const float li = p.part_lse[int64_t(piece_slot(i, s, per, G, cg)) * p.ncol + n];
+      den += li == -INFINITY ? 0.0f : expf(li - mx);
     }
-    p.o_latent[(int64_t(b) * p.qH + f) * p.r + c] = f32_to_bf16_rne(acc);
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) den += __shfl_xor_sync(0xffffffffu, den, o);
+    const float lse = mx == -INFINITY ? -INFINITY : mx + logf(den);
+    float acc[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+    for (int i = i0 + warp; i <= i1; i += 4) {
+      const int64_t sl = piece_slot(i, s, per, G, cg);
+      const float li = p.part_lse[sl * p.ncol + n];
+      if (li == -INFINITY) continue;
+      const float wgt = expf(li - lse);
+      const float* row = p.part_o + (sl * p.ncol + n) * p.r + ch * 128;
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        const int lat = lane + 32 * k;
+        if (ch * 128 + lat < p.r) acc[k] += wgt * row[lat];
+      }
+    }
+#pragma unroll
+    for (int k = 0; k < 4; ++k) part[warp][lane + 32 * k] = acc[k];
+    __syncthreads();
+    {
+      const int lat = threadIdx.x;
+      if (ch * 128 + lat < p.r) {
+        const float v = part[0][lat] + part[1][lat] + part[2][lat] + part[3][lat];
+        p.o_latent[(int64_t(b) * p.qH + f) * p.r + ch * 128 + lat] = f32_to_bf16_rne(v);
+      }
+      if (threadIdx.x == 0 && ch == 0) p.lse[int64_t(b) * p.qH + f] = lse;
+    }
+    __syncthreads();
   }
+}
+
+#ifdef MLA_TRACE
+extern "C" int mla_trace_read(unsigned long long* host, int n) {
+  return int(cudaMemcpyFromSymbol(host, g_mla_trace, sizeof(unsigned long long) *
+                                  size_t(n < 10 * kTraceTiles ? n : 10 * kTraceTiles)));
+}
+#endif
+
+cudaError_t launch_combine(const CombineParams& p, int grid, cudaStream_t stream) {
+  mla_combine_kernel<<<grid, 128, 0, stream>>>(p);
+  return cudaGetLastError();
 }
 
 template <int NCOL>
@@ -500,12 +761,6 @@ cudaError_t launch_decode(const DecodeParams& p, int ncol, dim3 grid, size_t sme
     case 64: return launch_decode_n<64>(p, grid, smem, stream);
     default: return cudaErrorInvalidValue;
   }
-}
-
-cudaError_t launch_combine(const CombineParams& p, cudaStream_t stream) {
-  dim3 grid(p.qH, p.batch);
-  mla_combine_kernel<<<grid, 128, 0, stream>>>(p);
-  return cudaGetLastError();
 }
 
 }  // namespace mla

@@ -54,25 +54,31 @@ struct DecodeParams {
   const int32_t* seq_lens;
   uint16_t* o_latent;        // [B, q, H, r]
   float* lse;                // [B, q, H]
-  float* part_o;             // [B, CG, S, NCOL, r]  (splits > 1)
-  float* part_lse;           // [B, CG, S, NCOL]
+  float* part_o;             // [grid, 2, NCOL, r]  partial outputs of cut units
+  float* part_lse;           // [grid, 2, NCOL]
+  int32_t* unit_start;       // [units] first tile of each unit in its row block (for the merge)
+  int32_t* range_len;        // [1] tiles per CTA range (for the merge)
   int32_t* dev_error;
   int64_t num_pages;
-  int32_t max_pages, batch, q_len, num_heads, qH, r, D, nblk, nch, col_groups, splits,
-      tiles_per_split, max_seq_len, causal, nslot, slot_blocks, tmem_cols, npt;
+  int32_t max_pages, batch, q_len, num_heads, qH, r, D, nblk, nch, col_groups, units,
+      max_seq_len, causal, nslot, slot_blocks, tmem_cols, npt;
   float scale_log2;          // softmax_scale * log2(e)
 };
 size_t decode_smem_bytes(int ncol, int nblk, int slot_blocks, int nslot, int npt);
 cudaError_t launch_decode(const DecodeParams& p, int ncol, dim3 grid, size_t smem,
                           cudaStream_t stream);
 
+// Merge of the per-piece partials of units cut between CTAs (log-sum-exp identity).
 struct CombineParams {
   const float* part_o;
   const float* part_lse;
+  const int32_t* unit_start;
+  const int32_t* range_len;
+  const int32_t* seq_lens;
   uint16_t* o_latent;
   float* lse;
-  int32_t batch, qH, r, ncol, col_groups, splits;
+  int32_t q_len, max_seq_len, max_pages, qH, r, ncol, col_groups, units;
 };
-cudaError_t launch_combine(const CombineParams& p, cudaStream_t stream);
+cudaError_t launch_combine(const CombineParams& p, int grid, cudaStream_t stream);
 
 }  // namespace mla

@@ -125,9 +125,11 @@ mla_status mla_absorb_q(const mla_dims* dims, const void* q_nope, const void* q_
 
 /*
  * Bytes of workspace mla_decode_attn needs for this problem (0 on invalid input).
- * num_splits: KV splits per sequence, 0 = let the library choose. The first 256 bytes
- * of the workspace hold the device error word (int32 at offset 0): zero them once
- * after allocating. The rest is scratch the library overwrites on every call.
+ * num_splits: 0 lets the library size the grid (one CTA per SM); n > 0 asks for n
+ * equal work ranges per (sequence, block of query rows) on average. The workspace holds
+ * the device error word (int32 at offset 0; zero it once after allocating), the
+ * schedule and the partial results of sequences cut between CTAs. A workspace can be
+ * reused by later calls on the same stream, not by calls running concurrently.
  */
 size_t mla_decode_workspace_size(const mla_dims* dims, int32_t batch, int32_t q_len,
                                  int32_t max_seq_len, int32_t num_splits);
@@ -143,8 +145,9 @@ size_t mla_decode_workspace_size(const mla_dims* dims, int32_t batch, int32_t q_
  * groups' rotary slots), p = softmax over l, and writes
  *     o_latent[b,i,h,:] = sum_l p * c_kv[l]      (einsum 4, bf16)
  *     lse[b,i,h]        = ln sum_l exp(s)        (fp32)
- * Long contexts are split across CTAs; the per-split results are merged with the
- * log-sum-exp identity.
+ * The cached pages of all sequences are cut into equal ranges, one per CTA, so ragged
+ * lengths balance; a sequence cut between CTAs is merged with the log-sum-exp identity
+ * by a second, small kernel launched right after.
  *
  *   q_ext       bf16 [B, q, H, D]   from mla_absorb_q
  *   cache       bf16 [num_pages, ps, D]

@@ -43,9 +43,28 @@ class GpuProblem:
 
         c_new = torch.empty((B, q, r), dtype=torch.bfloat16)
         k_new = torch.empty((B, q, G, dr), dtype=torch.bfloat16)
-        for b in range(B):
+        lens = [int(L) for L in wl.seq_lens]
+        # uniform lengths: one batched append (few launches); ragged: one per sequence
+        batched = len(set(lens)) == 1 and lens[0] > q and B * lens[0] * D * 2 <= (2 << 30)
+        if batched:
+            n = lens[0] - q
+            ctx = [wl.context(b) for b in range(B)]
+            cos, sin = wl.rope_table(np.arange(n))
+            cos = np.broadcast_to(cos[None], (B,) + cos.shape)
+            sin = np.broadcast_to(sin[None], (B,) + sin.shape)
+            mla.mla_cache_append(self.dims, torch.stack([c[:n] for c, _ in ctx]).to(dev),
+                                 torch.stack([k[:n] for _, k in ctx]).to(dev),
+                                 torch.from_numpy(np.ascontiguousarray(cos)).to(dev),
+                                 torch.from_numpy(np.ascontiguousarray(sin)).to(dev),
+                                 self.block_table, torch.zeros(B, dtype=torch.int32, device=dev),
+                                 self.cache, dev_error=self.err)
+            for b, (c_kv, k_r) in enumerate(ctx):
+                c_new[b] = c_kv[n:n + q]
+                k_new[b] = k_r[n:n + q]
+            del ctx
+        for b in range(0 if not batched else B, B):
             c_kv, k_r = wl.context(b)
-            L = int(wl.seq_lens[b])
+            L = lens[b]
             n = L - q
             if n > 0:
                 cos, sin = wl.rope_table(np.arange(n))

@@ -96,17 +96,20 @@ def test_decode_validation(mla_lib):
     assert _decode(_dims(), lens=None) == mla.MLA_ERR_INVALID_ARG
     assert _decode(_dims(), ws=None) == mla.MLA_ERR_WORKSPACE
     assert _decode(_dims(), ws=P(0x10010)) == mla.MLA_ERR_WORKSPACE          # not 256-aligned
-    assert _decode(_dims(), splits=4, wsb=256) == mla.MLA_ERR_WORKSPACE       # partials need room
+    assert _decode(_dims(), splits=4, wsb=4096) == mla.MLA_ERR_WORKSPACE      # partials need room
     assert _decode(_dims(), batch=0) == mla.MLA_OK
 
 
 def test_workspace_size(mla_lib):
     d = _dims()
     ws = lambda *a: mla.mla_decode_workspace_size(d, *a)  # noqa: E731
-    assert ws(64, 1, 8192, 1) == 256                    # one split: only the error word
-    # 4 splits, 2 column groups of 64 rows, 64 sequences: lse + fp32 partial outputs
-    rows = 64 * 2 * 4 * 64
-    assert ws(64, 1, 8192, 4) == 256 + (rows * 4 + 255) // 256 * 256 + rows * 512 * 4
+    a256 = lambda x: (x + 255) // 256 * 256  # noqa: E731
+    # 64 sequences x 2 blocks of 64 query rows = 128 units; n ranges per unit -> 128 n CTAs
+    for n in (1, 4):
+        grid = 128 * n
+        off = a256(256 + 256 + 128 * 4)                 # error word, range, unit starts
+        off = a256(off + grid * 2 * 64 * 4)             # partial lse, two slots per CTA
+        assert ws(64, 1, 8192, n) == off + grid * 2 * 64 * 512 * 4
     assert ws(64, 0, 8192, 1) == 0                      # invalid q_len
     assert mla.mla_decode_workspace_size(_dims(page_size=16), 1, 1, 64, 1) == 0
 
