@@ -34,7 +34,7 @@ STATUS_NAMES = {0: "MLA_OK", 1: "MLA_ERR_INVALID_ARG", 2: "MLA_ERR_UNSUPPORTED",
 # Public C symbols (kept in sync with include/mla.h; a CPU test checks both ways).
 C_SYMBOLS = ("mla_row_width", "mla_status_string", "mla_cache_append", "mla_absorb_q",
              "mla_decode_workspace_size", "mla_decode_attn", "mla_out_up",
-             "mla_get_device_status")
+             "mla_get_device_status", "mla_decode_attn_noalloc")
 
 
 class MlaError(RuntimeError):
@@ -93,6 +93,9 @@ def lib() -> ctypes.CDLL:
     L.mla_out_up.restype = _I32
     L.mla_get_device_status.argtypes = [_P, _I32, _P]
     L.mla_get_device_status.restype = _I32
+    L.mla_decode_attn_noalloc.argtypes = [D, _P, _P, _I64, _P, _I32, _P, _I32, _I32, _I32, _I32,
+                                          _P, _P, _P, _P]
+    L.mla_decode_attn_noalloc.restype = _I32
     _lib = L
     return L
 
@@ -213,6 +216,32 @@ def mla_decode_attn(dims: MlaDims, q_ext, cache, block_table, seq_lens, max_seq_
     _check(st, "mla_decode_attn")
 
 
+def mla_decode_attn_noalloc(dims: MlaDims, q_ext, cache, block_table, seq_lens,
+                            max_seq_len: int, dev_error, o_latent, lse, causal: bool = True,
+                            stream=None) -> None:
+    """mla_decode_attn without a workspace, for callers that cannot allocate device memory
+    at decode time: the library's own fixed scratch array stands in for the workspace.
+    Calls that overlap on the GPU share that array and must not be issued."""
+    B, q = q_ext.shape[0], q_ext.shape[1]
+    H, r = dims.num_heads, dims.kv_lora_rank
+    _need(q_ext, "q_ext", torch.bfloat16, (B, q, H, dims.row_width))
+    _need(cache, "cache", torch.bfloat16)
+    if cache.dim() != 3 or cache.shape[1] != dims.page_size or cache.shape[2] != dims.row_width:
+        raise MlaError(f"cache shape {tuple(cache.shape)} does not match dims", MLA_ERR_INVALID_ARG)
+    _need(block_table, "block_table", torch.int32)
+    if block_table.dim() != 2 or block_table.shape[0] != B:
+        raise MlaError("block_table must be [B, max_pages]", MLA_ERR_INVALID_ARG)
+    _need(seq_lens, "seq_lens", torch.int32, (B,))
+    _need(dev_error, "dev_error", torch.int32)
+    _need(o_latent, "o_latent", torch.bfloat16, (B, q, H, r))
+    _need(lse, "lse", torch.float32, (B, q, H))
+    st = lib().mla_decode_attn_noalloc(ctypes.byref(dims), _ptr(q_ext), _ptr(cache), cache.shape[0],
+                                       _ptr(block_table), block_table.shape[1], _ptr(seq_lens), B,
+                                       q, int(max_seq_len), 1 if causal else 0, _ptr(dev_error),
+                                       _ptr(o_latent), _ptr(lse), _stream(stream))
+    _check(st, "mla_decode_attn_noalloc")
+
+
 def mla_out_up(dims: MlaDims, o_latent, w_uv, o, bias=None,
                w_uv_head_stride: Optional[int] = None, stream=None) -> None:
     """o [rows, H, d_v] = W_UV o_latent (+ bias); o_latent is [rows, H, r] (any leading shape)."""
@@ -258,4 +287,5 @@ def mla_decode_step(dims: MlaDims, *, c_kv_new, k_r_new, cos_new, sin_new, start
 
 __all__ = ["MlaDims", "MlaError", "make_dims", "lib", "mla_row_width", "mla_cache_append",
            "mla_absorb_q", "mla_decode_workspace_size", "mla_decode_attn", "mla_out_up",
+           "mla_decode_attn_noalloc",
            "mla_get_device_status", "mla_decode_step", "C_SYMBOLS", "STATUS_NAMES"]

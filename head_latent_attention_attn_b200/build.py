@@ -17,7 +17,7 @@ ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 OBJ = os.path.join(ROOT, "_build", "mla")
 LIB = os.path.join(PKG, "libmla.so")
-SOURCES = ["host_common.cu", "api.cu", "append.cu", "wgemm.cu", "decode.cu"]
+SOURCES = ["host_common.cu", "api.cu", "append.cu", "wgemm.cu", "decode.cu", "noalloc.cu"]
 HEADERS = ["ptx.cuh", "kernels.h", "host_common.h"]
 
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]

@@ -182,6 +182,39 @@ mla_status mla_out_up(const mla_dims* dims, const void* o_latent, const void* w_
                       void* stream);
 
 /*
+ * mla_decode_attn_noalloc - mla_decode_attn for callers that cannot allocate device memory.
+ *
+ * The pages have no counterpart for this call; it exists for deployment. Code that runs
+ * where cudaMalloc is not allowed (inside an allocator or memory-pool hook that must not
+ * re-enter the allocator, or a runtime that fixes its device-memory budget at start-up)
+ * cannot provide mla_decode_attn's workspace. This variant computes the same o_latent and
+ * lse with the workspace replaced by a fixed scratch array of MLA_NOALLOC_SCRATCH_BYTES
+ * that the library keeps in its own device memory; every GPU that loads the library holds
+ * that array until the process exits. It never calls cudaMalloc or cudaFree.
+ *
+ *   Arguments are those of mla_decode_attn without num_splits / workspace, plus
+ *   dev_error: int32 device error word (required): bits the decode sets are ORed into it.
+ *
+ * - The first call on each device looks up the array's device address (a host-side
+ *   runtime query, done once per device with that device current); make that first call
+ *   before capturing the stream into a CUDA graph.
+ * - All calls share the one array and it keeps the last call's contents; each call
+ *   rewrites what it reads, so nothing has to be cleared between calls. Calls whose
+ *   execution overlaps on the GPU (different streams, or different host threads without
+ *   ordering) race on the array and must not be used.
+ * - The number of work ranges is the largest that fits in the array (at most one per SM);
+ *   a problem whose partial results cannot fit even with one range per (sequence, block of
+ *   query rows) returns MLA_ERR_WORKSPACE and launches nothing.
+ */
+#define MLA_NOALLOC_SCRATCH_BYTES ((size_t)32 << 20)
+mla_status mla_decode_attn_noalloc(const mla_dims* dims, const void* q_ext, const void* cache,
+                                   int64_t num_pages, const int32_t* block_table,
+                                   int32_t max_pages_per_seq, const int32_t* seq_lens,
+                                   int32_t batch, int32_t q_len, int32_t max_seq_len,
+                                   int32_t causal, int32_t* dev_error, void* o_latent,
+                                   float* lse, void* stream);
+
+/*
  * Synchronise `stream`, read the device error word at `dev_error` and, if reset != 0,
  * clear it. Returns MLA_ERR_DEVICE_TIMEOUT, MLA_ERR_DEVICE_BOUNDS or MLA_OK (or
  * MLA_ERR_CUDA if the read fails). For mla_decode_attn the word is the first int32

@@ -1,0 +1,69 @@
+"""mla_decode_attn_noalloc: decode attention for callers that cannot allocate device memory
+when they decode (for example code inside an allocator or memory-pool hook, or a runtime
+that fixes its device-memory budget at start-up). It must give the same o_latent and lse
+as mla_decode_attn with a caller-provided workspace, call after call, and refuse problems
+whose partial results do not fit in its fixed scratch array.
+
+This file is named to be collected last: a run that stops at the first failure has then
+already run every other test."""
+import ctypes
+
+import numpy as np
+import pytest
+import torch
+
+import head_latent_attention_attn_b200 as mla
+from mla_inputs import CONFIGS, make_workload, shrink
+from tests.gpu_harness import LSE_TOL, O_TOL, GpuProblem, dims_of, max_rel_err
+
+pytestmark = pytest.mark.gpu
+
+CASES = {
+    # ragged lengths: sequences are cut between CTAs, so the merge runs on the scratch
+    "qwen3_ragged": shrink(CONFIGS["qwen3_30b_a3b"], batch=6, lens_range=(100, 3000)),
+    # four query rows per sequence, causal inside the block
+    "hybrid_q4": shrink(CONFIGS["hybrid_1m_q4"], batch=2, context=5000),
+}
+
+
+@pytest.mark.parametrize("name", sorted(CASES))
+def test_noalloc_matches_workspace_decode(name):
+    cfg = CASES[name]
+    prob = GpuProblem(make_workload(cfg))
+    prob.step()                                    # workspace path: append, absorb, decode
+    torch.cuda.synchronize()
+    ref_o = prob.o_latent.float().cpu().numpy()
+    ref_l = prob.lse.cpu().numpy()
+    err = torch.zeros(1, dtype=torch.int32, device="cuda")
+    for call in range(2):                          # two calls in a row share the scratch
+        o = torch.full_like(prob.o_latent, float("nan"))
+        lse = torch.full_like(prob.lse, float("nan"))
+        mla.mla_decode_attn_noalloc(prob.dims, prob.q_ext, prob.cache, prob.block_table,
+                                    prob.seq_lens, prob.max_seq_len, err, o, lse,
+                                    causal=cfg.causal)
+        torch.cuda.synchronize()
+        got_o = o.float().cpu().numpy()
+        got_l = lse.cpu().numpy()
+        assert np.all(np.isfinite(got_o)) and np.all(np.isfinite(got_l)), f"call {call}"
+        assert max_rel_err(got_o, ref_o) <= O_TOL, f"call {call}: o_latent differs"
+        assert float(np.max(np.abs(got_l - ref_l))) <= LSE_TOL, f"call {call}: lse differs"
+    assert mla.mla_get_device_status(err) == mla.MLA_OK
+
+
+def test_noalloc_rejects_problems_beyond_the_scratch():
+    """64 sequences x 128 heads x rank 512 need more partial-result room than the scratch
+    holds even with one work range per (sequence, row block): refused, nothing launched."""
+    cfg = CONFIGS["deepseek_v2"]
+    dims = dims_of(cfg)
+    fake = ctypes.c_void_p(0x10000)
+    st = mla.lib().mla_decode_attn_noalloc(ctypes.byref(dims), fake, fake, 100000, fake, 128,
+                                           fake, cfg.batch, 1, cfg.context, 1, fake, fake, fake,
+                                           None)
+    assert st == mla.MLA_ERR_WORKSPACE
+    st = mla.lib().mla_decode_attn_noalloc(ctypes.byref(dims_of(cfg.with_(page_size=32))), fake,
+                                           fake, 100000, fake, 128, fake, 4, 1, 512, 1, fake,
+                                           fake, fake, None)
+    assert st == mla.MLA_ERR_UNSUPPORTED
+    st = mla.lib().mla_decode_attn_noalloc(ctypes.byref(dims), fake, fake, 100000, fake, 128,
+                                           fake, 4, 1, 512, 1, None, fake, fake, None)
+    assert st == mla.MLA_ERR_INVALID_ARG            # the error word is required
