@@ -343,9 +343,7 @@ mla_status mla_decode_attn(const mla_dims* dims, const void* q_ext, const void* 
     c.ncol = P.ncol;
     c.col_groups = P.col_groups;
     c.units = P.units;
-    const int64_t items = int64_t(P.units) * P.ncol * ((p.r + 127) / 128);
-    const int cgrid = int(std::min<int64_t>(items, int64_t(num_sms()) * 8));
-    if (launch_combine(c, cgrid, s) != cudaSuccess) return MLA_ERR_CUDA;
+    if (launch_combine(c, s) != cudaSuccess) return MLA_ERR_CUDA;
   }
   return MLA_OK;
 }

@@ -667,29 +667,27 @@ __global__ void __launch_bounds__(kThreads, 1)
 }
 
 // ---- merge of cut units: lse = log sum_i e^{lse_i}, o = sum_i e^{lse_i - lse} o_i ------
-// Grid-stride over items (unit, query row, 128-latent chunk); 4 warps split the pieces,
-// each lane owns 4 latents of the chunk, and the warps' sums meet in shared memory.
+// One block per (unit, query row): warp 0 reduces the pieces' lse, then the 4 warps split
+// the pieces and every lane accumulates up to 16 latents; shared memory adds the warps.
 __global__ void __launch_bounds__(128) mla_combine_kernel(const CombineParams p) {
-  __shared__ float part[4][128];
+  __shared__ float part[4][512];
+  __shared__ float lse_s;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int u = int(blockIdx.x / unsigned(p.ncol));
+  const int n = int(blockIdx.x % unsigned(p.ncol));
+  const int G = p.col_groups;
+  const int b = u / G, cg = u - b * G;
+  const int f = cg * p.ncol + n;
+  if (f >= p.qH) return;
+  int L = p.seq_lens[b];
+  const bool ok = L >= p.q_len && L <= p.max_seq_len && int64_t(L) <= int64_t(p.max_pages) * kDecodeTok;
+  if (!ok) L = 0;
+  const int tiles = L > 0 ? (L + kDecodeTok - 1) / kDecodeTok : 1;
   const int per = *p.range_len;
-  const int nchunk = (p.r + 127) / 128;
-  const int64_t items = int64_t(p.units) * p.ncol * nchunk;
-  for (int64_t it = blockIdx.x; it < items; it += gridDim.x) {
-    const int u = int(it / (p.ncol * nchunk));
-    const int rem = int(it - int64_t(u) * p.ncol * nchunk);
-    const int n = rem / nchunk, ch = rem - n * nchunk;
-    const int b = u / p.col_groups, cg = u - b * p.col_groups;
-    const int f = cg * p.ncol + n;
-    const int G = p.col_groups;
-    if (f >= p.qH) continue;
-    int L = p.seq_lens[b];
-    const bool ok = L >= p.q_len && L <= p.max_seq_len && int64_t(L) <= int64_t(p.max_pages) * kDecodeTok;
-    if (!ok) L = 0;
-    const int tiles = L > 0 ? (L + kDecodeTok - 1) / kDecodeTok : 1;
-    const int s = p.unit_start[u];
-    const int i0 = s / per, i1 = (s + tiles - 1) / per;
-    if (i0 == i1) continue;   // held whole by one CTA: already written
+  const int s = p.unit_start[u];
+  const int i0 = s / per, i1 = (s + tiles - 1) / per;
+  if (i0 == i1) return;   // held whole by one CTA: already written
+  if (warp == 0) {
     float mx = -INFINITY;
     for (int i = i0 + lane; i <= i1; i += 32)
       mx = fmaxf(mx, p.part_lse[int64_t(piece_slot(i, s, per, G, cg)) * p.ncol + n]);
@@ -702,33 +700,35 @@ __global__ void __launch_bounds__(128) mla_combine_kernel(const CombineParams p)
     }
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) den += __shfl_xor_sync(0xffffffffu, den, o);
-    const float lse = mx == -INFINITY ? -INFINITY : mx + logf(den);
-    float acc[4] = {0.0f, 0.0f, 0.0f, 0.0f};
-    for (int i = i0 + warp; i <= i1; i += 4) {
-      const int64_t sl = piece_slot(i, s, per, G, cg);
-      const float li = p.part_lse[sl * p.ncol + n];
-      if (li == -INFINITY) continue;
-      const float wgt = expf(li - lse);
-      const float* row = p.part_o + (sl * p.ncol + n) * p.r + ch * 128;
-#pragma unroll
-      for (int k = 0; k < 4; ++k) {
-        const int lat = lane + 32 * k;
-        if (ch * 128 + lat < p.r) acc[k] += wgt * row[lat];
-      }
-    }
-#pragma unroll
-    for (int k = 0; k < 4; ++k) part[warp][lane + 32 * k] = acc[k];
-    __syncthreads();
-    {
-      const int lat = threadIdx.x;
-      if (ch * 128 + lat < p.r) {
-        const float v = part[0][lat] + part[1][lat] + part[2][lat] + part[3][lat];
-        p.o_latent[(int64_t(b) * p.qH + f) * p.r + ch * 128 + lat] = f32_to_bf16_rne(v);
-      }
-      if (threadIdx.x == 0 && ch == 0) p.lse[int64_t(b) * p.qH + f] = lse;
-    }
-    __syncthreads();
+    if (lane == 0) lse_s = mx == -INFINITY ? -INFINITY : mx + logf(den);
   }
+  __syncthreads();
+  const float lse = lse_s;
+  float acc[16];
+#pragma unroll
+  for (int j = 0; j < 16; ++j) acc[j] = 0.0f;
+  for (int i = i0 + warp; i <= i1; i += 4) {
+    const int64_t sl = piece_slot(i, s, per, G, cg);
+    const float li = p.part_lse[sl * p.ncol + n];
+    if (li == -INFINITY) continue;
+    const float wgt = expf(li - lse);
+    const float* row = p.part_o + (sl * p.ncol + n) * p.r;
+#pragma unroll
+    for (int j = 0; j < 16; ++j) {
+      const int lat = lane + 32 * j;
+      if (lat < p.r) acc[j] += wgt * row[lat];
+    }
+  }
+#pragma unroll
+  for (int j = 0; j < 16; ++j) {
+    const int lat = lane + 32 * j;
+    if (lat < p.r) part[warp][lat] = acc[j];
+  }
+  __syncthreads();
+  uint16_t* out = p.o_latent + (int64_t(b) * p.qH + f) * p.r;
+  for (int lat = threadIdx.x; lat < p.r; lat += 128)
+    out[lat] = f32_to_bf16_rne(part[0][lat] + part[1][lat] + part[2][lat] + part[3][lat]);
+  if (threadIdx.x == 0) p.lse[int64_t(b) * p.qH + f] = lse;
 }
 
 #ifdef MLA_TRACE
@@ -738,8 +738,10 @@ extern "C" int mla_trace_read(unsigned long long* host, int n) {
 }
 #endif
 
-cudaError_t launch_combine(const CombineParams& p, int grid, cudaStream_t stream) {
-  mla_combine_kernel<<<grid, 128, 0, stream>>>(p);
+cudaError_t launch_combine(const CombineParams& p, cudaStream_t stream) {
+  const int64_t blocks = int64_t(p.units) * p.ncol;
+  if (blocks <= 0 || blocks > 0x7fffffffLL) return cudaErrorInvalidValue;
+  mla_combine_kernel<<<unsigned(blocks), 128, 0, stream>>>(p);
   return cudaGetLastError();
 }
 

@@ -79,6 +79,6 @@ struct CombineParams {
   float* lse;
   int32_t q_len, max_seq_len, max_pages, qH, r, ncol, col_groups, units;
 };
-cudaError_t launch_combine(const CombineParams& p, int grid, cudaStream_t stream);
+cudaError_t launch_combine(const CombineParams& p, cudaStream_t stream);
 
 }  // namespace mla
