@@ -128,7 +128,7 @@ class ClockSampler:
 
 def _source_hash():
     h = hashlib.sha256()
-    for f in ("decode.cu", "ptx.cuh", "kernels.h"):
+    for f in ("decode.cu", "decode_pair.cu", "decode_sched.cuh", "ptx.cuh", "kernels.h"):
         h.update(open(os.path.join(ROOT, "head_latent_attention_attn_b200", "csrc", f), "rb").read())
     return h.hexdigest()[:16]
 

@@ -17,8 +17,9 @@ ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 OBJ = os.path.join(ROOT, "_build", "mla")
 LIB = os.path.join(PKG, "libmla.so")
-SOURCES = ["host_common.cu", "api.cu", "append.cu", "wgemm.cu", "decode.cu", "noalloc.cu"]
-HEADERS = ["ptx.cuh", "kernels.h", "host_common.h"]
+SOURCES = ["host_common.cu", "api.cu", "append.cu", "wgemm.cu", "decode.cu", "decode_pair.cu",
+           "noalloc.cu"]
+HEADERS = ["ptx.cuh", "kernels.h", "host_common.h", "decode_sched.cuh"]
 
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 FLAGS = ["-O3", "-lineinfo", "-std=c++17", "-Xcompiler", "-fPIC", "-Xcompiler", "-O2",

@@ -3,6 +3,7 @@
 // buffer is the caller's.
 #include <algorithm>
 #include <cstring>
+#include <mutex>
 
 #include "host_common.h"
 #include "kernels.h"
@@ -27,6 +28,33 @@ int num_sms() {
   return n;
 }
 
+// Clusters of two pair-kernel CTAs that fit on the current device at once, cached per
+// (device, shared-memory size); falls back to half the SM count if the query fails.
+int pair_clusters(size_t smem) {
+  static std::mutex mu;
+  static int cache_dev[16], cache_val[16];
+  static size_t cache_smem[16];
+  static int cache_n = 0;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) {
+    cudaGetLastError();
+    return num_sms() / 2;
+  }
+  std::lock_guard<std::mutex> lock(mu);
+  for (int i = 0; i < cache_n; ++i)
+    if (cache_dev[i] == dev && cache_smem[i] == smem) return cache_val[i];
+  int n = decode_pair_max_clusters(smem);
+  if (n <= 0) n = num_sms() / 2;
+  n = std::min(n, num_sms() / 2);
+  if (cache_n < 16) {
+    cache_dev[cache_n] = dev;
+    cache_smem[cache_n] = smem;
+    cache_val[cache_n] = n;
+    ++cache_n;
+  }
+  return n;
+}
+
 int pow2_at_least(int x, int lo) {
   int v = lo;
   while (v < x) v <<= 1;
@@ -36,6 +64,9 @@ int pow2_at_least(int x, int lo) {
 // Launch geometry of one mla_decode_attn problem.
 struct DecodePlan {
   int ncol, col_groups, units, nblk, nch, slot_blocks, nslot, npt, tmem_cols, grid;
+  int pair;        // 1: blocks of 128 rows on clusters of two CTAs that split the latent
+  int rope_half;   // rotary columns per CTA of a pair
+  int vgrid;       // work ranges (CTAs, or clusters for the pair kernel)
   size_t smem;
   size_t ws_bytes;
   size_t range_off, unit_start_off, part_lse_off, part_o_off;
@@ -54,7 +85,13 @@ mla_status plan_decode(const mla_dims* d, int32_t batch, int32_t q_len, int32_t 
   const int D = row_width(d);
   if (r > 512 || D > 64 * kDecodeMaxBlk) return MLA_ERR_UNSUPPORTED;
   const int64_t qH = int64_t(q_len) * d->num_heads;
-  P->ncol = qH <= 16 ? 16 : (qH <= 32 ? 32 : 64);
+  const int R = d->num_kv_groups * d->rope_dim;
+  // More than 64 rows per sequence: 128-row blocks on clusters of two CTAs that split the
+  // latent (r a multiple of 128, rotary half of 16, 32 or 64 columns); else blocks of
+  // 16, 32 or 64 rows, one CTA each.
+  P->pair = (qH > 64 && r % 128 == 0 && (R == 32 || R == 64 || R == 128)) ? 1 : 0;
+  P->rope_half = R / 2;
+  P->ncol = P->pair ? kPairRows : (qH <= 16 ? 16 : (qH <= 32 ? 32 : 64));
   P->col_groups = int((qH + P->ncol - 1) / P->ncol);
   const int64_t units = int64_t(std::max(batch, 1)) * P->col_groups;
   if (units > (int64_t(1) << 24)) return MLA_ERR_UNSUPPORTED;
@@ -62,37 +99,49 @@ mla_status plan_decode(const mla_dims* d, int32_t batch, int32_t q_len, int32_t 
   P->nblk = (D + 63) / 64;
   P->nch = (r + 127) / 128;
   P->slot_blocks = std::max(P->nblk, 2 * P->nch);
-  P->tmem_cols = pow2_at_least((2 + P->nch) * P->ncol, 32);
-  if (P->tmem_cols > 512) return MLA_ERR_UNSUPPORTED;
-  // Most cache slots that fit, preferring two P^T buffers; at least two slots.
   P->nslot = 0;
-  for (int npt = 2; npt >= 1 && P->nslot == 0; --npt) {
-    for (int ns = kDecodeMaxSlots; ns >= 2; --ns) {
-      if (decode_smem_bytes(P->ncol, P->nblk, P->slot_blocks, ns, npt) <= size_t(kMaxSmem)) {
-        P->nslot = ns;
-        P->npt = npt;
-        break;
+  P->npt = 1;
+  if (P->pair) {
+    P->tmem_cols = 512;
+    for (int ns = kDecodeMaxSlots; ns >= 2 && P->nslot == 0; --ns)
+      if (decode_pair_smem_bytes(r, P->rope_half, ns) <= size_t(kMaxSmem)) P->nslot = ns;
+    if (P->nslot < 2) return MLA_ERR_UNSUPPORTED;
+    P->smem = decode_pair_smem_bytes(r, P->rope_half, P->nslot);
+  } else {
+    P->tmem_cols = pow2_at_least((2 + P->nch) * P->ncol, 32);
+    if (P->tmem_cols > 512) return MLA_ERR_UNSUPPORTED;
+    // Most cache slots that fit, preferring two P^T buffers; at least two slots.
+    for (int npt = 2; npt >= 1 && P->nslot == 0; --npt) {
+      for (int ns = kDecodeMaxSlots; ns >= 2; --ns) {
+        if (decode_smem_bytes(P->ncol, P->nblk, P->slot_blocks, ns, npt) <= size_t(kMaxSmem)) {
+          P->nslot = ns;
+          P->npt = npt;
+          break;
+        }
       }
     }
+    if (P->nslot < 2) return MLA_ERR_UNSUPPORTED;
+    P->smem = decode_smem_bytes(P->ncol, P->nblk, P->slot_blocks, P->nslot, P->npt);
   }
-  if (P->nslot < 2) return MLA_ERR_UNSUPPORTED;
-  P->smem = decode_smem_bytes(P->ncol, P->nblk, P->slot_blocks, P->nslot, P->npt);
-  // Persistent grid: the units' page tiles are cut into `grid` equal ranges. By default
-  // one CTA per SM; num_splits > 0 asks for num_splits ranges per unit on average.
+  // Persistent grid: the units' page tiles are cut into `vgrid` equal ranges, one per CTA
+  // (per cluster for the pair kernel). By default as many as fit on the device at once;
+  // num_splits > 0 asks for num_splits ranges per unit on average.
   const int64_t max_tiles = (int64_t(max_seq_len) + kDecodeTok - 1) / kDecodeTok;
-  // The grid is a multiple of the number of row blocks: CTA c works on row block
-  // c % col_groups, so the blocks of a sequence are read in lockstep.
+  // The range count is a multiple of the number of row blocks: range c works on row
+  // block c % col_groups, so the blocks of a sequence are read in lockstep.
   const int cgs = P->col_groups;
-  int64_t g = num_splits > 0 ? units * num_splits : num_sms();
+  const int64_t resident = P->pair ? pair_clusters(P->smem) : num_sms();
+  int64_t g = num_splits > 0 ? units * num_splits : resident;
   g = std::min<int64_t>(g, units * max_tiles);
   g = std::max<int64_t>(cgs, std::min<int64_t>(g, 1 << 20) / cgs * cgs);
-  P->grid = int(g);
+  P->vgrid = int(g);
+  P->grid = int(P->pair ? 2 * g : g);
   size_t off = 256;                              // device error word + padding
-  P->range_off = off;                            // int32: tiles per CTA range
+  P->range_off = off;                            // int32: tiles per range
   off += 256;
   P->unit_start_off = off;                       // int32 per unit: its first global tile
   off = align256(off + size_t(units) * sizeof(int32_t));
-  P->part_lse_off = off;
+  P->part_lse_off = off;                         // two partial slots per range
   off = align256(off + size_t(g) * 2 * P->ncol * sizeof(float));
   P->part_o_off = off;
   off += size_t(g) * 2 * P->ncol * size_t(r) * sizeof(float);
@@ -294,6 +343,17 @@ mla_status mla_decode_attn(const mla_dims* dims, const void* q_ext, const void* 
     if (!encode_bf16_map(&p.tm_q, q_ext, 3, d3, s3, box, CU_TENSOR_MAP_SWIZZLE_128B))
       return MLA_ERR_CUDA;
   }
+  if (P.pair) {
+    const uint64_t d2[2] = {uint64_t(D), uint64_t(num_pages) * kDecodeTok};
+    const uint64_t s2[1] = {uint64_t(D) * 2};
+    const uint32_t box[2] = {uint32_t(P.rope_half), uint32_t(kDecodeTok)};
+    const CUtensorMapSwizzle sw = P.rope_half == 64   ? CU_TENSOR_MAP_SWIZZLE_128B
+                                  : P.rope_half == 32 ? CU_TENSOR_MAP_SWIZZLE_64B
+                                                      : CU_TENSOR_MAP_SWIZZLE_32B;
+    if (!encode_bf16_map(&p.tm_rope, cache, 2, d2, s2, box, sw)) return MLA_ERR_CUDA;
+    p.q_ext = static_cast<const uint16_t*>(q_ext);
+    p.rope_half = P.rope_half;
+  }
   uint8_t* ws = static_cast<uint8_t*>(workspace);
   p.block_table = block_table;
   p.seq_lens = seq_lens;
@@ -324,8 +384,10 @@ mla_status mla_decode_attn(const mla_dims* dims, const void* q_ext, const void* 
   p.npt = P.npt;
   p.scale_log2 = dims->softmax_scale * 1.4426950408889634f;
   cudaStream_t s = as_stream(stream);
-  if (launch_decode(p, P.ncol, dim3(P.grid), P.smem, s) != cudaSuccess) return MLA_ERR_CUDA;
-  if (P.grid > 1) {
+  const cudaError_t le = P.pair ? launch_decode_pair(p, dim3(P.grid), P.smem, s)
+                                : launch_decode(p, P.ncol, dim3(P.grid), P.smem, s);
+  if (le != cudaSuccess) return MLA_ERR_CUDA;
+  if (P.vgrid > P.col_groups) {
     // merge the pieces of units cut between CTAs (units held whole are skipped)
     CombineParams c{};
     c.part_o = p.part_o;

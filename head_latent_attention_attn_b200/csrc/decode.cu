@@ -1,5 +1,5 @@
-// decode.cu - mla_decode_attn on sm_100a: paged, split-KV absorbed attention over the
-// latent cache, with the split merge fused into the same launch.
+// decode.cu - mla_decode_attn on sm_100a for blocks of up to 64 query rows: paged,
+// split-KV absorbed attention over the latent cache, and the merge of the split pieces.
 //
 // Formulation. Every query row (i, h) of a sequence scores the SAME cache rows, so the
 // CTA keeps a block of NCOL query rows resident and streams the cache pages once:
@@ -28,6 +28,7 @@
 // then the tile max is reduced over the CTA and O^T and the running sums are rescaled.
 #include <math.h>
 
+#include "decode_sched.cuh"
 #include "kernels.h"
 #include "ptx.cuh"
 
@@ -149,37 +150,6 @@ __host__ __device__ constexpr SmemSwizzle pt_swizzle(int ncol) {
   return ncol == 64 ? kSw128 : (ncol == 32 ? kSw64 : kSw32);
 }
 
-MLA_DEVICE int unit_tiles(int L) { return L > 0 ? (L + kDecodeTok - 1) / kDecodeTok : 1; }
-
-// Context length of sequence b if it is within the bounds the launch was planned for,
-// else 0 (the unit then produces zeros and lse = -inf, and the error word is set).
-MLA_DEVICE int valid_len(const DecodeParams& p, int L) {
-  const bool ok = L >= p.q_len && L <= p.max_seq_len &&
-                  int64_t(L) <= int64_t(p.max_pages) * kDecodeTok;
-  return ok ? L : 0;
-}
-
-// The walk over the sequences a CTA's tile range touches; every role runs the same walk.
-// A CTA works on one block cg of query rows: unit u = b * col_groups + cg.
-struct UnitWalk {
-  int b, s;       // sequence and the index of its first tile in this row block's tile space
-  int tiles, L, u;
-  MLA_DEVICE void load(const DecodeParams& p, int cg) {
-    L = valid_len(p, p.seq_lens[b]);
-    tiles = unit_tiles(L);
-    u = b * p.col_groups + cg;
-  }
-};
-
-// Partial-result slot of virtual CTA i (of row block cg) holding a piece of a unit whose
-// first tile is s, when ranges are `per` tiles long: slot 0 holds a CTA's first piece,
-// slot 1 its last. A unit is the first piece of every CTA it reaches except possibly the
-// one where it starts.
-MLA_DEVICE int piece_slot(int i, int s, int per, int col_groups, int cg) {
-  const int i0 = s / per;
-  return 2 * (i * col_groups + cg) + ((i == i0 && s != i0 * per) ? 1 : 0);
-}
-
 }  // namespace
 
 size_t decode_smem_bytes(int ncol, int nblk, int slot_blocks, int nslot, int npt) {
@@ -249,57 +219,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   // ---- schedule: this CTA's tile range [r0, r1) in its row block, first sequence -------
   // The row blocks of a sequence are worked on in lockstep by neighbouring CTAs, so the
   // second read of every page is served from L2.
-  {
-    int total = 0;
-    for (int b = threadIdx.x; b < p.batch; b += kThreads) {
-      const int Lv = valid_len(p, p.seq_lens[b]);
-      if (Lv == 0 && blockIdx.x == 0 && p.dev_error) atomicOr(p.dev_error, MLA_DEVERR_BOUNDS);
-      total += unit_tiles(Lv);
-    }
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) total += __shfl_xor_sync(0xffffffffu, total, o);
-    if (lane == 0) warp_sum[warp] = total;
-    __syncthreads();
-    total = 0;
-#pragma unroll
-    for (int w = 0; w < kThreads / 32; ++w) total += warp_sum[w];
-    const int per = max(1, (total + vgrid - 1) / vgrid);
-    const int r0 = min(total, vc * per);
-    const int r1 = min(total, r0 + per);
-    __syncthreads();
-    if (threadIdx.x == 0) {
-      sched[0] = -1;
-      sched[2] = r0;
-      sched[3] = r1;
-      sched[4] = per;
-      sched[5] = 0;   // running tile count before the current chunk of sequences
-    }
-    __syncthreads();
-    // chunked exclusive scan over the sequences until the one holding tile r0 is found
-    for (int b0 = 0; b0 < p.batch && r0 < r1; b0 += kThreads) {
-      const int b = b0 + threadIdx.x;
-      const int t = b < p.batch ? unit_tiles(valid_len(p, p.seq_lens[b])) : 0;
-      int incl = t;
-#pragma unroll
-      for (int o = 1; o < 32; o <<= 1) {
-        const int y = __shfl_up_sync(0xffffffffu, incl, o);
-        if (lane >= o) incl += y;
-      }
-      if (lane == 31) warp_sum[warp] = incl;
-      __syncthreads();
-      int before = sched[5];
-      for (int w = 0; w < warp; ++w) before += warp_sum[w];
-      const int start = before + incl - t;
-      if (b < p.batch && start <= r0 && r0 < start + t) {
-        sched[0] = b;
-        sched[1] = start;
-      }
-      __syncthreads();
-      if (threadIdx.x == kThreads - 1) sched[5] = before + incl;
-      __syncthreads();
-      if (sched[0] >= 0) break;
-    }
-  }
+  find_tile_range<kThreads>(p, vc, vgrid, blockIdx.x == 0, warp_sum, sched);
   tc_fence_before();
   __syncthreads();
   tc_fence_after();

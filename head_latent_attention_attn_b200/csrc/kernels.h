@@ -63,10 +63,22 @@ struct DecodeParams {
   int32_t max_pages, batch, q_len, num_heads, qH, r, D, nblk, nch, col_groups, units,
       max_seq_len, causal, nslot, slot_blocks, tmem_cols, npt;
   float scale_log2;          // softmax_scale * log2(e)
+  // used by the latent-split cluster kernel only
+  CUtensorMap tm_rope;       // 2D {D, num_pages*64}, box {rope_half, 64}
+  const uint16_t* q_ext;     // [B, q*H, D]
+  int32_t rope_half;         // rotary columns per CTA of the pair (G*d_r/2)
 };
 size_t decode_smem_bytes(int ncol, int nblk, int slot_blocks, int nslot, int npt);
 cudaError_t launch_decode(const DecodeParams& p, int ncol, dim3 grid, size_t smem,
                           cudaStream_t stream);
+
+// Blocks of up to 128 query rows: a cluster of two CTAs splits the latent (decode_pair.cu).
+constexpr int kPairRows = 128;
+size_t decode_pair_smem_bytes(int r, int rope_half, int nslot);
+// Clusters of two that can be resident at once with `smem` bytes each (0 if unknown).
+int decode_pair_max_clusters(size_t smem);
+cudaError_t launch_decode_pair(const DecodeParams& p, dim3 grid, size_t smem,
+                               cudaStream_t stream);
 
 // Merge of the per-piece partials of units cut between CTAs (log-sum-exp identity).
 struct CombineParams {

@@ -101,16 +101,28 @@ def test_decode_validation(mla_lib):
 
 
 def test_workspace_size(mla_lib):
-    d = _dims()
-    ws = lambda *a: mla.mla_decode_workspace_size(d, *a)  # noqa: E731
     a256 = lambda x: (x + 255) // 256 * 256  # noqa: E731
-    # 64 sequences x 2 blocks of 64 query rows = 128 units; n ranges per unit -> 128 n CTAs
+    # 128 heads, q = 1: one block of 128 query rows per sequence on a cluster of two CTAs
+    # that split the latent; 64 units, n ranges (clusters) per unit, two partial slots each
+    d = _dims()
     for n in (1, 4):
-        grid = 128 * n
-        off = a256(256 + 256 + 128 * 4)                 # error word, range, unit starts
-        off = a256(off + grid * 2 * 64 * 4)             # partial lse, two slots per CTA
-        assert ws(64, 1, 8192, n) == off + grid * 2 * 64 * 512 * 4
-    assert ws(64, 0, 8192, 1) == 0                      # invalid q_len
+        ranges = 64 * n
+        off = a256(256 + 256 + 64 * 4)                  # error word, range, unit starts
+        off = a256(off + ranges * 2 * 128 * 4)          # partial lse
+        assert mla.mla_decode_workspace_size(d, 64, 1, 8192, n) == off + ranges * 2 * 128 * 512 * 4
+    # 32 heads, q = 1: blocks of 32 rows, one CTA per range
+    d32 = _dims(num_heads=32)
+    for n in (1, 3):
+        ranges = 64 * n
+        off = a256(256 + 256 + 64 * 4)
+        off = a256(off + ranges * 2 * 32 * 4)
+        assert mla.mla_decode_workspace_size(d32, 64, 1, 8192, n) == off + ranges * 2 * 32 * 512 * 4
+    # 128 heads of rank 320 (not a multiple of 128): two blocks of 64 rows instead
+    d320 = _dims(kv_lora_rank=320)
+    off = a256(256 + 256 + 128 * 4)
+    off = a256(off + 128 * 2 * 64 * 4)
+    assert mla.mla_decode_workspace_size(d320, 64, 1, 8192, 1) == off + 128 * 2 * 64 * 320 * 4
+    assert mla.mla_decode_workspace_size(d, 64, 0, 8192, 1) == 0        # invalid q_len
     assert mla.mla_decode_workspace_size(_dims(page_size=16), 1, 1, 64, 1) == 0
 
 
