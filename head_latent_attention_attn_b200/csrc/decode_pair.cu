@@ -17,16 +17,17 @@
 // the partial of a tile (128 rows x 64 tokens) travels as 24-bit floats: fp32 rounded to
 // a 15-bit mantissa (relative error <= 2^-16, far below the bf16 rounding of P), 4 values
 // in 3 words, 24 KB per tile. Each CTA rounds its own partial the same way before adding,
-// so both sides add identical numbers. Every warp stages its 32 rows and sends them with
-// one bulk copy (cp.async.bulk shared::cta -> shared::cluster) that completes on the
-// partner's mbarrier. The softmax warps send tile j+1 before they finish tile j, so one
-// tile of exchange latency overlaps the softmax and PV work of the previous tile.
+// so both sides add identical numbers. Every thread sends its packed words straight from
+// registers (st.async, completing on the partner's mbarrier) and keeps them for its own
+// sum, so no shared memory is spent on staging and four cache slots fit. The softmax
+// warps send tile j+1 before they finish tile j, so one tile of exchange latency overlaps
+// the softmax and PV work of the previous tile.
 //
-// Roles (320 threads per CTA): warp 0 TMA producer, warp 1 S issuer and TMEM owner, warps
-// 2-9 the score exchange, softmax, P into TMEM, the PV issue (one thread) and the
-// epilogue. The M=128 accumulator puts row n on TMEM lane n, and a warp reaches only the
-// 32 lanes of its sub-partition (warp % 4), so two warps share every 32 rows: warps 2-5
-// take tokens 0-31 of each tile, warps 6-9 tokens 32-63, one thread per (row, half).
+// Roles (352 threads per CTA): warp 0 TMA producer, warp 1 S issuer and TMEM owner, warps
+// 2-9 the score exchange, softmax, P into TMEM and the epilogue, warp 10 the PV issuer.
+// The M=128 accumulator puts row n on TMEM lane n, and a warp reaches only the 32 lanes of
+// its sub-partition (warp % 4), so two warps share every 32 rows: softmax warp wi takes
+// tokens [32 q, 32 q + 32) of each tile, q = wi / 4, one thread per (row, part).
 //
 // TMEM columns: O [0, r/2), S [256, 320), P [320, 352) (bf16 pairs), Q [352, 352 +
 // (r/2 + rope_half)/2) (bf16 pairs: latent half, then rotary half).
@@ -39,11 +40,11 @@
 namespace mla {
 
 // Optional per-tile timeline of CTA 0 (compile with -DMLA_TRACE; read with
-// mla_pair_trace_read). Events: 0 producer issued the tile's loads, 1 S issuer saw every
-// block land, 2 S committed, 3 softmax read S, 4 partial sent, 5 partner's partial
-// received, 6 PV(j-1) seen done, 7 P written, 8 PV issued, 9 S issuer saw S free,
-// 10 scores unpacked, 11 scores scaled. After the 12 event rows: every CTA's start and
-// end (%globaltimer) as pairs.
+// mla_pair_trace_read). Events: 0 producer issued the tile's loads, 1 every block of the
+// tile landed (the S issuer waits for that before the S buffer), 2 S committed, 3 softmax
+// read S, 4 partial sent, 5 partner's partial received, 6 PV(j-1) seen done, 7 P written,
+// 8 PV issued, 9 S issuer saw S free, 10 scores unpacked, 11 scores scaled. After the 12
+// event rows: every CTA's start and end (%globaltimer) as pairs.
 #ifdef MLA_TRACE
 constexpr int kPairTraceTiles = 512;
 constexpr int kPairTraceEvents = 12;
@@ -61,23 +62,26 @@ __device__ unsigned long long g_mla_pair_trace[kPairTraceEvents * kPairTraceTile
 
 namespace {
 
-constexpr int kThreads = 320;
-constexpr int kSoftThreads = 256;                              // warps 2-9
-constexpr int kHalfTok = kDecodeTok / 2;                       // tokens per softmax thread
+constexpr int kQuarters = 2;                                   // softmax threads per row
+constexpr int kSoftWarps = 4 * kQuarters;                      // warps 2 .. 2 + kSoftWarps
+constexpr int kSoftThreads = 32 * kSoftWarps;
+constexpr int kPvWarp = 2 + kSoftWarps;
+constexpr int kThreads = 32 * (kPvWarp + 1);
+constexpr int kQTok = kDecodeTok / kQuarters;                  // tokens per softmax thread
 constexpr uint32_t kBlk = kDecodeTok * 128;                    // 64 x 64 bf16 block, 8 KB
-constexpr int kPackWords = kHalfTok * 3 / 4;                   // 24-bit values of a half row
-constexpr uint32_t kXWarpBytes = 32u * kPackWords * 4;          // one warp's half rows, 3 KB
-constexpr uint32_t kXBytes = 8u * kXWarpBytes;                  // one tile's partial, 24 KB
+constexpr int kPackWords = kQTok * 3 / 4;                      // 24-bit values of one part
+constexpr uint32_t kXWarpBytes = 32u * kPackWords * 4;          // one warp's parts
+constexpr uint32_t kXBytes = kSoftWarps * kXWarpBytes;          // one tile's partial, 24 KB
 constexpr uint32_t kColO = 0, kColS = 256, kColP = 320, kColQ = 352, kTmemCols = 512;
 constexpr float kLazyThreshold = 8.0f;   // log2 units; see decode.cu
 constexpr int kPrefetchAhead = 4;        // tiles brought into L2 ahead of their TMA load
 constexpr float kRefInit = -3.0e38f;
 constexpr float kLn2 = 0.69314718055994530942f;
-// misc ints: 0 TMEM base, 1 abort flag, [2,8) schedule, [8,18) warp sums
-constexpr int kMiscInts = 24;
+// misc ints: 0 TMEM base, 1 abort flag, [2,8) schedule, [8, 8 + warps) warp sums
+constexpr int kMiscInts = 32;
 
 struct PairLayout {
-  uint32_t slot_bytes, rope_off, stage_off, recv_off, red_off, misc_off, bar_off, total;
+  uint32_t slot_bytes, rope_off, recv_off, red_off, misc_off, bar_off, total;
   int nb;   // TMA barriers per slot: one per latent block and one for the rotary block
 };
 
@@ -85,7 +89,7 @@ __host__ __device__ inline uint32_t round_up_p(uint32_t x, uint32_t a) {
   return (x + a - 1) / a * a;
 }
 
-__host__ __device__ constexpr int pair_bars(int nslot, int nb) { return nslot * nb + nslot + 8; }
+__host__ __device__ constexpr int pair_bars(int nslot, int nb) { return nslot * nb + nslot + 10; }
 
 __host__ __device__ inline PairLayout pair_layout(int r, int rope_half, int nslot) {
   PairLayout L;
@@ -94,13 +98,11 @@ __host__ __device__ inline PairLayout pair_layout(int r, int rope_half, int nslo
   L.rope_off = uint32_t(lb) * kBlk;
   L.slot_bytes = round_up_p(L.rope_off + uint32_t(kDecodeTok) * rope_half * 2, 1024);
   uint32_t off = uint32_t(nslot) * L.slot_bytes;
-  L.stage_off = off;                              // own packed partials (two tiles)
-  off += 2 * kXBytes;
   L.recv_off = off;                               // partner's packed partials (two tiles)
   off += 2 * kXBytes;
-  L.red_off = off;                                // float half-row maxima [2][2][128]
-  off += 2 * 2 * kPairRows * 4;                   // and half-row sums [2][128]
-  off += 2 * kPairRows * 4;
+  L.red_off = off;                                // float part maxima [2][parts][128]
+  off += 2 * kQuarters * kPairRows * 4;           // and part sums [parts][128]
+  off += kQuarters * kPairRows * 4;
   L.misc_off = off;
   off += 4 * kMiscInts;
   L.bar_off = round_up_p(off, 8);
@@ -118,38 +120,40 @@ MLA_DEVICE SmemSwizzle rope_swizzle(int rope_half) {
 }
 
 // Byte offset of 16-byte chunk c (packed words 4c..4c+3) of lane `lane` of softmax warp
-// wi in a stage or receive buffer: each warp's half rows are one contiguous 3 KB block
-// (one bulk copy), chunk-major inside it, so a quarter-warp touches 128 consecutive bytes.
+// wi in a receive buffer: each warp's part rows are one contiguous block, chunk-major
+// inside it, so a quarter-warp touches 128 consecutive bytes.
 MLA_DEVICE uint32_t x_offset(int wi, int lane, int c) {
   return uint32_t(wi) * kXWarpBytes + uint32_t(c) * 512u + uint32_t(lane) * 16u;
 }
 
-// fp32 -> 24-bit float (sign, exponent, 15-bit mantissa), rounded to nearest.
-MLA_DEVICE uint32_t to_f24(float x) { return (__float_as_uint(x) + 0x80u) >> 8; }
+// TMEM loads of one part's scores (kQTok fp32 columns) and stores of its weights
+// (kQTok / 2 columns of bf16 pairs).
+MLA_DEVICE void tmem_ld_part(uint32_t taddr, float* v) {
+  if constexpr (kQTok == 32) tmem_ld32(taddr, v);
+  else tmem_ld16(taddr, v);
+}
+MLA_DEVICE void tmem_st_part(uint32_t taddr, const uint32_t* w) {
+  if constexpr (kQTok == 32) tmem_st16(taddr, reinterpret_cast<const float*>(w));
+  else tmem_st8(taddr, w);
+}
 
-// Four 24-bit values in three words, and back to fp32.
+// Four 24-bit values (fp32 rounded to sign, exponent and a 15-bit mantissa) in three words (value k's three bytes follow value k-1's), and back
+// to fp32 with a zero low byte. Rounding adds half of the dropped byte; the byte moves are
+// single byte permutes.
 MLA_DEVICE void pack_f24(const float* v, uint32_t* w) {
-  const uint32_t a = to_f24(v[0]), b = to_f24(v[1]), c = to_f24(v[2]), d = to_f24(v[3]);
-  w[0] = a | (b << 24);
-  w[1] = (b >> 8) | (c << 16);
-  w[2] = (c >> 16) | (d << 8);
+  const uint32_t a = __float_as_uint(v[0]) + 0x80u, b = __float_as_uint(v[1]) + 0x80u;
+  const uint32_t c = __float_as_uint(v[2]) + 0x80u, d = __float_as_uint(v[3]) + 0x80u;
+  w[0] = __byte_perm(a, b, 0x5321);   // a1 a2 a3 b1
+  w[1] = __byte_perm(b, c, 0x6532);   // b2 b3 c1 c2
+  w[2] = __byte_perm(c, d, 0x7653);   // c3 d1 d2 d3
 }
 MLA_DEVICE void unpack_f24(const uint32_t* w, float* v) {
-  v[0] = __uint_as_float(w[0] << 8);
-  v[1] = __uint_as_float((w[1] << 16) | ((w[0] >> 16) & 0xFF00u));
-  v[2] = __uint_as_float(((w[1] >> 8) & 0x00FFFF00u) | (w[2] << 24));
+  v[0] = __uint_as_float(__byte_perm(w[0], 0u, 0x2104));
+  v[1] = __uint_as_float(__byte_perm(w[0], w[1], 0x5433) & 0xFFFFFF00u);
+  v[2] = __uint_as_float(__byte_perm(w[1], w[2], 0x4322) & 0xFFFFFF00u);
   v[3] = __uint_as_float(w[2] & 0xFFFFFF00u);
 }
 
-// One bulk copy of `bytes` from this CTA's shared memory to another CTA of the cluster,
-// completing `bytes` of transactions on that CTA's mbarrier (addresses from map_to_rank).
-MLA_DEVICE void bulk_copy_to_peer(uint32_t dst_remote, uint32_t src_local, uint32_t bytes,
-                                  uint32_t remote_bar) {
-  asm volatile(
-      "cp.async.bulk.shared::cluster.shared::cta.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
-      ::"r"(dst_remote), "r"(src_local), "r"(bytes), "r"(remote_bar)
-      : "memory");
-}
 
 }  // namespace
 
@@ -164,7 +168,6 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int r = p.r, rh = p.rope_half, lb = r / 128, rhalf = r / 2;
   const PairLayout lay = pair_layout(r, rh, p.nslot);
   uint8_t* slots = base;
-  uint8_t* stage = base + lay.stage_off;
   uint8_t* recv = base + lay.recv_off;
   int* misc = reinterpret_cast<int*>(base + lay.misc_off);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(misc);
@@ -183,6 +186,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t* pv_done = s_free + 1;
   uint64_t* recv_full = pv_done + 1;                   // [2] partner's partial landed
   uint64_t* peer_free = recv_full + 2;                 // [2] partner consumed our partial
+  uint64_t* p_full = peer_free + 2;                    // P of the tile written
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -200,14 +204,15 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int k = 0; k < nb; ++k) mbar_init(&full[s * nb + k], 1);
       mbar_init(&empty[s], 1);
     }
-    mbar_init(q_full, 8);
+    mbar_init(q_full, kSoftWarps);
     mbar_init(s_full, 1);
-    mbar_init(s_free, 8);
+    mbar_init(s_free, kSoftWarps);
     mbar_init(pv_done, 1);
     for (int i = 0; i < 2; ++i) {
       mbar_init(&recv_full[i], 1);
-      mbar_init(&peer_free[i], 8);
+      mbar_init(&peer_free[i], kSoftWarps);
     }
+    mbar_init(p_full, kSoftWarps);
     *abort_flag = 0;
     fence_mbar_init();
     // both receive buffers expect their first partial
@@ -320,23 +325,22 @@ __global__ void __launch_bounds__(kThreads, 1)
         tc_fence_after();
         for (int t = tb; ok && t < te; ++t, ++jj) {
           const int slot = jj % p.nslot;
+          // every block of the tile landed, then the S accumulator free
+          for (int k = 0; ok && k <= lb; ++k)
+            ok = mbar_wait(&full[slot * nb + k], (jj / p.nslot) & 1, wc);
+          if (!ok) break;
+          MLA_PTRACE(1, jj);
           if (jj >= 1 && !mbar_wait(s_free, (jj - 1) & 1, wc)) { ok = false; break; }
           MLA_PTRACE(9, jj);
           tc_fence_after();
           const uint32_t soff = slot * lay.slot_bytes;
           for (int k = 0; k < lb; ++k) {
-            if (!mbar_wait(&full[slot * nb + k], (jj / p.nslot) & 1, wc)) { ok = false; break; }
-            tc_fence_after();
 #pragma unroll
             for (int kk = 0; kk < 4; ++kk)
               umma_bf16_ts(tmem + kColS, tmem + kColQ + (k * 4 + kk) * 8,
                            b0 + ((soff + k * kBlk + kk * 32) >> 4), idesc_s,
                            (k | kk) != 0 ? 1u : 0u);
           }
-          if (!ok) break;
-          if (!mbar_wait(&full[slot * nb + lb], (jj / p.nslot) & 1, wc)) { ok = false; break; }
-          MLA_PTRACE(1, jj);
-          tc_fence_after();
           for (int kk = 0; kk < rh / 16; ++kk)
             umma_bf16_ts(tmem + kColS, tmem + kColQ + (lb * 4 + kk) * 8,
                          br0 + ((soff + kk * 32) >> 4), idesc_s, 1u);
@@ -346,40 +350,67 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
     }
     __syncwarp();
+  } else if (warp == kPvWarp) {
+    // ============================== UMMA issuer for O += P C ==============================
+    if (has_work && elect_one()) {
+      const uint32_t idesc_o = make_idesc_bf16(128, rhalf, 0, 1);
+      // B operand: the latent blocks of the slot read MN-major (latent contiguous)
+      const uint64_t pb0 = make_sdesc(smem_u32(slots), kBlk, 1024, kSw128);
+      UnitWalk w{sched[0], sched[1]};
+      int jj = 0;
+      bool ok = true;
+      for (; ok && w.s < r1; w.s += w.tiles, ++w.b) {
+        w.load(p, cg);
+        const int tb = max(w.s, r0), te = min(w.s + w.tiles, r1);
+        for (int t = tb; t < te; ++t, ++jj) {
+          if (!mbar_wait(p_full, jj & 1, wc)) { ok = false; break; }
+          tc_fence_after();
+          // the first tile of a piece overwrites O: the previous piece's epilogue read O
+          // before its warps arrived on p_full for this tile
+          const bool first = (t == tb);
+          const uint32_t soff = (jj % p.nslot) * lay.slot_bytes;
+#pragma unroll
+          for (int kk = 0; kk < 4; ++kk)
+            umma_bf16_ts(tmem + kColO, tmem + kColP + kk * 8, pb0 + ((soff + kk * 2048) >> 4),
+                         idesc_o, (!first || kk > 0) ? 1u : 0u);
+          umma_commit(pv_done);
+          umma_commit(&empty[jj % p.nslot]);
+          MLA_PTRACE(8, jj);
+        }
+      }
+    }
+    __syncwarp();
   } else if (has_work) {
-    // ============ score exchange, softmax, PV issue, epilogue (row n, half hf) =============
+    // =========== score exchange, softmax, P, epilogue (row n, quarter qt of a tile) ===========
     const int sp = warp & 3;                  // TMEM sub-partition this warp may access
-    const int wi = warp - 2;                  // softmax warp 0..7 (exchange block index)
-    const int hf = wi >> 2;                   // which 32 tokens of a tile / half of O
+    const int wi = warp - 2;                  // softmax warp 0..15 (exchange block index)
+    const int qt = wi >> 2;                   // which 16 tokens of a tile / quarter of O
     const int n = 32 * sp + lane;             // query row of this thread in the block
-    const int tid = threadIdx.x - 64;         // 0..255
+    const int tid = threadIdx.x - 64;         // 0..511
     const uint32_t trow = tmem + (uint32_t(32 * sp) << 16);
-    const uint32_t stage_s = smem_u32(stage);
     const uint32_t recv_s = smem_u32(recv);
     const uint32_t recv_r = map_to_rank(recv_s, peer);
     const uint32_t rfull_r0 = map_to_rank(smem_u32(&recv_full[0]), peer);
     const uint32_t rfull_r1 = map_to_rank(smem_u32(&recv_full[1]), peer);
     const uint32_t pfree_r0 = map_to_rank(smem_u32(&peer_free[0]), peer);
     const uint32_t pfree_r1 = map_to_rank(smem_u32(&peer_free[1]), peer);
-    const uint32_t idesc_o = make_idesc_bf16(128, rhalf, 0, 1);
-    // PV B operand: the latent blocks of the slot read MN-major (latent contiguous)
-    const uint64_t pb0 = make_sdesc(smem_u32(slots), kBlk, 1024, kSw128);
     const float c_log2 = p.scale_log2;
     const int row = cg * kPairRows + n;       // row (i, h) of the sequence's q*H rows
     const bool row_ok = row < p.qH;
     const int qi = row / p.num_heads;
     const bool vec_out = (reinterpret_cast<uintptr_t>(p.o_latent) & 15u) == 0;
-    const int ocol0 = hf * (rhalf / 2);       // this thread's half of the O columns
-    float* hmax = red;                        // [tile parity][half][row]
-    float* hsum = red + 4 * kPairRows;        // [half][row]
-    const uint32_t pair_bar = 2 + sp;         // named barrier of the two warps of rows n
+    const int ocols = rhalf / kQuarters;      // O columns of this thread (16, 32 or 64)
+    const int ocol0 = qt * ocols;
+    float* qmax = red;                        // [tile parity][quarter][row]
+    float* qsum = red + 2 * kQuarters * kPairRows;   // [quarter][row]
+    const uint32_t grp_bar = 2 + sp;          // named barrier of the four warps of rows n
 
-    // Q half of this thread's row into TMEM (16-element chunks alternate between the two
-    // threads of the row): latent half, then rotary half; zero rows past q*H. Ends with
-    // this warp's arrival on q_full.
+    // Q half of this thread's row into TMEM (16-element chunks dealt round-robin to the
+    // four threads of the row): latent half, then rotary half; zero rows past q*H. Ends
+    // with this warp's arrival on q_full.
     auto load_q = [&](int b) {
       const uint16_t* q = p.q_ext + (int64_t(b) * p.qH + row) * p.D;
-      for (int c0 = 16 * hf; c0 < rhalf + rh; c0 += 32) {
+      for (int c0 = 16 * qt; c0 < rhalf + rh; c0 += 16 * kQuarters) {
         const int src = c0 < rhalf ? int(rank) * rhalf + c0 : r + int(rank) * rh + (c0 - rhalf);
         uint32_t v[8];
         if (row_ok) {
@@ -406,6 +437,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     sw.load(p, cg);
     int st_t = max(sw.s, r0);                // next tile to send (row-block tile index)
     int js = 0;                              // tiles sent so far
+    // this thread's packed partial of the tile last sent (own_next) and of the tile whose
+    // scores are formed now (own_cur): the own contribution never leaves the registers
+    uint32_t own_next[kPackWords], own_cur[kPackWords];
     load_q(sw.b);
     auto send_next = [&]() -> bool {
       if (st_t >= min(sw.s + sw.tiles, r1)) {
@@ -417,44 +451,38 @@ __global__ void __launch_bounds__(kThreads, 1)
         load_q(sw.b);
       }
       const int kb = js & 1;
-      uint32_t pw[kPackWords];
+      uint32_t* pw = own_next;                 // kept for this tile's own contribution
       {
-        float x[kHalfTok];
+        float x[kQTok];
         const bool got = __all_sync(0xffffffffu, mbar_wait(s_full, js & 1, wc));
         if (got) {
           tc_fence_after();
-          tmem_ld32(trow + kColS + hf * kHalfTok, x);
+          tmem_ld_part(trow + kColS + qt * kQTok, x);
           tmem_wait_ld();
         } else {
 #pragma unroll
-          for (int c = 0; c < kHalfTok; ++c) x[c] = 0.0f;
+          for (int c = 0; c < kQTok; ++c) x[c] = 0.0f;
         }
         if (threadIdx.x == 64) MLA_PTRACE(3, js);
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(s_free);    // the S accumulator may be overwritten
 #pragma unroll
-        for (int g = 0; g < kHalfTok / 4; ++g) pack_f24(x + 4 * g, pw + 3 * g);
+        for (int g = 0; g < kQTok / 4; ++g) pack_f24(x + 4 * g, pw + 3 * g);
       }
-      // The partner has consumed the partial this stage buffer held (tile js - 2), so the
-      // bulk copy that read it has completed and the buffer may be rewritten.
+      // Into the partner's receive buffer once the partner has consumed tile js - 2 from
+      // it: stores from registers over the SM-to-SM network, each completing its bytes on
+      // the partner's mbarrier.
       const bool free_ok = __all_sync(
           0xffffffffu, js < 2 || mbar_wait_cluster(&peer_free[kb], ((js - 2) >> 1) & 1, wc));
-      const uint32_t st_base = stage_s + kb * kXBytes;
       if (free_ok) {
+        const uint32_t dst = recv_r + kb * kXBytes;
+        const uint32_t rb = kb ? rfull_r1 : rfull_r0;
 #pragma unroll
         for (int c = 0; c < kPackWords / 4; ++c)
-          asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(
-                           st_base + x_offset(wi, lane, c)),
-                       "r"(pw[4 * c]), "r"(pw[4 * c + 1]), "r"(pw[4 * c + 2]), "r"(pw[4 * c + 3])
-                       : "memory");
-        fence_proxy_async_smem();
+          st_async_v4(dst + x_offset(wi, lane, c),
+                      make_uint4(pw[4 * c], pw[4 * c + 1], pw[4 * c + 2], pw[4 * c + 3]), rb);
       }
-      __syncwarp();
-      // Lane 31 issues the copy; the arrivals below come from other lanes.
-      if (lane == 31 && free_ok)
-        bulk_copy_to_peer(recv_r + kb * kXBytes + wi * kXWarpBytes, st_base + wi * kXWarpBytes,
-                          kXWarpBytes, kb ? rfull_r1 : rfull_r0);
       if (threadIdx.x == 64) MLA_PTRACE(4, js);
       ++js;
       ++st_t;
@@ -470,67 +498,68 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int L = w.L;
       // last position row n sees (causal: L - q + i); rows past q*H see L - 1
       const int lim = min(L - 1, p.causal ? L - p.q_len + qi : L - 1);
-      float m = kRefInit, l = 0.0f;          // m identical in both threads of a row
+      float m = kRefInit, l = 0.0f;          // m identical in the four threads of a row
       for (int t = tb; t < te; ++t, ++jj) {
-        const int kb = jj & 1;                 // stage / receive buffer of this tile
+        const int kb = jj & 1;                 // receive buffer of this tile
         const int slot = jj % p.nslot;
-        const int pos0 = (t - w.s) * kDecodeTok + hf * kHalfTok;   // first token of the half
+        const int tile_pos0 = (t - w.s) * kDecodeTok;
+        const int pos0 = tile_pos0 + qt * kQTok;   // first token of this thread's quarter
         // ---- send the next tile's partial before finishing this one ----
+#pragma unroll
+        for (int i = 0; i < kPackWords; ++i) own_cur[i] = own_next[i];
         if (sending) sending = send_next();
         // ---- this tile's scores: own rounded partial + the partner's ----
         const bool rcv =
             __all_sync(0xffffffffu, mbar_wait_cluster(&recv_full[kb], (jj >> 1) & 1, wc));
         if (threadIdx.x == 64) MLA_PTRACE(5, jj);
-        float s[kHalfTok];
+        float s[kQTok];
         {
-          const uint32_t own = stage_s + kb * kXBytes, oth = recv_s + kb * kXBytes;
+          const uint32_t oth = recv_s + kb * kXBytes;
+          uint32_t wb[kPackWords];
 #pragma unroll
-          for (int c = 0; c < kPackWords / 4; c += 3) {
-            // three chunks = 12 words = 16 values
-            uint32_t wa[12], wb[12];
+          for (int c = 0; c < kPackWords / 4; ++c) {
+            const uint4 vb = ld_shared_v4(oth + x_offset(wi, lane, c));
+            wb[4 * c] = vb.x; wb[4 * c + 1] = vb.y; wb[4 * c + 2] = vb.z; wb[4 * c + 3] = vb.w;
+          }
 #pragma unroll
-            for (int i = 0; i < 3; ++i) {
-              const uint4 va = ld_shared_v4(own + x_offset(wi, lane, c + i));
-              const uint4 vb = ld_shared_v4(oth + x_offset(wi, lane, c + i));
-              wa[4 * i] = va.x; wa[4 * i + 1] = va.y; wa[4 * i + 2] = va.z; wa[4 * i + 3] = va.w;
-              wb[4 * i] = vb.x; wb[4 * i + 1] = vb.y; wb[4 * i + 2] = vb.z; wb[4 * i + 3] = vb.w;
-            }
+          for (int g = 0; g < kQTok / 4; ++g) {
+            float fa[4], fb[4];
+            unpack_f24(own_cur + 3 * g, fa);
+            unpack_f24(wb + 3 * g, fb);
 #pragma unroll
-            for (int g = 0; g < 4; ++g) {
-              float fa[4], fb[4];
-              unpack_f24(wa + 3 * g, fa);
-              unpack_f24(wb + 3 * g, fb);
-              const int v0 = (c / 3) * 16 + 4 * g;
-#pragma unroll
-              for (int i = 0; i < 4; ++i) s[v0 + i] = rcv ? fa[i] + fb[i] : 0.0f;
-            }
+            for (int i = 0; i < 4; ++i) s[4 * g + i] = rcv ? fa[i] + fb[i] : 0.0f;
           }
         }
         if (threadIdx.x == 64) MLA_PTRACE(10, jj);
         __syncwarp();
         // The received words are in registers (consumed above): release the buffer to the
-        // partner without a release fence, which would wait for this warp's bulk copy.
+        // partner without a release fence, which would wait for this warp's remote stores.
         if (lane == 1) mbar_arrive_remote_relaxed(kb ? pfree_r1 : pfree_r0);
-        // re-arm this buffer for tile jj + 2 (the partner sends it only after all eight
+        // re-arm this buffer for tile jj + 2 (the partner sends it only after all sixteen
         // warps have released the buffer above)
         if (threadIdx.x == 65 && rcv) mbar_arrive_expect_tx_relaxed(&recv_full[kb], kXBytes);
 
         // ---- online softmax of row n over this tile (log2 domain, lazy reference) ----
-        if (pos0 + kHalfTok - 1 > lim) {
+        if (pos0 + kQTok - 1 > lim) {
 #pragma unroll
-          for (int c = 0; c < kHalfTok; ++c)
+          for (int c = 0; c < kQTok; ++c)
             if (pos0 + c > lim) s[c] = -INFINITY;
         }
-        float mh = -INFINITY;
+        // maximum of the raw scores (a tree; the positive scale is applied once after it)
+        float mt[kQTok / 2];
 #pragma unroll
-        for (int c = 0; c < kHalfTok; ++c) {
-          s[c] *= c_log2;
-          mh = fmaxf(mh, s[c]);
-        }
-        // the row's maximum over both halves (same value in both threads)
-        hmax[(kb * 2 + hf) * kPairRows + n] = mh;
-        named_bar_sync(pair_bar, 64);
-        const float mx = fmaxf(mh, hmax[(kb * 2 + (hf ^ 1)) * kPairRows + n]);
+        for (int c = 0; c < kQTok / 2; ++c) mt[c] = fmaxf(s[c], s[c + kQTok / 2]);
+#pragma unroll
+        for (int w2 = kQTok / 4; w2 >= 1; w2 >>= 1)
+#pragma unroll
+          for (int c = 0; c < w2; ++c) mt[c] = fmaxf(mt[c], mt[c + w2]);
+        // the row's maximum over the four quarters (same value in all four threads)
+        qmax[(kb * kQuarters + qt) * kPairRows + n] = mt[0] * c_log2;
+        named_bar_sync(grp_bar, 32 * kQuarters);
+        const float* qm = qmax + kb * kQuarters * kPairRows + n;
+        float mx = qm[0];
+#pragma unroll
+        for (int q = 1; q < kQuarters; ++q) mx = fmaxf(mx, qm[q * kPairRows]);
         if (threadIdx.x == 64) MLA_PTRACE(11, jj);
         float alpha = 1.0f;
         if (mx > m + kLazyThreshold) {
@@ -544,28 +573,31 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (threadIdx.x == 64) MLA_PTRACE(6, jj);
         tc_fence_after();
         if (t > tb && pv_ok && __any_sync(0xffffffffu, alpha != 1.0f)) {
-          for (int c0 = 0; c0 < rhalf / 2; c0 += 32) {
-            float o[32];
-            tmem_ld32(trow + kColO + ocol0 + c0, o);
+          for (int c0 = 0; c0 < ocols; c0 += 16) {
+            float o[16];
+            tmem_ld16(trow + kColO + ocol0 + c0, o);
             tmem_wait_ld();
 #pragma unroll
-            for (int c = 0; c < 32; ++c) o[c] *= alpha;
-            tmem_st32(trow + kColO + ocol0 + c0, reinterpret_cast<const uint32_t*>(o));
+            for (int c = 0; c < 16; ++c) o[c] *= alpha;
+            tmem_st16(trow + kColO + ocol0 + c0, o);
           }
         }
-        uint32_t pk[kHalfTok / 2];
+        // weights 2^(s * scale - m); the tile's sum in two chains, added to l in a fixed
+        // order (both CTAs of the pair agree bit for bit)
+        uint32_t pk[kQTok / 2];
+        float sa = 0.0f, sb = 0.0f;
 #pragma unroll
-        for (int c = 0; c < kHalfTok / 2; ++c) {
-          const float p0 = ex2_approx(s[2 * c] - m);
-          const float p1 = ex2_approx(s[2 * c + 1] - m);
-          l += p0;
-          l += p1;
+        for (int c = 0; c < kQTok / 2; ++c) {
+          const float p0 = ex2_approx(fmaf(s[2 * c], c_log2, -m));
+          const float p1 = ex2_approx(fmaf(s[2 * c + 1], c_log2, -m));
+          sa += p0;
+          sb += p1;
           pk[c] = cvt_bf16x2(p0, p1);
         }
-        tmem_st16(trow + kColP + hf * (kHalfTok / 2), reinterpret_cast<const float*>(pk));
+        l += sa + sb;
+        tmem_st_part(trow + kColP + qt * (kQTok / 2), pk);
         // cache rows past the context may hold anything (even NaN): zero their latent half
         // so that 0-weight x garbage cannot reach O
-        const int tile_pos0 = (t - w.s) * kDecodeTok;
         if (tile_pos0 + kDecodeTok > L) {
           const int tok = tid & (kDecodeTok - 1);
           if (tile_pos0 + tok >= L) {
@@ -577,53 +609,44 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
           }
         }
+        // P (and any O rescale and zeroed rows) complete: hand the tile to the PV issuer
         tmem_wait_st();
         if (threadIdx.x == 64) MLA_PTRACE(7, jj);
         fence_proxy_async_smem();
         tc_fence_before();
-        named_bar_sync(1, kSoftThreads);
-        if (threadIdx.x == 64) {
-          // O += P C_half for this tile; the first tile of a piece overwrites O (the
-          // previous piece's epilogue reads finished before the barrier above)
-          tc_fence_after();
-          const bool first = (t == tb);
-          const uint32_t soff = slot * lay.slot_bytes;
-#pragma unroll
-          for (int kk = 0; kk < 4; ++kk)
-            umma_bf16_ts(tmem + kColO, tmem + kColP + kk * 8, pb0 + ((soff + kk * 2048) >> 4),
-                         idesc_o, (!first || kk > 0) ? 1u : 0u);
-          umma_commit(pv_done);
-          umma_commit(&empty[slot]);
-          MLA_PTRACE(8, jj);
-        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(p_full);
       }
 
       // ---------------------------- epilogue of this piece --------------------------------
       const bool fin = __all_sync(0xffffffffu, mbar_wait(pv_done, (jj - 1) & 1, wc));
       tc_fence_after();
       const bool aborted = __any_sync(0xffffffffu, !fin || *abort_flag != 0);
-      hsum[hf * kPairRows + n] = l;
-      named_bar_sync(pair_bar, 64);
-      const float lt = l + hsum[(hf ^ 1) * kPairRows + n];   // same sum in both threads
-      named_bar_sync(pair_bar, 64);                          // hsum may be reused
+      qsum[qt * kPairRows + n] = l;
+      named_bar_sync(grp_bar, 32 * kQuarters);
+      // the row sum, added in the same order by every thread of the row
+      float lt = qsum[n];
+#pragma unroll
+      for (int q = 1; q < kQuarters; ++q) lt += qsum[q * kPairRows + n];
+      named_bar_sync(grp_bar, 32 * kQuarters);               // qsum may be reused
       const bool whole = (tb == w.s) && (te == w.s + w.tiles);
       const int64_t grow = int64_t(w.b) * p.qH + row;   // global (b, i, h) row
       const int pslot = piece_slot(vc, w.s, per, p.col_groups, cg);
       const float lse = (lt > 0.0f && !aborted) ? (m + __log2f(lt)) * kLn2 : -INFINITY;
-      if (row_ok && rank == 0 && hf == 0) {
+      if (row_ok && rank == 0 && qt == 0) {
         if (whole) p.lse[grow] = lse;
         else p.part_lse[int64_t(pslot) * kPairRows + n] = lse;
       }
       const float inv = (lt > 0.0f && !aborted) ? 1.0f / lt : 0.0f;
       const int64_t lat0 = int64_t(rank) * rhalf + ocol0;
-      for (int c0 = 0; c0 < rhalf / 2; c0 += 32) {
-        float o[32];
+      for (int c0 = 0; c0 < ocols; c0 += 16) {
+        float o[16];
         if (!aborted) {
-          tmem_ld32(trow + kColO + ocol0 + c0, o);
+          tmem_ld16(trow + kColO + ocol0 + c0, o);
           tmem_wait_ld();
         } else {
 #pragma unroll
-          for (int c = 0; c < 32; ++c) o[c] = 0.0f;
+          for (int c = 0; c < 16; ++c) o[c] = 0.0f;
         }
         if (!row_ok) {
           // padding row past q*H: nothing to write
@@ -631,7 +654,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           uint16_t* dst = p.o_latent + grow * r + lat0 + c0;
           if (vec_out) {
 #pragma unroll
-            for (int c = 0; c < 32; c += 8)
+            for (int c = 0; c < 16; c += 8)
               *reinterpret_cast<uint4*>(dst + c) =
                   make_uint4(cvt_bf16x2(o[c] * inv, o[c + 1] * inv),
                              cvt_bf16x2(o[c + 2] * inv, o[c + 3] * inv),
@@ -639,12 +662,12 @@ __global__ void __launch_bounds__(kThreads, 1)
                              cvt_bf16x2(o[c + 6] * inv, o[c + 7] * inv));
           } else {
 #pragma unroll
-            for (int c = 0; c < 32; ++c) dst[c] = f32_to_bf16_rne(o[c] * inv);
+            for (int c = 0; c < 16; ++c) dst[c] = f32_to_bf16_rne(o[c] * inv);
           }
         } else {
           float* dst = p.part_o + (int64_t(pslot) * kPairRows + n) * r + lat0 + c0;
 #pragma unroll
-          for (int c = 0; c < 32; c += 4)
+          for (int c = 0; c < 16; c += 4)
             *reinterpret_cast<float4*>(dst + c) =
                 make_float4(o[c] * inv, o[c + 1] * inv, o[c + 2] * inv, o[c + 3] * inv);
         }
