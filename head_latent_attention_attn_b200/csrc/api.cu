@@ -405,6 +405,7 @@ mla_status mla_decode_attn(const mla_dims* dims, const void* q_ext, const void* 
     c.ncol = P.ncol;
     c.col_groups = P.col_groups;
     c.units = P.units;
+    c.vgrid = P.vgrid;
     if (launch_combine(c, s) != cudaSuccess) return MLA_ERR_CUDA;
   }
   return MLA_OK;

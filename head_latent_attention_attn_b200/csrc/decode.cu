@@ -56,6 +56,7 @@ namespace {
 constexpr int kThreads = 192;
 constexpr int kBlkBytes = kDecodeTok * 128;   // one 64 x 64 bf16 block, 8 KB
 constexpr float kLazyThreshold = 8.0f;        // log2 units
+constexpr int kPrefetchTiles = 4;             // tiles brought into L2 ahead of their load
 // Initial reference max: finite, so a masked score (-inf) minus it is exactly -inf (weight
 // 0) and any finite score exceeds it, forcing the first real reference to be computed.
 constexpr float kRefInit = -3.0e38f;
@@ -234,6 +235,29 @@ __global__ void __launch_bounds__(kThreads, 1)
       prefetch_tensormap(&p.tm_q);
       if (blockIdx.x == 0) *p.range_len = per;
       UnitWalk w{sched[0], sched[1]};
+      // L2 prefetch walk, kPrefetchTiles tiles ahead of the loads (row block 0 only: the
+      // other row blocks read the same pages in lockstep): only one or two tiles fit in
+      // shared memory, too little lead time to hide DRAM latency behind the loads alone.
+      UnitWalk pf{sched[0], sched[1]};
+      pf.load(p, cg);
+      int pf_t = max(pf.s, r0), pf_n = 0;
+      auto prefetch_upto = [&](int upto) {
+        while (cg == 0 && pf_n < upto && pf.s < r1) {
+          if (pf_t >= min(pf.s + pf.tiles, r1)) {
+            pf.s += pf.tiles;
+            ++pf.b;
+            if (pf.s >= r1) break;
+            pf.load(p, cg);
+            pf_t = pf.s;
+          }
+          const int32_t page = p.block_table[int64_t(pf.b) * p.max_pages + (pf_t - pf.s)];
+          if (page >= 0 && page < p.num_pages)
+            for (int k = 0; k < p.nblk; ++k)
+              tma_prefetch_l2_2d(&p.tm_cache, k * 64, page * kDecodeTok);
+          ++pf_t;
+          ++pf_n;
+        }
+      };
       int jj = 0, pc = 0;
       bool ok = true;
       for (; ok && w.s < r1; w.s += w.tiles, ++w.b, ++pc) {
@@ -263,6 +287,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             mbar_arrive_expect_tx(fb, kBlkBytes);
             tma_load_2d(sbase + k * kBlkBytes, &p.tm_cache, k * 64, page * kDecodeTok, fb);
           }
+          // after the loads: a prefetch queued ahead of them would delay them
+          prefetch_upto(jj + 1 + kPrefetchTiles);
           MLA_TRACE_AT(8, jj);
         }
       }
@@ -651,6 +677,80 @@ __global__ void __launch_bounds__(128) mla_combine_kernel(const CombineParams p)
   if (threadIdx.x == 0) p.lse[int64_t(b) * p.qH + f] = lse;
 }
 
+// The same merge with one warp per (unit, query row), four rows per block: for units cut
+// into a few pieces. Lanes own latents 4 * lane + 128 k + {0..3}: every load of a piece's
+// row is one 512-byte coalesced segment per warp.
+__global__ void __launch_bounds__(128) mla_combine_rows_kernel(const CombineParams p) {
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int64_t gw = int64_t(blockIdx.x) * 4 + warp;
+  if (gw >= int64_t(p.units) * p.ncol) return;
+  const int u = int(gw / p.ncol);
+  const int n = int(gw - int64_t(u) * p.ncol);
+  const int G = p.col_groups;
+  const int b = u / G, cg = u - b * G;
+  const int f = cg * p.ncol + n;
+  if (f >= p.qH) return;
+  int L = p.seq_lens[b];
+  const bool ok = L >= p.q_len && L <= p.max_seq_len && int64_t(L) <= int64_t(p.max_pages) * kDecodeTok;
+  if (!ok) L = 0;
+  const int tiles = L > 0 ? (L + kDecodeTok - 1) / kDecodeTok : 1;
+  const int per = *p.range_len;
+  const int s = p.unit_start[u];
+  const int i0 = s / per, i1 = (s + tiles - 1) / per;
+  if (i0 == i1) return;   // held whole by one range: already written
+  float mx = -INFINITY;
+  for (int i = i0 + lane; i <= i1; i += 32)
+    mx = fmaxf(mx, p.part_lse[int64_t(piece_slot(i, s, per, G, cg)) * p.ncol + n]);
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+  float den = 0.0f;
+  for (int i = i0 + lane; i <= i1; i += 32) {
+    const float li = p.part_lse[int64_t(piece_slot(i, s, per, G, cg)) * p.ncol + n];
+    den += li == -INFINITY ? 0.0f : expf(li - mx);
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) den += __shfl_xor_sync(0xffffffffu, den, o);
+  const float lse = mx == -INFINITY ? -INFINITY : mx + logf(den);
+  float4 acc[4];
+#pragma unroll
+  for (int k = 0; k < 4; ++k) acc[k] = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+  for (int i = i0; i <= i1; ++i) {
+    const int64_t sl = piece_slot(i, s, per, G, cg);
+    const float li = p.part_lse[sl * p.ncol + n];
+    if (li == -INFINITY) continue;
+    const float wgt = expf(li - lse);
+    const float* row = p.part_o + (sl * p.ncol + n) * p.r;
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      const int lat = 4 * lane + 128 * k;
+      if (lat < p.r) {
+        const float4 v = *reinterpret_cast<const float4*>(row + lat);
+        acc[k].x += wgt * v.x;
+        acc[k].y += wgt * v.y;
+        acc[k].z += wgt * v.z;
+        acc[k].w += wgt * v.w;
+      }
+    }
+  }
+  uint16_t* out = p.o_latent + (int64_t(b) * p.qH + f) * p.r;
+  const bool vec = (reinterpret_cast<uintptr_t>(out) & 7u) == 0;
+#pragma unroll
+  for (int k = 0; k < 4; ++k) {
+    const int lat = 4 * lane + 128 * k;
+    if (lat >= p.r) continue;
+    if (vec) {
+      *reinterpret_cast<uint2*>(out + lat) =
+          make_uint2(cvt_bf16x2(acc[k].x, acc[k].y), cvt_bf16x2(acc[k].z, acc[k].w));
+    } else {
+      out[lat] = f32_to_bf16_rne(acc[k].x);
+      out[lat + 1] = f32_to_bf16_rne(acc[k].y);
+      out[lat + 2] = f32_to_bf16_rne(acc[k].z);
+      out[lat + 3] = f32_to_bf16_rne(acc[k].w);
+    }
+  }
+  if (lane == 0) p.lse[int64_t(b) * p.qH + f] = lse;
+}
+
 #ifdef MLA_TRACE
 extern "C" int mla_trace_read(unsigned long long* host, int n) {
   return int(cudaMemcpyFromSymbol(host, g_mla_trace, sizeof(unsigned long long) *
@@ -659,9 +759,15 @@ extern "C" int mla_trace_read(unsigned long long* host, int n) {
 #endif
 
 cudaError_t launch_combine(const CombineParams& p, cudaStream_t stream) {
-  const int64_t blocks = int64_t(p.units) * p.ncol;
-  if (blocks <= 0 || blocks > 0x7fffffffLL) return cudaErrorInvalidValue;
-  mla_combine_kernel<<<unsigned(blocks), 128, 0, stream>>>(p);
+  const int64_t rows = int64_t(p.units) * p.ncol;
+  if (rows <= 0 || rows > 0x7fffffffLL || p.r > 512 || p.r % 4 != 0) return cudaErrorInvalidValue;
+  if (int64_t(p.vgrid) <= 4 * int64_t(p.units)) {
+    // a few pieces per unit: one warp per row
+    mla_combine_rows_kernel<<<unsigned((rows + 3) / 4), 128, 0, stream>>>(p);
+  } else {
+    // many pieces per unit: the four warps of a block split one row's pieces
+    mla_combine_kernel<<<unsigned(rows), 128, 0, stream>>>(p);
+  }
   return cudaGetLastError();
 }
 

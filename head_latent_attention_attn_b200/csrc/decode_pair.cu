@@ -278,7 +278,6 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int32_t* bt = p.block_table + int64_t(w.b) * p.max_pages;
         for (int t = tb; t < te; ++t, ++jj) {
           const int slot = jj % p.nslot;
-          prefetch_upto(jj + 1 + kPrefetchAhead);
           if (jj >= p.nslot && !mbar_wait(&empty[slot], ((jj / p.nslot) - 1) & 1, wc)) {
             ok = false;
             break;
@@ -299,6 +298,8 @@ __global__ void __launch_bounds__(kThreads, 1)
           mbar_arrive_expect_tx(fb, rope_bytes);
           tma_load_2d(sbase + lay.rope_off, &p.tm_rope, r + int(rank) * rh, page * kDecodeTok,
                       fb);
+          // after the load: a prefetch queued ahead of it would delay it
+          prefetch_upto(jj + 1 + kPrefetchAhead);
           MLA_PTRACE(0, jj);
         }
       }

@@ -90,6 +90,7 @@ struct CombineParams {
   uint16_t* o_latent;
   float* lse;
   int32_t q_len, max_seq_len, max_pages, qH, r, ncol, col_groups, units;
+  int32_t vgrid;             // work ranges the decode used (pieces per unit ~ vgrid / units)
 };
 cudaError_t launch_combine(const CombineParams& p, cudaStream_t stream);
 
