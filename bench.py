@@ -126,22 +126,37 @@ class ClockSampler:
                 "reasons": sorted(reasons)}
 
 
-def _source_hash():
+def uses_pair_kernel(cfg):
+    """True when mla_decode_attn runs this shape on the two-CTA latent-split kernel (more than
+    64 query rows, rank a multiple of 128, rotary columns of 32, 64 or 128)."""
+    rope = cfg.num_kv_groups * cfg.rope_dim
+    return (cfg.q_len * cfg.num_heads > 64 and cfg.kv_lora_rank % 128 == 0
+            and rope in (32, 64, 128))
+
+
+def decode_kernel_name(cfg):
+    return "mla_decode_pair_kernel" if uses_pair_kernel(cfg) else "mla_decode_kernel"
+
+
+def _source_hash(cfg):
+    """Hash of the sources of the decode kernel that runs this shape."""
+    files = ("decode_pair.cu" if uses_pair_kernel(cfg) else "decode.cu",
+             "decode_sched.cuh", "ptx.cuh", "kernels.h")
     h = hashlib.sha256()
-    for f in ("decode.cu", "decode_pair.cu", "decode_sched.cuh", "ptx.cuh", "kernels.h"):
+    for f in files:
         h.update(open(os.path.join(ROOT, "head_latent_attention_attn_b200", "csrc", f), "rb").read())
     return h.hexdigest()[:16]
 
 
-def _traffic(config_name):
-    """Per-launch DRAM bytes of mla_decode_attn from a committed ncu summary, if it was taken
-    on the current kernel source; else None."""
+def _traffic(cfg):
+    """Per-launch DRAM bytes of the decode kernel from a committed ncu summary, if it was
+    taken on the current kernel source; else None."""
     path = os.path.join(ROOT, "profiles", "decode_traffic.json")
     if not os.path.exists(path):
         return None
     d = json.load(open(path))
-    e = d.get(config_name)
-    if not e or e.get("source_hash") != _source_hash():
+    e = d.get(cfg.name)
+    if not e or e.get("source_hash") != _source_hash(cfg):
         return None
     return e.get("dram_bytes_per_launch")
 
@@ -327,9 +342,9 @@ def run_gpu(args, cfg, rank, world, dist):
     else:
         roof = {"bound": "tensor", "achieved": tfl, "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
                 "frac": tfl / peaks["bf16_tflops"]}
-    roof["traffic"] = _traffic(cfg.name)
+    roof["traffic"] = _traffic(cfg)
     roof["peak_source"] = peaks["source"]
-    roof["kernel"] = "mla_decode_attn (decode kernel + split combine when splits > 1)"
+    roof["kernel"] = decode_kernel_name(cfg) + " (+ merge of cut units when the work is split)"
     roof["algorithmic_bytes_per_launch"] = nbytes
     roof["algorithmic_flops_per_launch"] = flops
     roof["roofline_time_us"] = 1e6 * max(t_hbm, t_tc)

@@ -56,7 +56,6 @@ namespace {
 constexpr int kThreads = 192;
 constexpr int kBlkBytes = kDecodeTok * 128;   // one 64 x 64 bf16 block, 8 KB
 constexpr float kLazyThreshold = 8.0f;        // log2 units
-constexpr int kPrefetchTiles = 4;             // tiles brought into L2 ahead of their load
 // Initial reference max: finite, so a masked score (-inf) minus it is exactly -inf (weight
 // 0) and any finite score exceeds it, forcing the first real reference to be computed.
 constexpr float kRefInit = -3.0e38f;
@@ -235,29 +234,6 @@ __global__ void __launch_bounds__(kThreads, 1)
       prefetch_tensormap(&p.tm_q);
       if (blockIdx.x == 0) *p.range_len = per;
       UnitWalk w{sched[0], sched[1]};
-      // L2 prefetch walk, kPrefetchTiles tiles ahead of the loads (row block 0 only: the
-      // other row blocks read the same pages in lockstep): only one or two tiles fit in
-      // shared memory, too little lead time to hide DRAM latency behind the loads alone.
-      UnitWalk pf{sched[0], sched[1]};
-      pf.load(p, cg);
-      int pf_t = max(pf.s, r0), pf_n = 0;
-      auto prefetch_upto = [&](int upto) {
-        while (cg == 0 && pf_n < upto && pf.s < r1) {
-          if (pf_t >= min(pf.s + pf.tiles, r1)) {
-            pf.s += pf.tiles;
-            ++pf.b;
-            if (pf.s >= r1) break;
-            pf.load(p, cg);
-            pf_t = pf.s;
-          }
-          const int32_t page = p.block_table[int64_t(pf.b) * p.max_pages + (pf_t - pf.s)];
-          if (page >= 0 && page < p.num_pages)
-            for (int k = 0; k < p.nblk; ++k)
-              tma_prefetch_l2_2d(&p.tm_cache, k * 64, page * kDecodeTok);
-          ++pf_t;
-          ++pf_n;
-        }
-      };
       int jj = 0, pc = 0;
       bool ok = true;
       for (; ok && w.s < r1; w.s += w.tiles, ++w.b, ++pc) {
@@ -287,8 +263,6 @@ __global__ void __launch_bounds__(kThreads, 1)
             mbar_arrive_expect_tx(fb, kBlkBytes);
             tma_load_2d(sbase + k * kBlkBytes, &p.tm_cache, k * 64, page * kDecodeTok, fb);
           }
-          // after the loads: a prefetch queued ahead of them would delay them
-          prefetch_upto(jj + 1 + kPrefetchTiles);
           MLA_TRACE_AT(8, jj);
         }
       }
