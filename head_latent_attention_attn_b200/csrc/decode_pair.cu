@@ -26,8 +26,10 @@
 // Roles (352 threads per CTA): warp 0 TMA producer, warp 1 S issuer and TMEM owner, warps
 // 2-9 the score exchange, softmax, P into TMEM and the epilogue, warp 10 the PV issuer.
 // The M=128 accumulator puts row n on TMEM lane n, and a warp reaches only the 32 lanes of
-// its sub-partition (warp % 4), so two warps share every 32 rows: softmax warp wi takes
-// tokens [32 q, 32 q + 32) of each tile, q = wi / 4, one thread per (row, part).
+// its sub-partition (warp % 4); with 16x32bx2 TMEM accesses a warp covers 16 rows with two
+// threads each (lanes i and i + 16: tokens 0-31 and 32-63 of every tile), so the row's
+// maximum and sum need one shuffle, and the two warps of a sub-partition take its lanes
+// 0-15 and 16-31.
 //
 // TMEM columns: O [0, r/2), S [256, 320), P [320, 352) (bf16 pairs), Q [352, 352 +
 // (r/2 + rope_half)/2) (bf16 pairs: latent half, then rotary half).
@@ -62,12 +64,12 @@ __device__ unsigned long long g_mla_pair_trace[kPairTraceEvents * kPairTraceTile
 
 namespace {
 
-constexpr int kQuarters = 2;                                   // softmax threads per row
-constexpr int kSoftWarps = 4 * kQuarters;                      // warps 2 .. 2 + kSoftWarps
+constexpr int kRowThreads = 2;                                   // softmax threads per row
+constexpr int kSoftWarps = 8;                                  // 16 rows per warp
 constexpr int kSoftThreads = 32 * kSoftWarps;
 constexpr int kPvWarp = 2 + kSoftWarps;
 constexpr int kThreads = 32 * (kPvWarp + 1);
-constexpr int kQTok = kDecodeTok / kQuarters;                  // tokens per softmax thread
+constexpr int kQTok = kDecodeTok / kRowThreads;                  // tokens per softmax thread
 constexpr uint32_t kBlk = kDecodeTok * 128;                    // 64 x 64 bf16 block, 8 KB
 constexpr int kPackWords = kQTok * 3 / 4;                      // 24-bit values of one part
 constexpr uint32_t kXWarpBytes = 32u * kPackWords * 4;          // one warp's parts
@@ -81,7 +83,7 @@ constexpr float kLn2 = 0.69314718055994530942f;
 constexpr int kMiscInts = 32;
 
 struct PairLayout {
-  uint32_t slot_bytes, rope_off, recv_off, red_off, misc_off, bar_off, total;
+  uint32_t slot_bytes, rope_off, recv_off, misc_off, bar_off, total;
   int nb;   // TMA barriers per slot: one per latent block and one for the rotary block
 };
 
@@ -100,9 +102,6 @@ __host__ __device__ inline PairLayout pair_layout(int r, int rope_half, int nslo
   uint32_t off = uint32_t(nslot) * L.slot_bytes;
   L.recv_off = off;                               // partner's packed partials (two tiles)
   off += 2 * kXBytes;
-  L.red_off = off;                                // float part maxima [2][parts][128]
-  off += 2 * kQuarters * kPairRows * 4;           // and part sums [parts][128]
-  off += kQuarters * kPairRows * 4;
   L.misc_off = off;
   off += 4 * kMiscInts;
   L.bar_off = round_up_p(off, 8);
@@ -120,26 +119,15 @@ MLA_DEVICE SmemSwizzle rope_swizzle(int rope_half) {
 }
 
 // Byte offset of 16-byte chunk c (packed words 4c..4c+3) of lane `lane` of softmax warp
-// wi in a receive buffer: each warp's part rows are one contiguous block, chunk-major
-// inside it, so a quarter-warp touches 128 consecutive bytes.
+// wi in a receive buffer: each warp's 32 (row, token half) threads are one contiguous
+// block, chunk-major inside it, so a quarter-warp touches 128 consecutive bytes.
 MLA_DEVICE uint32_t x_offset(int wi, int lane, int c) {
   return uint32_t(wi) * kXWarpBytes + uint32_t(c) * 512u + uint32_t(lane) * 16u;
 }
 
-// TMEM loads of one part's scores (kQTok fp32 columns) and stores of its weights
-// (kQTok / 2 columns of bf16 pairs).
-MLA_DEVICE void tmem_ld_part(uint32_t taddr, float* v) {
-  if constexpr (kQTok == 32) tmem_ld32(taddr, v);
-  else tmem_ld16(taddr, v);
-}
-MLA_DEVICE void tmem_st_part(uint32_t taddr, const uint32_t* w) {
-  if constexpr (kQTok == 32) tmem_st16(taddr, reinterpret_cast<const float*>(w));
-  else tmem_st8(taddr, w);
-}
-
-// Four 24-bit values (fp32 rounded to sign, exponent and a 15-bit mantissa) in three words (value k's three bytes follow value k-1's), and back
-// to fp32 with a zero low byte. Rounding adds half of the dropped byte; the byte moves are
-// single byte permutes.
+// Four 24-bit values (fp32 rounded to sign, exponent and a 15-bit mantissa) in three words
+// (value k's three bytes follow value k-1's), and back to fp32 with a zero low byte.
+// Rounding adds half of the dropped byte; the byte moves are single byte permutes.
 MLA_DEVICE void pack_f24(const float* v, uint32_t* w) {
   const uint32_t a = __float_as_uint(v[0]) + 0x80u, b = __float_as_uint(v[1]) + 0x80u;
   const uint32_t c = __float_as_uint(v[2]) + 0x80u, d = __float_as_uint(v[3]) + 0x80u;
@@ -154,6 +142,50 @@ MLA_DEVICE void unpack_f24(const uint32_t* w, float* v) {
   v[3] = __uint_as_float(w[2] & 0xFFFFFF00u);
 }
 
+// 16x32bx2 TMEM accesses: a warp reaches 16 lanes (rows) of its sub-partition; threads
+// 0-15 take columns [c, c + N) of those lanes and threads 16-31 columns [c + split,
+// c + split + N), so the two threads i and i + 16 share row i.
+MLA_DEVICE void tm_ld_x32_s32(uint32_t taddr, float* v) {   // N 32, split 32
+  uint32_t* r = reinterpret_cast<uint32_t*>(v);
+  asm volatile(
+      "tcgen05.ld.sync.aligned.16x32bx2.x32.b32 "
+      "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
+      "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32], 32;"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+        "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]),
+        "=r"(r[13]), "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]),
+        "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]),
+        "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]),
+        "=r"(r[31])
+      : "r"(taddr)
+      : "memory");
+}
+MLA_DEVICE void tm_ld_x16_s16(uint32_t taddr, float* v) {   // N 16, split 16
+  uint32_t* r = reinterpret_cast<uint32_t*>(v);
+  asm volatile(
+      "tcgen05.ld.sync.aligned.16x32bx2.x16.b32 "
+      "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16], 16;"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+        "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]),
+        "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
+      : "r"(taddr)
+      : "memory");
+}
+MLA_DEVICE void tm_st_x16_s16(uint32_t taddr, const uint32_t* r) {   // N 16, split 16
+  asm volatile(
+      "tcgen05.st.sync.aligned.16x32bx2.x16.b32 [%0], 16, "
+      "{%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};" ::"r"(taddr),
+      "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]),
+      "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]),
+      "r"(r[15])
+      : "memory");
+}
+MLA_DEVICE void tm_st_x8_s8(uint32_t taddr, const uint32_t* r) {   // N 8, split 8
+  asm volatile(
+      "tcgen05.st.sync.aligned.16x32bx2.x8.b32 [%0], 8, {%1,%2,%3,%4,%5,%6,%7,%8};" ::"r"(taddr),
+      "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7])
+      : "memory");
+}
 
 }  // namespace
 
@@ -175,7 +207,6 @@ __global__ void __launch_bounds__(kThreads, 1)
   int* sched = misc + 2;
   int* warp_sum = misc + 8;
   static_assert(8 + kThreads / 32 <= kMiscInts, "misc ints overflow into the mbarriers");
-  float* red = reinterpret_cast<float*>(base + lay.red_off);
   uint64_t* bars = reinterpret_cast<uint64_t*>(base + lay.bar_off);
   const int nb = lay.nb;
   uint64_t* full = bars;                               // [slot][nb]
@@ -382,13 +413,14 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     __syncwarp();
   } else if (has_work) {
-    // =========== score exchange, softmax, P, epilogue (row n, quarter qt of a tile) ===========
+    // =========== score exchange, softmax, P, epilogue (row n, half qt of a tile) ================
     const int sp = warp & 3;                  // TMEM sub-partition this warp may access
-    const int wi = warp - 2;                  // softmax warp 0..15 (exchange block index)
-    const int qt = wi >> 2;                   // which 16 tokens of a tile / quarter of O
-    const int n = 32 * sp + lane;             // query row of this thread in the block
-    const int tid = threadIdx.x - 64;         // 0..511
-    const uint32_t trow = tmem + (uint32_t(32 * sp) << 16);
+    const int wi = warp - 2;                  // softmax warp 0..7 (exchange block index)
+    const int hl = wi >> 2;                   // which 16 lanes of the sub-partition
+    const int qt = lane >> 4;                 // which 32 tokens of a tile / half of O
+    const int n = 32 * sp + 16 * hl + (lane & 15);   // query row: lanes i and i + 16 share it
+    const int tid = threadIdx.x - 64;         // 0..255
+    const uint32_t trow = tmem + (uint32_t(32 * sp + 16 * hl) << 16);
     const uint32_t recv_s = smem_u32(recv);
     const uint32_t recv_r = map_to_rank(recv_s, peer);
     const uint32_t rfull_r0 = map_to_rank(smem_u32(&recv_full[0]), peer);
@@ -400,21 +432,18 @@ __global__ void __launch_bounds__(kThreads, 1)
     const bool row_ok = row < p.qH;
     const int qi = row / p.num_heads;
     const bool vec_out = (reinterpret_cast<uintptr_t>(p.o_latent) & 15u) == 0;
-    const int ocols = rhalf / kQuarters;      // O columns of this thread (16, 32 or 64)
-    const int ocol0 = qt * ocols;
-    float* qmax = red;                        // [tile parity][quarter][row]
-    float* qsum = red + 2 * kQuarters * kPairRows;   // [quarter][row]
-    const uint32_t grp_bar = 2 + sp;          // named barrier of the four warps of rows n
 
-    // Q half of this thread's row into TMEM (16-element chunks dealt round-robin to the
-    // four threads of the row): latent half, then rotary half; zero rows past q*H. Ends
+    // Q half of this thread's row into TMEM (16-element chunks dealt alternately to the
+    // two threads of the row): latent half, then rotary half; zero rows past q*H. Ends
     // with this warp's arrival on q_full.
     auto load_q = [&](int b) {
       const uint16_t* q = p.q_ext + (int64_t(b) * p.qH + row) * p.D;
-      for (int c0 = 16 * qt; c0 < rhalf + rh; c0 += 16 * kQuarters) {
-        const int src = c0 < rhalf ? int(rank) * rhalf + c0 : r + int(rank) * rh + (c0 - rhalf);
+      // 16-element chunks: chunk c0 / 16 + qt of the row per store (two per store)
+      for (int c0 = 0; c0 < rhalf + rh; c0 += 32) {
+        const int e = c0 + 16 * qt;           // past the end for an odd chunk count: zeros
+        const int src = e < rhalf ? int(rank) * rhalf + e : r + int(rank) * rh + (e - rhalf);
         uint32_t v[8];
-        if (row_ok) {
+        if (row_ok && e < rhalf + rh) {
           const uint4 a = *reinterpret_cast<const uint4*>(q + src);
           const uint4 bb = *reinterpret_cast<const uint4*>(q + src + 8);
           v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w;
@@ -423,7 +452,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
           for (int i = 0; i < 8; ++i) v[i] = 0u;
         }
-        tmem_st8(trow + kColQ + c0 / 2, v);
+        tm_st_x8_s8(trow + kColQ + c0 / 2, v);
       }
       tmem_wait_st();
       tc_fence_before();
@@ -458,7 +487,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         const bool got = __all_sync(0xffffffffu, mbar_wait(s_full, js & 1, wc));
         if (got) {
           tc_fence_after();
-          tmem_ld_part(trow + kColS + qt * kQTok, x);
+          tm_ld_x32_s32(trow + kColS, x);
           tmem_wait_ld();
         } else {
 #pragma unroll
@@ -499,12 +528,12 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int L = w.L;
       // last position row n sees (causal: L - q + i); rows past q*H see L - 1
       const int lim = min(L - 1, p.causal ? L - p.q_len + qi : L - 1);
-      float m = kRefInit, l = 0.0f;          // m identical in the four threads of a row
+      float m = kRefInit, l = 0.0f;          // m identical in the two threads of a row
       for (int t = tb; t < te; ++t, ++jj) {
         const int kb = jj & 1;                 // receive buffer of this tile
         const int slot = jj % p.nslot;
         const int tile_pos0 = (t - w.s) * kDecodeTok;
-        const int pos0 = tile_pos0 + qt * kQTok;   // first token of this thread's quarter
+        const int pos0 = tile_pos0 + qt * kQTok;   // first token of this thread's half
         // ---- send the next tile's partial before finishing this one ----
 #pragma unroll
         for (int i = 0; i < kPackWords; ++i) own_cur[i] = own_next[i];
@@ -536,7 +565,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         // The received words are in registers (consumed above): release the buffer to the
         // partner without a release fence, which would wait for this warp's remote stores.
         if (lane == 1) mbar_arrive_remote_relaxed(kb ? pfree_r1 : pfree_r0);
-        // re-arm this buffer for tile jj + 2 (the partner sends it only after all sixteen
+        // re-arm this buffer for tile jj + 2 (the partner sends it only after all eight
         // warps have released the buffer above)
         if (threadIdx.x == 65 && rcv) mbar_arrive_expect_tx_relaxed(&recv_full[kb], kXBytes);
 
@@ -554,13 +583,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int w2 = kQTok / 4; w2 >= 1; w2 >>= 1)
 #pragma unroll
           for (int c = 0; c < w2; ++c) mt[c] = fmaxf(mt[c], mt[c + w2]);
-        // the row's maximum over the four quarters (same value in all four threads)
-        qmax[(kb * kQuarters + qt) * kPairRows + n] = mt[0] * c_log2;
-        named_bar_sync(grp_bar, 32 * kQuarters);
-        const float* qm = qmax + kb * kQuarters * kPairRows + n;
-        float mx = qm[0];
-#pragma unroll
-        for (int q = 1; q < kQuarters; ++q) mx = fmaxf(mx, qm[q * kPairRows]);
+        // the row's maximum over both halves (lanes i and i + 16: the same value in both)
+        const float mh = mt[0] * c_log2;
+        const float mx = fmaxf(mh, __shfl_xor_sync(0xffffffffu, mh, 16));
         if (threadIdx.x == 64) MLA_PTRACE(11, jj);
         float alpha = 1.0f;
         if (mx > m + kLazyThreshold) {
@@ -574,13 +599,13 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (threadIdx.x == 64) MLA_PTRACE(6, jj);
         tc_fence_after();
         if (t > tb && pv_ok && __any_sync(0xffffffffu, alpha != 1.0f)) {
-          for (int c0 = 0; c0 < ocols; c0 += 16) {
+          for (int c0 = 0; c0 < rhalf; c0 += 32) {
             float o[16];
-            tmem_ld16(trow + kColO + ocol0 + c0, o);
+            tm_ld_x16_s16(trow + kColO + c0, o);
             tmem_wait_ld();
 #pragma unroll
             for (int c = 0; c < 16; ++c) o[c] *= alpha;
-            tmem_st16(trow + kColO + ocol0 + c0, o);
+            tm_st_x16_s16(trow + kColO + c0, reinterpret_cast<const uint32_t*>(o));
           }
         }
         // weights 2^(s * scale - m); the tile's sum in two chains, added to l in a fixed
@@ -596,7 +621,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           pk[c] = cvt_bf16x2(p0, p1);
         }
         l += sa + sb;
-        tmem_st_part(trow + kColP + qt * (kQTok / 2), pk);
+        tm_st_x16_s16(trow + kColP, pk);
         // cache rows past the context may hold anything (even NaN): zero their latent half
         // so that 0-weight x garbage cannot reach O
         if (tile_pos0 + kDecodeTok > L) {
@@ -623,13 +648,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       const bool fin = __all_sync(0xffffffffu, mbar_wait(pv_done, (jj - 1) & 1, wc));
       tc_fence_after();
       const bool aborted = __any_sync(0xffffffffu, !fin || *abort_flag != 0);
-      qsum[qt * kPairRows + n] = l;
-      named_bar_sync(grp_bar, 32 * kQuarters);
-      // the row sum, added in the same order by every thread of the row
-      float lt = qsum[n];
-#pragma unroll
-      for (int q = 1; q < kQuarters; ++q) lt += qsum[q * kPairRows + n];
-      named_bar_sync(grp_bar, 32 * kQuarters);               // qsum may be reused
+      // the row sum over both halves (the same value in both threads: a + b = b + a)
+      const float lt = l + __shfl_xor_sync(0xffffffffu, l, 16);
       const bool whole = (tb == w.s) && (te == w.s + w.tiles);
       const int64_t grow = int64_t(w.b) * p.qH + row;   // global (b, i, h) row
       const int pslot = piece_slot(vc, w.s, per, p.col_groups, cg);
@@ -639,11 +659,11 @@ __global__ void __launch_bounds__(kThreads, 1)
         else p.part_lse[int64_t(pslot) * kPairRows + n] = lse;
       }
       const float inv = (lt > 0.0f && !aborted) ? 1.0f / lt : 0.0f;
-      const int64_t lat0 = int64_t(rank) * rhalf + ocol0;
-      for (int c0 = 0; c0 < ocols; c0 += 16) {
+      const int64_t lat0 = int64_t(rank) * rhalf + 16 * qt;   // this thread's 16 of every 32
+      for (int c0 = 0; c0 < rhalf; c0 += 32) {
         float o[16];
         if (!aborted) {
-          tmem_ld16(trow + kColO + ocol0 + c0, o);
+          tm_ld_x16_s16(trow + kColO + c0, o);
           tmem_wait_ld();
         } else {
 #pragma unroll
