@@ -103,7 +103,7 @@ mla_status plan_decode(const mla_dims* d, int32_t batch, int32_t q_len, int32_t 
   P->npt = 1;
   if (P->pair) {
     P->tmem_cols = 512;
-    for (int ns = kDecodeMaxSlots; ns >= 2 && P->nslot == 0; --ns)
+    for (int ns = kPairMaxSlots; ns >= 2 && P->nslot == 0; --ns)
       if (decode_pair_smem_bytes(r, P->rope_half, ns) <= size_t(kMaxSmem)) P->nslot = ns;
     if (P->nslot < 2) return MLA_ERR_UNSUPPORTED;
     P->smem = decode_pair_smem_bytes(r, P->rope_half, P->nslot);

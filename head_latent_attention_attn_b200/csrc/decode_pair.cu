@@ -1,5 +1,5 @@
 // decode_pair.cu - mla_decode_attn on sm_100a for blocks of 65..128 query rows: a cluster
-// of two CTAs splits the latent dimension.
+// of two CTAs splits the latent dimension and shares the softmax by rows.
 //
 // Formulation, for one block of up to 128 query rows n = (i, h) of a sequence:
 //   S[n, tok]  = Q[n, :] . C[tok, :]        UMMA M=128 rows, N=64 tokens, K = row width
@@ -7,32 +7,36 @@
 // O for 128 rows and the whole latent of rank 512 would fill all 512 TMEM columns of an
 // SM, so the two CTAs of a cluster split the latent. CTA k loads, for every page, only the
 // latent columns [k r/2, (k+1) r/2) and half of the rotary columns, keeps the same half of
-// the Q rows in TMEM, and computes the partial scores over its half of the row width. The
-// partials are swapped through distributed shared memory; both CTAs add the same two
-// partials, run the same online softmax on the same numbers and so hold the same weights
-// P, which each applies to its latent half. Each page crosses HBM once per cluster; Q and
-// P are UMMA A operands read from TMEM, so shared-memory bandwidth goes to the cache half.
+// every Q row, and computes the partial scores S_k over its half of the row width. Each
+// page crosses HBM once per cluster.
 //
-// The exchange. The SM-to-SM network moves about 13 bytes per clock per SM each way, so
-// the partial of a tile (128 rows x 64 tokens) travels as 24-bit floats: fp32 rounded to
-// a 15-bit mantissa (relative error <= 2^-16, far below the bf16 rounding of P), 4 values
-// in 3 words, 24 KB per tile. Each CTA rounds its own partial the same way before adding,
-// so both sides add identical numbers. Every thread sends its packed words straight from
-// registers (st.async, completing on the partner's mbarrier) and keeps them for its own
-// sum, so no shared memory is spent on staging and four cache slots fit. The softmax
-// warps send tile j+1 before they finish tile j, so one tile of exchange latency overlaps
-// the softmax and PV work of the previous tile.
+// The softmax is split by rows. CTA k owns rows [64k, 64k + 64): it receives the partner's
+// partial scores for those rows only, adds them to its own, runs the online softmax and
+// writes P for its rows into its TMEM; it also sends those weights (bf16), with the row's
+// rescale factor and running sum, to the partner, whose O half needs P for all 128 rows.
+// Per tile and direction that is 12 KB of partial scores (24-bit floats: fp32 rounded to
+// a 15-bit mantissa, relative error <= 2^-16, 4 values in 3 words) and 8.5 KB of weights,
+// and each CTA evaluates 64 x 64 exponentials instead of 128 x 64.
 //
-// Roles (352 threads per CTA): warp 0 TMA producer, warp 1 S issuer and TMEM owner, warps
-// 2-9 the score exchange, softmax, P into TMEM and the epilogue, warp 10 the PV issuer.
-// The M=128 accumulator puts row n on TMEM lane n, and a warp reaches only the 32 lanes of
-// its sub-partition (warp % 4); with 16x32bx2 TMEM accesses a warp covers 16 rows with two
-// threads each (lanes i and i + 16: tokens 0-31 and 32-63 of every tile), so the row's
-// maximum and sum need one shuffle, and the two warps of a sub-partition take its lanes
-// 0-15 and 16-31.
+// TMEM (512 columns): O [0, r/2), two S buffers [256, 320) and [320, 384), the latent half
+// of Q [384, 384 + r/4) (bf16 pairs). The rotary half of Q is a shared-memory operand (the
+// S UMMA takes A from TMEM for the latent K steps and from shared memory for the rotary
+// ones), which frees the columns for the second S buffer. P of a tile (bf16 pairs) is
+// written over the first 32 columns of that tile's S buffer once its scores have been
+// read, so S of tile j + 2 waits for PV of tile j, while S of tile j + 1 is computed as soon
+// as its page has landed: the score exchange of one tile overlaps the softmax of the other.
 //
-// TMEM columns: O [0, r/2), S [256, 320), P [320, 352) (bf16 pairs), Q [352, 352 +
-// (r/2 + rope_half)/2) (bf16 pairs: latent half, then rotary half).
+// Roles (352 threads): warp 0 TMA producer, warp 1 S issuer and TMEM owner, warp 2 PV
+// issuer, warps 3-10 the rows. TMEM lane n holds row n and a warp reaches only the 32 lanes
+// of its sub-partition (warp % 4), so the rows of CTA k are the lanes of sub-partitions 2k
+// and 2k + 1:
+//   owners    (4 warps on the own sub-partitions; 16x32bx2 accesses, 16 rows per warp,
+//              lanes i and i + 16 take tokens 0-31 and 32-63 of row i): combine the two
+//              partials, softmax, P, the epilogue of the own rows;
+//   senders   (one warp per partner sub-partition, one row per lane): read the partner
+//              rows' partial scores and send them;
+//   receivers (one warp per partner sub-partition): take the partner's P and rescale
+//              factors for its rows into TMEM, the epilogue of those rows.
 #include <math.h>
 
 #include "decode_sched.cuh"
@@ -43,10 +47,10 @@ namespace mla {
 
 // Optional per-tile timeline of CTA 0 (compile with -DMLA_TRACE; read with
 // mla_pair_trace_read). Events: 0 producer issued the tile's loads, 1 every block of the
-// tile landed (the S issuer waits for that before the S buffer), 2 S committed, 3 softmax
-// read S, 4 partial sent, 5 partner's partial received, 6 PV(j-1) seen done, 7 P written,
-// 8 PV issued, 9 S issuer saw S free, 10 scores unpacked, 11 scores scaled. After the 12
-// event rows: every CTA's start and end (%globaltimer) as pairs.
+// tile landed, 2 S committed, 3 sender read S, 4 sender's partial sent, 5 owner has the
+// partner's partial, 6 owner's P written and sent, 7 receiver has the partner's P, 8 PV
+// issued, 9 S issuer saw the S buffer free, 10 owner read S, 11 receiver's P written.
+// After the 12 event rows: every CTA's start and end (%globaltimer) as pairs.
 #ifdef MLA_TRACE
 constexpr int kPairTraceTiles = 512;
 constexpr int kPairTraceEvents = 12;
@@ -64,26 +68,25 @@ __device__ unsigned long long g_mla_pair_trace[kPairTraceEvents * kPairTraceTile
 
 namespace {
 
-constexpr int kRowThreads = 2;                                   // softmax threads per row
-constexpr int kSoftWarps = 8;                                  // 16 rows per warp
-constexpr int kSoftThreads = 32 * kSoftWarps;
-constexpr int kPvWarp = 2 + kSoftWarps;
-constexpr int kThreads = 32 * (kPvWarp + 1);
-constexpr int kQTok = kDecodeTok / kRowThreads;                  // tokens per softmax thread
+constexpr int kPvWarp = 2;
+constexpr int kRowWarp0 = 3;                                   // first of the 8 row warps
+constexpr int kThreads = 32 * (kRowWarp0 + 8);
+constexpr int kHalfTok = kDecodeTok / 2;                       // tokens per owner thread
 constexpr uint32_t kBlk = kDecodeTok * 128;                    // 64 x 64 bf16 block, 8 KB
-constexpr int kPackWords = kQTok * 3 / 4;                      // 24-bit values of one part
-constexpr uint32_t kXWarpBytes = 32u * kPackWords * 4;          // one warp's parts
-constexpr uint32_t kXBytes = kSoftWarps * kXWarpBytes;          // one tile's partial, 24 KB
-constexpr uint32_t kColO = 0, kColS = 256, kColP = 320, kColQ = 352, kTmemCols = 512;
+constexpr int kPackWords = kHalfTok * 3 / 4;                   // 24-bit values of a half row
+constexpr uint32_t kXsWarpBytes = 32u * kPackWords * 4;        // one owner warp's rows
+constexpr uint32_t kXsBytes = 4 * kXsWarpBytes;                // partials of 64 rows, 12 KB
+constexpr uint32_t kXpRowsBytes = 64u * kDecodeTok * 2;        // P of 64 rows (bf16), 8 KB
+constexpr uint32_t kXpBytes = kXpRowsBytes + 64u * 8;          // + (alpha, sum) per row
+constexpr uint32_t kColO = 0, kColS = 256, kColQ = 384, kTmemCols = 512;
 constexpr float kLazyThreshold = 8.0f;   // log2 units; see decode.cu
-constexpr int kPrefetchAhead = 4;        // tiles brought into L2 ahead of their TMA load
 constexpr float kRefInit = -3.0e38f;
 constexpr float kLn2 = 0.69314718055994530942f;
 // misc ints: 0 TMEM base, 1 abort flag, [2,8) schedule, [8, 8 + warps) warp sums
 constexpr int kMiscInts = 32;
 
 struct PairLayout {
-  uint32_t slot_bytes, rope_off, recv_off, misc_off, bar_off, total;
+  uint32_t slot_bytes, rope_off, qrope_off, xs_off, xp_off, misc_off, bar_off, total;
   int nb;   // TMA barriers per slot: one per latent block and one for the rotary block
 };
 
@@ -91,7 +94,7 @@ __host__ __device__ inline uint32_t round_up_p(uint32_t x, uint32_t a) {
   return (x + a - 1) / a * a;
 }
 
-__host__ __device__ constexpr int pair_bars(int nslot, int nb) { return nslot * nb + nslot + 10; }
+__host__ __device__ constexpr int pair_bars(int nslot, int nb) { return nslot * nb + nslot + 16; }
 
 __host__ __device__ inline PairLayout pair_layout(int r, int rope_half, int nslot) {
   PairLayout L;
@@ -100,8 +103,12 @@ __host__ __device__ inline PairLayout pair_layout(int r, int rope_half, int nslo
   L.rope_off = uint32_t(lb) * kBlk;
   L.slot_bytes = round_up_p(L.rope_off + uint32_t(kDecodeTok) * rope_half * 2, 1024);
   uint32_t off = uint32_t(nslot) * L.slot_bytes;
-  L.recv_off = off;                               // partner's packed partials (two tiles)
-  off += 2 * kXBytes;
+  L.qrope_off = off;                              // rotary half of the 128 Q rows (swizzled)
+  off += round_up_p(uint32_t(kPairRows) * rope_half * 2, 1024);
+  L.xs_off = off;                                 // partner's partials for the own rows (x2)
+  off += 2 * kXsBytes;
+  L.xp_off = off;                                 // partner's P for its rows
+  off += kXpBytes;
   L.misc_off = off;
   off += 4 * kMiscInts;
   L.bar_off = round_up_p(off, 8);
@@ -118,11 +125,38 @@ MLA_DEVICE SmemSwizzle rope_swizzle(int rope_half) {
   return rope_half == 64 ? kSw128 : (rope_half == 32 ? kSw64 : kSw32);
 }
 
-// Byte offset of 16-byte chunk c (packed words 4c..4c+3) of lane `lane` of softmax warp
-// wi in a receive buffer: each warp's 32 (row, token half) threads are one contiguous
-// block, chunk-major inside it, so a quarter-warp touches 128 consecutive bytes.
-MLA_DEVICE uint32_t x_offset(int wi, int lane, int c) {
-  return uint32_t(wi) * kXWarpBytes + uint32_t(c) * 512u + uint32_t(lane) * 16u;
+// Byte offset, in a partial-score buffer, of 16-byte chunk c (packed words 4c..4c+3) for
+// lane `lane` of owner warp ow: each owner warp's 32 (row, token half) threads are one
+// contiguous block, chunk-major inside it, so a quarter-warp touches 128 consecutive bytes.
+MLA_DEVICE uint32_t xs_offset(int ow, int lane, int c) {
+  return uint32_t(ow) * kXsWarpBytes + uint32_t(c) * 512u + uint32_t(lane) * 16u;
+}
+
+// Byte offset of 16-byte chunk c (tokens 8c..8c+7, bf16) of own-block row m (0..63) in a
+// weight buffer: chunk-major, so the 32 rows a receiver warp reads are consecutive; the
+// rows' (alpha, running sum) pairs follow the weights.
+MLA_DEVICE uint32_t xp_offset(int m, int c) { return uint32_t(c) * 1024u + uint32_t(m) * 16u; }
+MLA_DEVICE uint32_t xp_scalars(int m) { return kXpRowsBytes + uint32_t(m) * 8u; }
+
+// Byte offset of 16-byte chunk c of row `row` in a K-major tile with rows of `pitch` bytes
+// (32, 64 or 128) stored with the matching 32/64/128-byte swizzle: the chunk index is
+// XORed with bits 7.. of the linear offset (the layout TMA writes and UMMA reads).
+MLA_DEVICE uint32_t swizzled_chunk(int row, int c, int pitch) {
+  const uint32_t lin = uint32_t(row) * uint32_t(pitch) + uint32_t(c) * 16u;
+  const uint32_t mask = uint32_t(pitch / 16 - 1);
+  return lin ^ (((lin >> 7) & mask) << 4);
+}
+
+MLA_DEVICE void st_async_v2(uint32_t remote_addr, uint2 v, uint32_t remote_bar) {
+  asm volatile(
+      "st.async.shared::cluster.mbarrier::complete_tx::bytes.v2.b32 [%0], {%1, %2}, [%3];"
+      ::"r"(remote_addr), "r"(v.x), "r"(v.y), "r"(remote_bar)
+      : "memory");
+}
+MLA_DEVICE uint2 ld_shared_v2(uint32_t saddr) {
+  uint2 v;
+  asm volatile("ld.shared.v2.b32 {%0, %1}, [%2];" : "=r"(v.x), "=r"(v.y) : "r"(saddr) : "memory");
+  return v;
 }
 
 // Four 24-bit values (fp32 rounded to sign, exponent and a 15-bit mantissa) in three words
@@ -200,7 +234,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int r = p.r, rh = p.rope_half, lb = r / 128, rhalf = r / 2;
   const PairLayout lay = pair_layout(r, rh, p.nslot);
   uint8_t* slots = base;
-  uint8_t* recv = base + lay.recv_off;
+  uint8_t* qrope = base + lay.qrope_off;
+  uint8_t* xs = base + lay.xs_off;
+  uint8_t* xp = base + lay.xp_off;
   int* misc = reinterpret_cast<int*>(base + lay.misc_off);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(misc);
   volatile int* abort_flag = misc + 1;
@@ -211,13 +247,15 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int nb = lay.nb;
   uint64_t* full = bars;                               // [slot][nb]
   uint64_t* empty = full + p.nslot * nb;               // [slot]
-  uint64_t* q_full = empty + p.nslot;
-  uint64_t* s_full = q_full + 1;
-  uint64_t* s_free = s_full + 1;
-  uint64_t* pv_done = s_free + 1;
-  uint64_t* recv_full = pv_done + 1;                   // [2] partner's partial landed
-  uint64_t* peer_free = recv_full + 2;                 // [2] partner consumed our partial
-  uint64_t* p_full = peer_free + 2;                    // P of the tile written
+  uint64_t* q_full = empty + p.nslot;                  // Q of the piece in TMEM and smem
+  uint64_t* s_full = q_full + 1;                       // [2] S buffer computed
+  uint64_t* s_free = s_full + 2;                       // [2] S buffer read by all readers
+  uint64_t* pv_done = s_free + 2;                      // [2] PV of the buffer's tile done
+  uint64_t* p_full = pv_done + 2;                      // [2] P of all 128 rows written
+  uint64_t* xs_full = p_full + 2;                      // [2] partner's partials landed
+  uint64_t* xs_free = xs_full + 2;                     // [2] partner consumed ours
+  uint64_t* xp_full = xs_free + 2;                     // partner's P landed
+  uint64_t* xp_free = xp_full + 1;                     // partner consumed our P
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -235,20 +273,23 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int k = 0; k < nb; ++k) mbar_init(&full[s * nb + k], 1);
       mbar_init(&empty[s], 1);
     }
-    mbar_init(q_full, kSoftWarps);
-    mbar_init(s_full, 1);
-    mbar_init(s_free, kSoftWarps);
-    mbar_init(pv_done, 1);
+    mbar_init(q_full, 6);                              // 4 owner + 2 sender warps
     for (int i = 0; i < 2; ++i) {
-      mbar_init(&recv_full[i], 1);
-      mbar_init(&peer_free[i], kSoftWarps);
+      mbar_init(&s_full[i], 1);
+      mbar_init(&s_free[i], 6);                        // 4 owner + 2 sender warps
+      mbar_init(&pv_done[i], 1);
+      mbar_init(&p_full[i], 6);                        // 4 owner + 2 receiver warps
+      mbar_init(&xs_full[i], 1);
+      mbar_init(&xs_free[i], 4);                       // the partner's 4 owner warps
     }
-    mbar_init(p_full, kSoftWarps);
+    mbar_init(xp_full, 1);
+    mbar_init(xp_free, 2);                             // the partner's 2 receiver warps
     *abort_flag = 0;
     fence_mbar_init();
-    // both receive buffers expect their first partial
-    mbar_arrive_expect_tx(&recv_full[0], kXBytes);
-    mbar_arrive_expect_tx(&recv_full[1], kXBytes);
+    // the receive buffers expect their first messages
+    mbar_arrive_expect_tx(&xs_full[0], kXsBytes);
+    mbar_arrive_expect_tx(&xs_full[1], kXsBytes);
+    mbar_arrive_expect_tx(xp_full, kXpBytes);
   }
   if (warp == 1) {
     tmem_alloc(tmem_slot, kTmemCols);
@@ -276,30 +317,6 @@ __global__ void __launch_bounds__(kThreads, 1)
       prefetch_tensormap(&p.tm_rope);
       if (blockIdx.x == 0) *p.range_len = per;
       UnitWalk w{sched[0], sched[1]};
-      // L2 prefetch walk, kPrefetchAhead tiles ahead of the loads: the few shared-memory
-      // slots leave too little lead time to hide DRAM latency behind the loads alone.
-      UnitWalk pf{sched[0], sched[1]};
-      pf.load(p, cg);
-      int pf_t = max(pf.s, r0), pf_n = 0;
-      auto prefetch_upto = [&](int upto) {
-        while (pf_n < upto && pf.s < r1) {
-          if (pf_t >= min(pf.s + pf.tiles, r1)) {
-            pf.s += pf.tiles;
-            ++pf.b;
-            if (pf.s >= r1) break;
-            pf.load(p, cg);
-            pf_t = pf.s;
-          }
-          const int32_t page = p.block_table[int64_t(pf.b) * p.max_pages + (pf_t - pf.s)];
-          if (page >= 0 && page < p.num_pages) {
-            for (int k = 0; k < lb; ++k)
-              tma_prefetch_l2_2d(&p.tm_cache, int(rank) * rhalf + k * 64, page * kDecodeTok);
-            tma_prefetch_l2_2d(&p.tm_rope, r + int(rank) * rh, page * kDecodeTok);
-          }
-          ++pf_t;
-          ++pf_n;
-        }
-      };
       int jj = 0;
       bool ok = true;
       for (; ok && w.s < r1; w.s += w.tiles, ++w.b) {
@@ -329,8 +346,6 @@ __global__ void __launch_bounds__(kThreads, 1)
           mbar_arrive_expect_tx(fb, rope_bytes);
           tma_load_2d(sbase + lay.rope_off, &p.tm_rope, r + int(rank) * rh, page * kDecodeTok,
                       fb);
-          // after the load: a prefetch queued ahead of it would delay it
-          prefetch_upto(jj + 1 + kPrefetchAhead);
           MLA_PTRACE(0, jj);
         }
       }
@@ -342,11 +357,14 @@ __global__ void __launch_bounds__(kThreads, 1)
     __syncwarp();
   } else if (warp == 1) {
     // ============================ UMMA issuer for the partial S ==========================
+    // S of tile j goes to buffer j % 2: it waits for its page, for the readers of tile j - 2
+    // and for PV of tile j - 2 (whose P was written over that buffer).
     if (has_work && elect_one()) {
       const uint32_t idesc_s = make_idesc_bf16(128, kDecodeTok, 0, 0);
       const uint64_t b0 = make_sdesc(smem_u32(slots), 16, 1024, kSw128);
       const uint64_t br0 =
           make_sdesc(smem_u32(slots + lay.rope_off), 16, 8 * rh * 2, rope_swizzle(rh));
+      const uint64_t aq0 = make_sdesc(smem_u32(qrope), 16, 8 * rh * 2, rope_swizzle(rh));
       UnitWalk w{sched[0], sched[1]};
       int jj = 0, pc = 0;
       bool ok = true;
@@ -357,26 +375,31 @@ __global__ void __launch_bounds__(kThreads, 1)
         tc_fence_after();
         for (int t = tb; ok && t < te; ++t, ++jj) {
           const int slot = jj % p.nslot;
-          // every block of the tile landed, then the S accumulator free
+          const int sb = jj & 1;
+          // every block of the tile landed, then the S buffer free
           for (int k = 0; ok && k <= lb; ++k)
             ok = mbar_wait(&full[slot * nb + k], (jj / p.nslot) & 1, wc);
           if (!ok) break;
           MLA_PTRACE(1, jj);
-          if (jj >= 1 && !mbar_wait(s_free, (jj - 1) & 1, wc)) { ok = false; break; }
+          if (jj >= 2 && (!mbar_wait(&s_free[sb], ((jj - 2) >> 1) & 1, wc) ||
+                          !mbar_wait(&pv_done[sb], ((jj - 2) >> 1) & 1, wc))) {
+            ok = false;
+            break;
+          }
           MLA_PTRACE(9, jj);
           tc_fence_after();
+          const uint32_t dS = tmem + kColS + 64 * sb;
           const uint32_t soff = slot * lay.slot_bytes;
           for (int k = 0; k < lb; ++k) {
 #pragma unroll
             for (int kk = 0; kk < 4; ++kk)
-              umma_bf16_ts(tmem + kColS, tmem + kColQ + (k * 4 + kk) * 8,
+              umma_bf16_ts(dS, tmem + kColQ + (k * 4 + kk) * 8,
                            b0 + ((soff + k * kBlk + kk * 32) >> 4), idesc_s,
                            (k | kk) != 0 ? 1u : 0u);
           }
           for (int kk = 0; kk < rh / 16; ++kk)
-            umma_bf16_ts(tmem + kColS, tmem + kColQ + (lb * 4 + kk) * 8,
-                         br0 + ((soff + kk * 32) >> 4), idesc_s, 1u);
-          umma_commit(s_full);
+            umma_bf16(dS, aq0 + ((kk * 32) >> 4), br0 + ((soff + kk * 32) >> 4), idesc_s, 1u);
+          umma_commit(&s_full[sb]);
           MLA_PTRACE(2, jj);
         }
       }
@@ -395,7 +418,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         w.load(p, cg);
         const int tb = max(w.s, r0), te = min(w.s + w.tiles, r1);
         for (int t = tb; t < te; ++t, ++jj) {
-          if (!mbar_wait(p_full, jj & 1, wc)) { ok = false; break; }
+          const int sb = jj & 1;
+          if (!mbar_wait(&p_full[sb], (jj >> 1) & 1, wc)) { ok = false; break; }
           tc_fence_after();
           // the first tile of a piece overwrites O: the previous piece's epilogue read O
           // before its warps arrived on p_full for this tile
@@ -403,9 +427,10 @@ __global__ void __launch_bounds__(kThreads, 1)
           const uint32_t soff = (jj % p.nslot) * lay.slot_bytes;
 #pragma unroll
           for (int kk = 0; kk < 4; ++kk)
-            umma_bf16_ts(tmem + kColO, tmem + kColP + kk * 8, pb0 + ((soff + kk * 2048) >> 4),
-                         idesc_o, (!first || kk > 0) ? 1u : 0u);
-          umma_commit(pv_done);
+            umma_bf16_ts(tmem + kColO, tmem + kColS + 64 * sb + kk * 8,
+                         pb0 + ((soff + kk * 2048) >> 4), idesc_o,
+                         (!first || kk > 0) ? 1u : 0u);
+          umma_commit(&pv_done[sb]);
           umma_commit(&empty[jj % p.nslot]);
           MLA_PTRACE(8, jj);
         }
@@ -413,291 +438,466 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     __syncwarp();
   } else if (has_work) {
-    // =========== score exchange, softmax, P, epilogue (row n, half qt of a tile) ================
-    const int sp = warp & 3;                  // TMEM sub-partition this warp may access
-    const int wi = warp - 2;                  // softmax warp 0..7 (exchange block index)
-    const int hl = wi >> 2;                   // which 16 lanes of the sub-partition
-    const int qt = lane >> 4;                 // which 32 tokens of a tile / half of O
-    const int n = 32 * sp + 16 * hl + (lane & 15);   // query row: lanes i and i + 16 share it
-    const int tid = threadIdx.x - 64;         // 0..255
-    const uint32_t trow = tmem + (uint32_t(32 * sp + 16 * hl) << 16);
-    const uint32_t recv_s = smem_u32(recv);
-    const uint32_t recv_r = map_to_rank(recv_s, peer);
-    const uint32_t rfull_r0 = map_to_rank(smem_u32(&recv_full[0]), peer);
-    const uint32_t rfull_r1 = map_to_rank(smem_u32(&recv_full[1]), peer);
-    const uint32_t pfree_r0 = map_to_rank(smem_u32(&peer_free[0]), peer);
-    const uint32_t pfree_r1 = map_to_rank(smem_u32(&peer_free[1]), peer);
+    // ==================================== the 128 rows ====================================
+    const int wi = warp - kRowWarp0;          // 0..7
+    const int sp = warp & 3;                  // TMEM sub-partition this warp reaches
+    const int hl = wi >> 2;                   // each sub-partition has two row warps
+    const bool owner = (sp >> 1) == int(rank);
     const float c_log2 = p.scale_log2;
-    const int row = cg * kPairRows + n;       // row (i, h) of the sequence's q*H rows
-    const bool row_ok = row < p.qH;
-    const int qi = row / p.num_heads;
     const bool vec_out = (reinterpret_cast<uintptr_t>(p.o_latent) & 15u) == 0;
+    const int rpitch = rh * 2;                // bytes per Q rotary row in shared memory
+    const uint32_t xs_s = smem_u32(xs), xp_s = smem_u32(xp);
+    const uint32_t xs_r = map_to_rank(xs_s, peer), xp_r = map_to_rank(xp_s, peer);
+    const uint32_t xs_full_r0 = map_to_rank(smem_u32(&xs_full[0]), peer);
+    const uint32_t xs_full_r1 = map_to_rank(smem_u32(&xs_full[1]), peer);
+    const uint32_t xs_free_r0 = map_to_rank(smem_u32(&xs_free[0]), peer);
+    const uint32_t xs_free_r1 = map_to_rank(smem_u32(&xs_free[1]), peer);
+    const uint32_t xp_full_r = map_to_rank(smem_u32(xp_full), peer);
+    const uint32_t xp_free_r = map_to_rank(smem_u32(xp_free), peer);
 
-    // Q half of this thread's row into TMEM (16-element chunks dealt alternately to the
-    // two threads of the row): latent half, then rotary half; zero rows past q*H. Ends
-    // with this warp's arrival on q_full.
-    auto load_q = [&](int b) {
-      const uint16_t* q = p.q_ext + (int64_t(b) * p.qH + row) * p.D;
-      // 16-element chunks: chunk c0 / 16 + qt of the row per store (two per store)
-      for (int c0 = 0; c0 < rhalf + rh; c0 += 32) {
-        const int e = c0 + 16 * qt;           // past the end for an odd chunk count: zeros
-        const int src = e < rhalf ? int(rank) * rhalf + e : r + int(rank) * rh + (e - rhalf);
-        uint32_t v[8];
-        if (row_ok && e < rhalf + rh) {
-          const uint4 a = *reinterpret_cast<const uint4*>(q + src);
-          const uint4 bb = *reinterpret_cast<const uint4*>(q + src + 8);
-          v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w;
-          v[4] = bb.x; v[5] = bb.y; v[6] = bb.z; v[7] = bb.w;
-        } else {
-#pragma unroll
-          for (int i = 0; i < 8; ++i) v[i] = 0u;
-        }
-        tm_st_x8_s8(trow + kColQ + c0 / 2, v);
-      }
-      tmem_wait_st();
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(q_full);
-    };
+    if (owner) {
+      // ---------------- owner: rows of this CTA, 16 per warp, two threads per row --------
+      const int ow = 2 * hl + (sp & 1);       // owner warp index (block of the partial buffer)
+      const int qt = lane >> 4;               // token half of this thread
+      const int n = 32 * sp + 16 * hl + (lane & 15);   // query row (TMEM lane)
+      const int m = n & 63;                   // row within the own block
+      const uint32_t trow = tmem + (uint32_t(32 * sp + 16 * hl) << 16);
+      const int row = cg * kPairRows + n;     // row (i, h) of the sequence's q*H rows
+      const bool row_ok = row < p.qH;
+      const int qi = row / p.num_heads;
+      const bool tr = (ow == 0 && lane == 0);
+      (void)tr;
 
-    // ---- send side: the partial of the next tile of this CTA's range ----------------
-    // `sw` walks the units one tile ahead of the softmax; it loads the Q of every new
-    // piece as soon as the previous piece's last S has been read out of TMEM.
-    UnitWalk sw{sched[0], sched[1]};
-    sw.load(p, cg);
-    int st_t = max(sw.s, r0);                // next tile to send (row-block tile index)
-    int js = 0;                              // tiles sent so far
-    // this thread's packed partial of the tile last sent (own_next) and of the tile whose
-    // scores are formed now (own_cur): the own contribution never leaves the registers
-    uint32_t own_next[kPackWords], own_cur[kPackWords];
-    load_q(sw.b);
-    auto send_next = [&]() -> bool {
-      if (st_t >= min(sw.s + sw.tiles, r1)) {
-        sw.s += sw.tiles;
-        ++sw.b;
-        if (sw.s >= r1) return false;
-        sw.load(p, cg);
-        st_t = sw.s;
-        load_q(sw.b);
-      }
-      const int kb = js & 1;
-      uint32_t* pw = own_next;                 // kept for this tile's own contribution
-      {
-        float x[kQTok];
-        const bool got = __all_sync(0xffffffffu, mbar_wait(s_full, js & 1, wc));
-        if (got) {
-          tc_fence_after();
-          tm_ld_x32_s32(trow + kColS, x);
-          tmem_wait_ld();
-        } else {
+      // This CTA's half of Q row n: latent half into TMEM (16-element chunks dealt
+      // alternately to the two threads of the row), rotary half into shared memory; zero
+      // rows past q*H. Ends with this warp's arrival on q_full.
+      auto load_q = [&](int b) {
+        const uint16_t* q = p.q_ext + (int64_t(b) * p.qH + row) * p.D;
+        for (int c0 = 0; c0 < rhalf; c0 += 32) {
+          const uint16_t* src = q + int(rank) * rhalf + c0 + 16 * qt;
+          uint32_t v[8];
+          if (row_ok) {
+            const uint4 a = *reinterpret_cast<const uint4*>(src);
+            const uint4 bb = *reinterpret_cast<const uint4*>(src + 8);
+            v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w;
+            v[4] = bb.x; v[5] = bb.y; v[6] = bb.z; v[7] = bb.w;
+          } else {
 #pragma unroll
-          for (int c = 0; c < kQTok; ++c) x[c] = 0.0f;
-        }
-        if (threadIdx.x == 64) MLA_PTRACE(3, js);
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(s_free);    // the S accumulator may be overwritten
-#pragma unroll
-        for (int g = 0; g < kQTok / 4; ++g) pack_f24(x + 4 * g, pw + 3 * g);
-      }
-      // Into the partner's receive buffer once the partner has consumed tile js - 2 from
-      // it: stores from registers over the SM-to-SM network, each completing its bytes on
-      // the partner's mbarrier.
-      const bool free_ok = __all_sync(
-          0xffffffffu, js < 2 || mbar_wait_cluster(&peer_free[kb], ((js - 2) >> 1) & 1, wc));
-      if (free_ok) {
-        const uint32_t dst = recv_r + kb * kXBytes;
-        const uint32_t rb = kb ? rfull_r1 : rfull_r0;
-#pragma unroll
-        for (int c = 0; c < kPackWords / 4; ++c)
-          st_async_v4(dst + x_offset(wi, lane, c),
-                      make_uint4(pw[4 * c], pw[4 * c + 1], pw[4 * c + 2], pw[4 * c + 3]), rb);
-      }
-      if (threadIdx.x == 64) MLA_PTRACE(4, js);
-      ++js;
-      ++st_t;
-      return true;
-    };
-
-    bool sending = send_next();              // tile 0 (the range is not empty)
-    UnitWalk w{sched[0], sched[1]};
-    w.load(p, cg);
-    int jj = 0;
-    while (true) {
-      const int tb = max(w.s, r0), te = min(w.s + w.tiles, r1);
-      const int L = w.L;
-      // last position row n sees (causal: L - q + i); rows past q*H see L - 1
-      const int lim = min(L - 1, p.causal ? L - p.q_len + qi : L - 1);
-      float m = kRefInit, l = 0.0f;          // m identical in the two threads of a row
-      for (int t = tb; t < te; ++t, ++jj) {
-        const int kb = jj & 1;                 // receive buffer of this tile
-        const int slot = jj % p.nslot;
-        const int tile_pos0 = (t - w.s) * kDecodeTok;
-        const int pos0 = tile_pos0 + qt * kQTok;   // first token of this thread's half
-        // ---- send the next tile's partial before finishing this one ----
-#pragma unroll
-        for (int i = 0; i < kPackWords; ++i) own_cur[i] = own_next[i];
-        if (sending) sending = send_next();
-        // ---- this tile's scores: own rounded partial + the partner's ----
-        const bool rcv =
-            __all_sync(0xffffffffu, mbar_wait_cluster(&recv_full[kb], (jj >> 1) & 1, wc));
-        if (threadIdx.x == 64) MLA_PTRACE(5, jj);
-        float s[kQTok];
-        {
-          const uint32_t oth = recv_s + kb * kXBytes;
-          uint32_t wb[kPackWords];
-#pragma unroll
-          for (int c = 0; c < kPackWords / 4; ++c) {
-            const uint4 vb = ld_shared_v4(oth + x_offset(wi, lane, c));
-            wb[4 * c] = vb.x; wb[4 * c + 1] = vb.y; wb[4 * c + 2] = vb.z; wb[4 * c + 3] = vb.w;
+            for (int i = 0; i < 8; ++i) v[i] = 0u;
           }
-#pragma unroll
-          for (int g = 0; g < kQTok / 4; ++g) {
-            float fa[4], fb[4];
-            unpack_f24(own_cur + 3 * g, fa);
-            unpack_f24(wb + 3 * g, fb);
-#pragma unroll
-            for (int i = 0; i < 4; ++i) s[4 * g + i] = rcv ? fa[i] + fb[i] : 0.0f;
-          }
+          tm_st_x8_s8(trow + kColQ + c0 / 2, v);
         }
-        if (threadIdx.x == 64) MLA_PTRACE(10, jj);
-        __syncwarp();
-        // The received words are in registers (consumed above): release the buffer to the
-        // partner without a release fence, which would wait for this warp's remote stores.
-        if (lane == 1) mbar_arrive_remote_relaxed(kb ? pfree_r1 : pfree_r0);
-        // re-arm this buffer for tile jj + 2 (the partner sends it only after all eight
-        // warps have released the buffer above)
-        if (threadIdx.x == 65 && rcv) mbar_arrive_expect_tx_relaxed(&recv_full[kb], kXBytes);
-
-        // ---- online softmax of row n over this tile (log2 domain, lazy reference) ----
-        if (pos0 + kQTok - 1 > lim) {
-#pragma unroll
-          for (int c = 0; c < kQTok; ++c)
-            if (pos0 + c > lim) s[c] = -INFINITY;
+        for (int c = qt; c < rh / 8; c += 2) {
+          const uint4 v = row_ok ? *reinterpret_cast<const uint4*>(q + r + int(rank) * rh + 8 * c)
+                                 : make_uint4(0, 0, 0, 0);
+          *reinterpret_cast<uint4*>(qrope + swizzled_chunk(n, c, rpitch)) = v;
         }
-        // maximum of the raw scores (a tree; the positive scale is applied once after it)
-        float mt[kQTok / 2];
-#pragma unroll
-        for (int c = 0; c < kQTok / 2; ++c) mt[c] = fmaxf(s[c], s[c + kQTok / 2]);
-#pragma unroll
-        for (int w2 = kQTok / 4; w2 >= 1; w2 >>= 1)
-#pragma unroll
-          for (int c = 0; c < w2; ++c) mt[c] = fmaxf(mt[c], mt[c + w2]);
-        // the row's maximum over both halves (lanes i and i + 16: the same value in both)
-        const float mh = mt[0] * c_log2;
-        const float mx = fmaxf(mh, __shfl_xor_sync(0xffffffffu, mh, 16));
-        if (threadIdx.x == 64) MLA_PTRACE(11, jj);
-        float alpha = 1.0f;
-        if (mx > m + kLazyThreshold) {
-          alpha = ex2_approx(m - mx);          // 0 while m is still kRefInit
-          l *= alpha;
-          m = mx;
-        }
-        // PV(jj-1) reads P and accumulates into O: wait for it before touching either
-        const bool pv_ok =
-            __all_sync(0xffffffffu, jj == 0 || mbar_wait(pv_done, (jj - 1) & 1, wc));
-        if (threadIdx.x == 64) MLA_PTRACE(6, jj);
-        tc_fence_after();
-        if (t > tb && pv_ok && __any_sync(0xffffffffu, alpha != 1.0f)) {
-          for (int c0 = 0; c0 < rhalf; c0 += 32) {
-            float o[16];
-            tm_ld_x16_s16(trow + kColO + c0, o);
-            tmem_wait_ld();
-#pragma unroll
-            for (int c = 0; c < 16; ++c) o[c] *= alpha;
-            tm_st_x16_s16(trow + kColO + c0, reinterpret_cast<const uint32_t*>(o));
-          }
-        }
-        // weights 2^(s * scale - m); the tile's sum in two chains, added to l in a fixed
-        // order (both CTAs of the pair agree bit for bit)
-        uint32_t pk[kQTok / 2];
-        float sa = 0.0f, sb = 0.0f;
-#pragma unroll
-        for (int c = 0; c < kQTok / 2; ++c) {
-          const float p0 = ex2_approx(fmaf(s[2 * c], c_log2, -m));
-          const float p1 = ex2_approx(fmaf(s[2 * c + 1], c_log2, -m));
-          sa += p0;
-          sb += p1;
-          pk[c] = cvt_bf16x2(p0, p1);
-        }
-        l += sa + sb;
-        tm_st_x16_s16(trow + kColP, pk);
-        // cache rows past the context may hold anything (even NaN): zero their latent half
-        // so that 0-weight x garbage cannot reach O
-        if (tile_pos0 + kDecodeTok > L) {
-          const int tok = tid & (kDecodeTok - 1);
-          if (tile_pos0 + tok >= L) {
-            uint8_t* sbase = slots + slot * lay.slot_bytes;
-            for (int k = tid >> 6; k < lb; k += kSoftThreads / kDecodeTok) {
-              uint4* rowp = reinterpret_cast<uint4*>(sbase + k * kBlk + tok * 128);
-#pragma unroll
-              for (int ch = 0; ch < 8; ++ch) rowp[ch] = make_uint4(0, 0, 0, 0);
-            }
-          }
-        }
-        // P (and any O rescale and zeroed rows) complete: hand the tile to the PV issuer
         tmem_wait_st();
-        if (threadIdx.x == 64) MLA_PTRACE(7, jj);
         fence_proxy_async_smem();
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) mbar_arrive(p_full);
-      }
+        if (lane == 0) mbar_arrive(q_full);
+      };
 
-      // ---------------------------- epilogue of this piece --------------------------------
-      const bool fin = __all_sync(0xffffffffu, mbar_wait(pv_done, (jj - 1) & 1, wc));
-      tc_fence_after();
-      const bool aborted = __any_sync(0xffffffffu, !fin || *abort_flag != 0);
-      // the row sum over both halves (the same value in both threads: a + b = b + a)
-      const float lt = l + __shfl_xor_sync(0xffffffffu, l, 16);
-      const bool whole = (tb == w.s) && (te == w.s + w.tiles);
-      const int64_t grow = int64_t(w.b) * p.qH + row;   // global (b, i, h) row
-      const int pslot = piece_slot(vc, w.s, per, p.col_groups, cg);
-      const float lse = (lt > 0.0f && !aborted) ? (m + __log2f(lt)) * kLn2 : -INFINITY;
-      if (row_ok && rank == 0 && qt == 0) {
-        if (whole) p.lse[grow] = lse;
-        else p.part_lse[int64_t(pslot) * kPairRows + n] = lse;
-      }
-      const float inv = (lt > 0.0f && !aborted) ? 1.0f / lt : 0.0f;
-      const int64_t lat0 = int64_t(rank) * rhalf + 16 * qt;   // this thread's 16 of every 32
-      for (int c0 = 0; c0 < rhalf; c0 += 32) {
-        float o[16];
-        if (!aborted) {
-          tm_ld_x16_s16(trow + kColO + c0, o);
-          tmem_wait_ld();
-        } else {
-#pragma unroll
-          for (int c = 0; c < 16; ++c) o[c] = 0.0f;
-        }
-        if (!row_ok) {
-          // padding row past q*H: nothing to write
-        } else if (whole) {
-          uint16_t* dst = p.o_latent + grow * r + lat0 + c0;
-          if (vec_out) {
-#pragma unroll
-            for (int c = 0; c < 16; c += 8)
-              *reinterpret_cast<uint4*>(dst + c) =
-                  make_uint4(cvt_bf16x2(o[c] * inv, o[c + 1] * inv),
-                             cvt_bf16x2(o[c + 2] * inv, o[c + 3] * inv),
-                             cvt_bf16x2(o[c + 4] * inv, o[c + 5] * inv),
-                             cvt_bf16x2(o[c + 6] * inv, o[c + 7] * inv));
+      load_q(sched[0]);
+      UnitWalk w{sched[0], sched[1]};
+      w.load(p, cg);
+      int jj = 0;
+      while (true) {
+        const int tb = max(w.s, r0), te = min(w.s + w.tiles, r1);
+        const int L = w.L;
+        // last position row n sees (causal: L - q + i); rows past q*H see L - 1
+        const int lim = min(L - 1, p.causal ? L - p.q_len + qi : L - 1);
+        float mref = kRefInit, l = 0.0f, lt = 0.0f;   // the same in both threads of a row
+        for (int t = tb; t < te; ++t, ++jj) {
+          const int sb = jj & 1;                 // S buffer and partial buffer of this tile
+          const int slot = jj % p.nslot;
+          const int tile_pos0 = (t - w.s) * kDecodeTok;
+          const int pos0 = tile_pos0 + qt * kHalfTok;   // first token of this thread's half
+          // ---- own partial scores ----
+          float s[kHalfTok];
+          const bool got = __all_sync(0xffffffffu, mbar_wait(&s_full[sb], (jj >> 1) & 1, wc));
+          tc_fence_after();
+          if (got) {
+            tm_ld_x32_s32(trow + kColS + 64 * sb, s);
+            tmem_wait_ld();
           } else {
 #pragma unroll
-            for (int c = 0; c < 16; ++c) dst[c] = f32_to_bf16_rne(o[c] * inv);
+            for (int c = 0; c < kHalfTok; ++c) s[c] = 0.0f;
           }
-        } else {
-          float* dst = p.part_o + (int64_t(pslot) * kPairRows + n) * r + lat0 + c0;
+          if (tr) MLA_PTRACE(10, jj);
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&s_free[sb]);
+          // S of the piece's last tile is complete: the next piece's Q may replace this one
+          if (t == te - 1 && w.s + w.tiles < r1) load_q(w.b + 1);
+          // ---- plus the partner's partial ----
+          const bool rcv =
+              __all_sync(0xffffffffu, mbar_wait_cluster(&xs_full[sb], (jj >> 1) & 1, wc));
+          if (tr) MLA_PTRACE(5, jj);
+          {
+            const uint32_t src = xs_s + sb * kXsBytes;
+            uint32_t wb[kPackWords];
 #pragma unroll
-          for (int c = 0; c < 16; c += 4)
-            *reinterpret_cast<float4*>(dst + c) =
-                make_float4(o[c] * inv, o[c + 1] * inv, o[c + 2] * inv, o[c + 3] * inv);
+            for (int c = 0; c < kPackWords / 4; ++c) {
+              const uint4 v = ld_shared_v4(src + xs_offset(ow, lane, c));
+              wb[4 * c] = v.x; wb[4 * c + 1] = v.y; wb[4 * c + 2] = v.z; wb[4 * c + 3] = v.w;
+            }
+#pragma unroll
+            for (int g = 0; g < kHalfTok / 4; ++g) {
+              float f[4];
+              unpack_f24(wb + 3 * g, f);
+#pragma unroll
+              for (int i = 0; i < 4; ++i) s[4 * g + i] = rcv ? s[4 * g + i] + f[i] : 0.0f;
+            }
+          }
+          __syncwarp();
+          // The received words are in registers: release the buffer to the partner without a
+          // release fence (which would wait for this warp's remote stores), and re-arm it for
+          // tile jj + 2 (the partner sends that only after all four owner warps released it).
+          if (lane == 1) mbar_arrive_remote_relaxed(sb ? xs_free_r1 : xs_free_r0);
+          if (ow == 0 && lane == 0 && rcv) mbar_arrive_expect_tx_relaxed(&xs_full[sb], kXsBytes);
+
+          // ---- online softmax of row n over this tile (log2 domain, lazy reference) ----
+          if (pos0 + kHalfTok - 1 > lim) {
+#pragma unroll
+            for (int c = 0; c < kHalfTok; ++c)
+              if (pos0 + c > lim) s[c] = -INFINITY;
+          }
+          float mt[kHalfTok / 2];
+#pragma unroll
+          for (int c = 0; c < kHalfTok / 2; ++c) mt[c] = fmaxf(s[c], s[c + kHalfTok / 2]);
+#pragma unroll
+          for (int w2 = kHalfTok / 4; w2 >= 1; w2 >>= 1)
+#pragma unroll
+            for (int c = 0; c < w2; ++c) mt[c] = fmaxf(mt[c], mt[c + w2]);
+          const float mh = mt[0] * c_log2;
+          const float mx = fmaxf(mh, __shfl_xor_sync(0xffffffffu, mh, 16));
+          float alpha = 1.0f;
+          if (mx > mref + kLazyThreshold) {
+            alpha = ex2_approx(mref - mx);       // 0 while mref is still kRefInit
+            l *= alpha;
+            mref = mx;
+          }
+          // O rows of an earlier tile of the piece: rescale once PV(jj - 1) has landed
+          if (t > tb && __any_sync(0xffffffffu, alpha != 1.0f)) {
+            const bool pv_ok = __all_sync(
+                0xffffffffu, mbar_wait(&pv_done[(jj - 1) & 1], ((jj - 1) >> 1) & 1, wc));
+            tc_fence_after();
+            if (pv_ok) {
+              for (int c0 = 0; c0 < rhalf; c0 += 32) {
+                float o[16];
+                tm_ld_x16_s16(trow + kColO + c0, o);
+                tmem_wait_ld();
+#pragma unroll
+                for (int c = 0; c < 16; ++c) o[c] *= alpha;
+                tm_st_x16_s16(trow + kColO + c0, reinterpret_cast<const uint32_t*>(o));
+              }
+            }
+          }
+          // weights 2^(s * scale - m) over the S buffer (its scores are in registers)
+          uint32_t pk[kHalfTok / 2];
+          float sa = 0.0f, sc = 0.0f;
+#pragma unroll
+          for (int c = 0; c < kHalfTok / 2; ++c) {
+            const float p0 = ex2_approx(fmaf(s[2 * c], c_log2, -mref));
+            const float p1 = ex2_approx(fmaf(s[2 * c + 1], c_log2, -mref));
+            sa += p0;
+            sc += p1;
+            pk[c] = cvt_bf16x2(p0, p1);
+          }
+          l += sa + sc;
+          lt = l + __shfl_xor_sync(0xffffffffu, l, 16);
+          tm_st_x16_s16(trow + kColS + 64 * sb, pk);
+          // ---- the same weights, the rescale factor and the running sum to the partner ----
+          const bool pfree =
+              __all_sync(0xffffffffu, jj == 0 || mbar_wait_cluster(xp_free, (jj - 1) & 1, wc));
+          if (pfree) {
+#pragma unroll
+            for (int i = 0; i < 4; ++i)
+              st_async_v4(xp_r + xp_offset(m, 4 * qt + i),
+                          make_uint4(pk[4 * i], pk[4 * i + 1], pk[4 * i + 2], pk[4 * i + 3]),
+                          xp_full_r);
+            if (qt == 0)
+              st_async_v2(xp_r + xp_scalars(m),
+                          make_uint2(__float_as_uint(alpha), __float_as_uint(lt)), xp_full_r);
+          }
+          if (tr) MLA_PTRACE(6, jj);
+          // cache rows past the context may hold anything (even NaN): zero their latent half
+          // so that 0-weight x garbage cannot reach O
+          if (tile_pos0 + kDecodeTok > L) {
+            const int tid = ow * 32 + lane;      // 0..127
+            const int tok = tid & (kDecodeTok - 1);
+            if (tile_pos0 + tok >= L) {
+              uint8_t* sbase = slots + slot * lay.slot_bytes;
+              for (int k = tid >> 6; k < lb; k += 2) {
+                uint4* rowp = reinterpret_cast<uint4*>(sbase + k * kBlk + tok * 128);
+#pragma unroll
+                for (int ch = 0; ch < 8; ++ch) rowp[ch] = make_uint4(0, 0, 0, 0);
+              }
+            }
+          }
+          // P (and any O rescale and zeroed rows) complete: hand the tile to the PV issuer
+          tmem_wait_st();
+          fence_proxy_async_smem();
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&p_full[sb]);
+        }
+
+        // ------------------------- epilogue of this piece (own rows) -----------------------
+        const int jl = jj - 1;
+        const bool fin = __all_sync(0xffffffffu, mbar_wait(&pv_done[jl & 1], (jl >> 1) & 1, wc));
+        tc_fence_after();
+        const bool aborted = __any_sync(0xffffffffu, !fin || *abort_flag != 0);
+        const bool whole = (tb == w.s) && (te == w.s + w.tiles);
+        const int64_t grow = int64_t(w.b) * p.qH + row;   // global (b, i, h) row
+        const int pslot = piece_slot(vc, w.s, per, p.col_groups, cg);
+        const float lse = (lt > 0.0f && !aborted) ? (mref + __log2f(lt)) * kLn2 : -INFINITY;
+        if (row_ok && qt == 0) {
+          if (whole) p.lse[grow] = lse;
+          else p.part_lse[int64_t(pslot) * kPairRows + n] = lse;
+        }
+        const float inv = (lt > 0.0f && !aborted) ? 1.0f / lt : 0.0f;
+        const int64_t lat0 = int64_t(rank) * rhalf + 16 * qt;   // this thread's 16 of every 32
+        for (int c0 = 0; c0 < rhalf; c0 += 32) {
+          float o[16];
+          if (!aborted) {
+            tm_ld_x16_s16(trow + kColO + c0, o);
+            tmem_wait_ld();
+          } else {
+#pragma unroll
+            for (int c = 0; c < 16; ++c) o[c] = 0.0f;
+          }
+          if (!row_ok) {
+            // padding row past q*H: nothing to write
+          } else if (whole) {
+            uint16_t* dst = p.o_latent + grow * r + lat0 + c0;
+            if (vec_out) {
+#pragma unroll
+              for (int c = 0; c < 16; c += 8)
+                *reinterpret_cast<uint4*>(dst + c) =
+                    make_uint4(cvt_bf16x2(o[c] * inv, o[c + 1] * inv),
+                               cvt_bf16x2(o[c + 2] * inv, o[c + 3] * inv),
+                               cvt_bf16x2(o[c + 4] * inv, o[c + 5] * inv),
+                               cvt_bf16x2(o[c + 6] * inv, o[c + 7] * inv));
+            } else {
+#pragma unroll
+              for (int c = 0; c < 16; ++c) dst[c] = f32_to_bf16_rne(o[c] * inv);
+            }
+          } else {
+            float* dst = p.part_o + (int64_t(pslot) * kPairRows + n) * r + lat0 + c0;
+#pragma unroll
+            for (int c = 0; c < 16; c += 4)
+              *reinterpret_cast<float4*>(dst + c) =
+                  make_float4(o[c] * inv, o[c + 1] * inv, o[c + 2] * inv, o[c + 3] * inv);
+          }
+        }
+        tc_fence_before();
+        w.s += w.tiles;
+        ++w.b;
+        if (w.s >= r1) break;
+        w.load(p, cg);
+      }
+    } else if (hl == 0) {
+      // ---------------- sender: the partner rows' partial scores, one row per lane ---------
+      const int n = 32 * sp + lane;           // query row (TMEM lane)
+      const uint32_t tq = tmem + (uint32_t(32 * sp) << 16);
+      const int row = cg * kPairRows + n;
+      const bool row_ok = row < p.qH;
+      // where the partner's owner threads of this row read: warp 2 (lane / 16) + (sp & 1),
+      // lanes (lane % 16) and (lane % 16) + 16 for the two token halves
+      const int ow_o = 2 * (lane >> 4) + (sp & 1);
+      const bool tr = ((sp & 1) == 0 && lane == 0);
+      (void)tr;
+
+      // This CTA's half of Q row n (one thread per row), as the owners' load_q.
+      auto load_q = [&](int b) {
+        const uint16_t* q = p.q_ext + (int64_t(b) * p.qH + row) * p.D;
+        for (int c0 = 0; c0 < rhalf; c0 += 16) {
+          const uint16_t* src = q + int(rank) * rhalf + c0;
+          uint32_t v[8];
+          if (row_ok) {
+            const uint4 a = *reinterpret_cast<const uint4*>(src);
+            const uint4 bb = *reinterpret_cast<const uint4*>(src + 8);
+            v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w;
+            v[4] = bb.x; v[5] = bb.y; v[6] = bb.z; v[7] = bb.w;
+          } else {
+#pragma unroll
+            for (int i = 0; i < 8; ++i) v[i] = 0u;
+          }
+          tmem_st8(tq + kColQ + c0 / 2, v);
+        }
+        for (int c = 0; c < rh / 8; ++c) {
+          const uint4 v = row_ok ? *reinterpret_cast<const uint4*>(q + r + int(rank) * rh + 8 * c)
+                                 : make_uint4(0, 0, 0, 0);
+          *reinterpret_cast<uint4*>(qrope + swizzled_chunk(n, c, rpitch)) = v;
+        }
+        tmem_wait_st();
+        fence_proxy_async_smem();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(q_full);
+      };
+
+      load_q(sched[0]);
+      UnitWalk w{sched[0], sched[1]};
+      int jj = 0;
+      for (; w.s < r1; w.s += w.tiles, ++w.b) {
+        w.load(p, cg);
+        const int tb = max(w.s, r0), te = min(w.s + w.tiles, r1);
+        for (int t = tb; t < te; ++t, ++jj) {
+          const int sb = jj & 1;
+          float x[kDecodeTok];
+          const bool got = __all_sync(0xffffffffu, mbar_wait(&s_full[sb], (jj >> 1) & 1, wc));
+          tc_fence_after();
+          if (got) {
+            tmem_ld32(tq + kColS + 64 * sb, x);
+            tmem_ld32(tq + kColS + 64 * sb + 32, x + 32);
+            tmem_wait_ld();
+          } else {
+#pragma unroll
+            for (int c = 0; c < kDecodeTok; ++c) x[c] = 0.0f;
+          }
+          if (tr) MLA_PTRACE(3, jj);
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&s_free[sb]);
+          if (t == te - 1 && w.s + w.tiles < r1) load_q(w.b + 1);
+          uint32_t pw[2 * kPackWords];
+#pragma unroll
+          for (int g = 0; g < kDecodeTok / 4; ++g) pack_f24(x + 4 * g, pw + 3 * g);
+          // into the partner's buffer sb once its owners consumed tile jj - 2 from it: stores
+          // from registers over the SM-to-SM network, completing on the partner's mbarrier
+          const bool free_ok = __all_sync(
+              0xffffffffu, jj < 2 || mbar_wait_cluster(&xs_free[sb], ((jj - 2) >> 1) & 1, wc));
+          if (free_ok) {
+            const uint32_t dst = xs_r + sb * kXsBytes;
+            const uint32_t rb = sb ? xs_full_r1 : xs_full_r0;
+#pragma unroll
+            for (int h = 0; h < 2; ++h)
+#pragma unroll
+              for (int c = 0; c < kPackWords / 4; ++c) {
+                const uint32_t* wp = pw + kPackWords * h + 4 * c;
+                st_async_v4(dst + xs_offset(ow_o, (lane & 15) + 16 * h, c),
+                            make_uint4(wp[0], wp[1], wp[2], wp[3]), rb);
+              }
+          }
+          if (tr) MLA_PTRACE(4, jj);
         }
       }
-      tc_fence_before();
-      w.s += w.tiles;
-      ++w.b;
-      if (w.s >= r1) break;
+    } else {
+      // ---------------- receiver: the partner's weights for its rows; their epilogue ------
+      const int n = 32 * sp + lane;           // query row (TMEM lane)
+      const int m = n & 63;                   // row within the partner's block
+      const uint32_t tq = tmem + (uint32_t(32 * sp) << 16);
+      const int row = cg * kPairRows + n;
+      const bool row_ok = row < p.qH;
+      const bool tr = ((sp & 1) == 0 && lane == 0);
+      (void)tr;
+      UnitWalk w{sched[0], sched[1]};
       w.load(p, cg);
+      int jj = 0;
+      while (true) {
+        const int tb = max(w.s, r0), te = min(w.s + w.tiles, r1);
+        float lt = 0.0f;
+        for (int t = tb; t < te; ++t, ++jj) {
+          const int sb = jj & 1;
+          const bool rcv = __all_sync(0xffffffffu, mbar_wait_cluster(xp_full, jj & 1, wc));
+          if (tr) MLA_PTRACE(7, jj);
+          uint32_t pk[kDecodeTok / 2];
+          float alpha = 1.0f;
+          if (rcv) {
+#pragma unroll
+            for (int c = 0; c < kDecodeTok / 8; ++c) {
+              const uint4 v = ld_shared_v4(xp_s + xp_offset(m, c));
+              pk[4 * c] = v.x; pk[4 * c + 1] = v.y; pk[4 * c + 2] = v.z; pk[4 * c + 3] = v.w;
+            }
+            const uint2 sc = ld_shared_v2(xp_s + xp_scalars(m));
+            alpha = __uint_as_float(sc.x);
+            lt = __uint_as_float(sc.y);
+          } else {
+#pragma unroll
+            for (int c = 0; c < kDecodeTok / 2; ++c) pk[c] = 0u;
+            lt = 0.0f;
+          }
+          __syncwarp();
+          // consumed into registers: release the buffer (relaxed) and re-arm it for tile jj + 1
+          if (lane == 1) mbar_arrive_remote_relaxed(xp_free_r);
+          if ((sp & 1) == 0 && lane == 0 && rcv) mbar_arrive_expect_tx_relaxed(xp_full, kXpBytes);
+          // the owner moved its reference: rescale these rows of this CTA's O half the same way
+          if (t > tb && __any_sync(0xffffffffu, alpha != 1.0f)) {
+            const bool pv_ok = __all_sync(
+                0xffffffffu, mbar_wait(&pv_done[(jj - 1) & 1], ((jj - 1) >> 1) & 1, wc));
+            tc_fence_after();
+            if (pv_ok) {
+              for (int c0 = 0; c0 < rhalf; c0 += 32) {
+                float o[32];
+                tmem_ld32(tq + kColO + c0, o);
+                tmem_wait_ld();
+#pragma unroll
+                for (int c = 0; c < 32; ++c) o[c] *= alpha;
+                tmem_st32(tq + kColO + c0, reinterpret_cast<const uint32_t*>(o));
+              }
+            }
+          }
+          tmem_st32(tq + kColS + 64 * sb, pk);
+          tmem_wait_st();
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&p_full[sb]);
+          if (tr) MLA_PTRACE(11, jj);
+        }
+
+        // ---------------------- epilogue of this piece (the partner's rows) ----------------
+        const int jl = jj - 1;
+        const bool fin = __all_sync(0xffffffffu, mbar_wait(&pv_done[jl & 1], (jl >> 1) & 1, wc));
+        tc_fence_after();
+        const bool aborted = __any_sync(0xffffffffu, !fin || *abort_flag != 0);
+        const bool whole = (tb == w.s) && (te == w.s + w.tiles);
+        const int64_t grow = int64_t(w.b) * p.qH + row;
+        const int pslot = piece_slot(vc, w.s, per, p.col_groups, cg);
+        const float inv = (lt > 0.0f && !aborted) ? 1.0f / lt : 0.0f;
+        const int64_t lat0 = int64_t(rank) * rhalf;
+        for (int c0 = 0; c0 < rhalf; c0 += 32) {
+          float o[32];
+          if (!aborted) {
+            tmem_ld32(tq + kColO + c0, o);
+            tmem_wait_ld();
+          } else {
+#pragma unroll
+            for (int c = 0; c < 32; ++c) o[c] = 0.0f;
+          }
+          if (!row_ok) {
+            // padding row past q*H: nothing to write
+          } else if (whole) {
+            uint16_t* dst = p.o_latent + grow * r + lat0 + c0;
+            if (vec_out) {
+#pragma unroll
+              for (int c = 0; c < 32; c += 8)
+                *reinterpret_cast<uint4*>(dst + c) =
+                    make_uint4(cvt_bf16x2(o[c] * inv, o[c + 1] * inv),
+                               cvt_bf16x2(o[c + 2] * inv, o[c + 3] * inv),
+                               cvt_bf16x2(o[c + 4] * inv, o[c + 5] * inv),
+                               cvt_bf16x2(o[c + 6] * inv, o[c + 7] * inv));
+            } else {
+#pragma unroll
+              for (int c = 0; c < 32; ++c) dst[c] = f32_to_bf16_rne(o[c] * inv);
+            }
+          } else {
+            float* dst = p.part_o + (int64_t(pslot) * kPairRows + n) * r + lat0 + c0;
+#pragma unroll
+            for (int c = 0; c < 32; c += 4)
+              *reinterpret_cast<float4*>(dst + c) =
+                  make_float4(o[c] * inv, o[c + 1] * inv, o[c + 2] * inv, o[c + 3] * inv);
+          }
+        }
+        tc_fence_before();
+        w.s += w.tiles;
+        ++w.b;
+        if (w.s >= r1) break;
+        w.load(p, cg);
+      }
     }
   }
 

@@ -74,6 +74,9 @@ cudaError_t launch_decode(const DecodeParams& p, int ncol, dim3 grid, size_t sme
 
 // Blocks of up to 128 query rows: a cluster of two CTAs splits the latent (decode_pair.cu).
 constexpr int kPairRows = 128;
+// Cache slots per CTA of the pair kernel. More TMA tiles in flight per SM lengthened each
+// tile's load latency by more than they added bandwidth (measured on B200: 4 slots beat 5).
+constexpr int kPairMaxSlots = 4;
 size_t decode_pair_smem_bytes(int r, int rope_half, int nslot);
 // Clusters of two that can be resident at once with `smem` bytes each (0 if unknown).
 int decode_pair_max_clusters(size_t smem);
