@@ -67,46 +67,129 @@ def algorithmic_work(cfg, seq_lens):
     return nbytes, flops
 
 
+# Child process of ClockSampler: polls NVML in a tight loop (no GIL shared with the timed
+# loop) and appends "time, sm_mhz, max_mhz, power_w, reasons" rows to a file until killed.
+_NVML_SAMPLER = r"""
+import sys, time
+import pynvml
+pynvml.nvmlInit()
+gpu, path = sys.argv[1], sys.argv[2]
+h = (pynvml.nvmlDeviceGetHandleByUUID(gpu) if gpu.startswith("GPU-")
+     else pynvml.nvmlDeviceGetHandleByIndex(int(gpu)))
+reasons = getattr(pynvml, "nvmlDeviceGetCurrentClocksEventReasons", None) or \
+    pynvml.nvmlDeviceGetCurrentClocksThrottleReasons
+mx = pynvml.nvmlDeviceGetMaxClockInfo(h, pynvml.NVML_CLOCK_SM)
+with open(path, "w", buffering=1) as fh:
+    while True:
+        t = time.time()
+        sm = pynvml.nvmlDeviceGetClockInfo(h, pynvml.NVML_CLOCK_SM)
+        rs = int(reasons(h))
+        pw = pynvml.nvmlDeviceGetPowerUsage(h) / 1000.0
+        fh.write(f"{t:.6f},{sm},{mx},{pw:.2f},{rs}\n")
+"""
+
+
 class ClockSampler:
-    """nvidia-smi clocks and throttle reasons sampled every 200 ms while running."""
+    """SM clock, power and clock-event (throttle) reasons of this GPU during the timed region:
+    a child process polls NVML as fast as it answers (a timed region of a few milliseconds
+    still gets samples); nvidia-smi every 200 ms when NVML is not importable. Only samples
+    between mark_start() and mark_end() count. Rows go to gpurun_out/clocks_rank<R>.csv."""
     Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
          "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
          "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    # NVML clock-event reason bits, in the order of the last four nvidia-smi columns above
+    BITS = (0x8, 0x40, 0x20, 0x4)
+    NAMES = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
 
     def __init__(self, gpu_id: str):
-        self.gpu = gpu_id  # nvidia-smi -i accepts an index or a UUID
+        self.gpu = gpu_id  # a UUID ("GPU-...") or an index
         self.proc = None
+        self.kind = None   # "nvml" or "nvidia-smi"
         self.path = None
+        self.rows = None   # (time, sm_mhz, max_mhz, power_w, reasons bitmask) for "nvml"
+        self.t0 = self.t1 = None
 
     def __enter__(self):
         try:
             out_dir = os.path.join(ROOT, "gpurun_out")
             os.makedirs(out_dir, exist_ok=True)
             self.path = os.path.join(out_dir, f"clocks_rank{os.environ.get('RANK', '0')}.csv")
-            self.fh = open(self.path, "w")
-            self.proc = subprocess.Popen(["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.Q}",
-                                          "--format=csv,noheader,nounits", "-lms", "200"],
-                                         stdout=self.fh, stderr=subprocess.DEVNULL)
-            time.sleep(0.3)
+            if os.path.exists(self.path):
+                os.remove(self.path)
         except Exception:
-            self.proc = None
+            self.path = None
+            return self
+        try:
+            import pynvml  # noqa: F401  (the child needs it)
+            self.proc = subprocess.Popen([sys.executable, "-c", _NVML_SAMPLER, str(self.gpu), self.path],
+                                         stdout=subprocess.DEVNULL, stderr=subprocess.DEVNULL)
+            self.kind = "nvml"
+            t_end = time.time() + 10.0
+            while time.time() < t_end and self.proc.poll() is None:
+                if os.path.exists(self.path) and os.path.getsize(self.path) > 0:
+                    break
+                time.sleep(0.01)
+            if self.proc.poll() is not None:
+                raise RuntimeError("NVML sampler exited")
+        except Exception:
+            self._stop()
+            self.kind = None
+            try:
+                self.fh = open(self.path, "w")
+                self.proc = subprocess.Popen(["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.Q}",
+                                              "--format=csv,noheader,nounits", "-lms", "200"],
+                                             stdout=self.fh, stderr=subprocess.DEVNULL)
+                self.kind = "nvidia-smi"
+                time.sleep(0.3)
+            except Exception:
+                self.proc = None
         return self
 
-    def __exit__(self, *a):
+    def mark_start(self):
+        self.t0 = time.time()
+
+    def mark_end(self):
+        self.t1 = time.time()
+
+    def _stop(self):
         if self.proc is not None:
-            time.sleep(0.25)
             self.proc.terminate()
             try:
                 self.proc.wait(timeout=5)
             except Exception:
                 self.proc.kill()
+        self.proc = None
+
+    def __exit__(self, *a):
+        if self.kind == "nvidia-smi":
+            time.sleep(0.25)
+            self._stop()
             self.fh.close()
+        else:
+            time.sleep(0.02)
+            self._stop()
+            self.rows = []
+            try:
+                for line in open(self.path):
+                    f = line.strip().split(",")
+                    if len(f) == 5:
+                        self.rows.append((float(f[0]), float(f[1]), float(f[2]), float(f[3]), int(f[4])))
+            except Exception:
+                pass
 
     def summary(self):
-        if self.proc is None or self.path is None or not os.path.exists(self.path):
+        if self.kind == "nvml":
+            rows = [r for r in (self.rows or [])
+                    if self.t0 is None or self.t1 is None or self.t0 <= r[0] <= self.t1]
+            if not rows:
+                return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"]}
+            reasons = sorted({n for r in rows for n, b in zip(self.NAMES, self.BITS) if r[4] & b})
+            return {"sm_mhz": statistics.median(r[1] for r in rows), "sm_max_mhz": rows[0][2],
+                    "power_w": round(statistics.median(r[3] for r in rows), 1),
+                    "samples": len(rows), "source": "nvml", "reasons": reasons}
+        if self.kind != "nvidia-smi" or self.path is None or not os.path.exists(self.path):
             return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"]}
         sms, mx, reasons = [], None, set()
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
         for line in open(self.path):
             f = [x.strip() for x in line.split(",")]
             if len(f) < 9:
@@ -116,14 +199,14 @@ class ClockSampler:
             except ValueError:
                 continue
             sms.append(sm)
-            for n, v in zip(names, f[5:9]):
+            for n, v in zip(self.NAMES, f[5:9]):
                 if v.lower() == "active":
                     reasons.add(n)
         if not sms:
             return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"]}
         loaded = [s for s in sms if s > 0.5 * (mx or max(sms))] or sms
         return {"sm_mhz": statistics.median(loaded), "sm_max_mhz": mx, "samples": len(sms),
-                "reasons": sorted(reasons)}
+                "source": "nvidia-smi", "reasons": sorted(reasons)}
 
 
 def uses_pair_kernel(cfg):
@@ -268,6 +351,7 @@ def run_gpu(args, cfg, rank, world, dist):
     evs = []
     with ClockSampler(_gpu_id(local)) as clk:
         barrier()
+        clk.mark_start()
         for _ in range(args.steps):
             if flush is not None:
                 flush.zero_()
@@ -275,6 +359,7 @@ def run_gpu(args, cfg, rank, world, dist):
             one_step(e)
             evs.append(e)
         barrier()
+        clk.mark_end()
     step_ms = [e[0].elapsed_time(e[3]) for e in evs]
     dec_ms = [e[1].elapsed_time(e[2]) for e in evs]
     t_step = sum(step_ms) / len(step_ms)

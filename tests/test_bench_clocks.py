@@ -1,0 +1,50 @@
+"""Host logic of bench.py's clock record: only samples inside the timed region count, and the
+clock-event reason bits decode to the names the JSON line reports (no GPU, no NVML)."""
+import importlib.util
+import os
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _bench():
+    spec = importlib.util.spec_from_file_location("bench_mod", os.path.join(ROOT, "bench.py"))
+    mod = importlib.util.module_from_spec(spec)
+    spec.loader.exec_module(mod)
+    return mod
+
+
+def _sampler(rows, t0, t1):
+    b = _bench()
+    s = b.ClockSampler("0")
+    s.kind = "nvml"              # as if the NVML sampler had run
+    s.rows = rows
+    s.t0, s.t1 = t0, t1
+    return s
+
+
+def test_window_and_reasons():
+    rows = [
+        (0.0, 1965, 1965, 250.0, 0x0),     # before the timed region: ignored
+        (1.0, 1900, 1965, 990.0, 0x4),     # sw_power_cap
+        (1.1, 1880, 1965, 995.0, 0x4),
+        (1.2, 1920, 1965, 985.0, 0x0),
+        (3.0, 1965, 1965, 240.0, 0x40),    # after: ignored (hw_thermal_slowdown not reported)
+    ]
+    s = _sampler(rows, 0.5, 2.0).summary()
+    assert s["samples"] == 3
+    assert s["sm_mhz"] == 1900
+    assert s["sm_max_mhz"] == 1965
+    assert s["power_w"] == 990.0
+    assert s["reasons"] == ["sw_power_cap"]
+
+
+def test_all_reason_bits():
+    rows = [(1.0, 1000, 1965, 500.0, 0x8 | 0x20 | 0x40 | 0x4)]
+    s = _sampler(rows, 0.0, 2.0).summary()
+    assert s["reasons"] == sorted(["hw_slowdown", "sw_thermal_slowdown", "hw_thermal_slowdown",
+                                   "sw_power_cap"])
+
+
+def test_no_samples_in_window():
+    s = _sampler([(0.0, 1965, 1965, 250.0, 0)], 1.0, 2.0).summary()
+    assert s["reasons"] == ["unsampled"]
