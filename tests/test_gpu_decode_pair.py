@@ -1,8 +1,10 @@
 """Decode with more than 64 query rows per sequence: blocks of 128 rows on clusters of two
-CTAs that split the latent and swap partial scores through distributed shared memory.
-Parity with the fp64 oracle of the unabsorbed form on the shapes that take this path:
-several row blocks, padding rows past q*H, rank 256, ragged and edge lengths; plus split
-and paging invariance and the bounds guard on this path."""
+CTAs that split the latent; each CTA runs the softmax of half the rows on its own and the
+partner's partial scores (swapped through distributed shared memory) and returns the
+weights. Parity with the fp64 oracle of the unabsorbed form on the shapes that take this
+path: several row blocks, padding rows past q*H, ranks 256 / 384 / 512, rotary widths 32 /
+64 / 128 (the three shared-memory swizzles of Q's rotary half), ragged and edge lengths;
+plus split and paging invariance and the bounds guard on this path."""
 import numpy as np
 import pytest
 import torch
@@ -27,6 +29,15 @@ PAIR = {
     "deepseek_ragged": shrink(DS, batch=9, lens_range=(1, 900), name="deepseek_ragged"),
     # heads sharing 4 rotary groups of 16: rotary half 32
     "groups4": shrink(DS, batch=2, context=260, num_kv_groups=4, rope_dim=16, name="groups4"),
+    # rank 384: three latent blocks per CTA, one of them from shared memory
+    "rank384": shrink(DS, batch=2, context=300, kv_lora_rank=384, name="rank384"),
+    # 2 groups x 64 rotary dims: rotary half 64 (128-byte swizzle), fewer cache slots
+    "rope128": shrink(DS, batch=2, context=400, num_kv_groups=2, rope_dim=64, name="rope128"),
+    # 32 rotary dims shared by all heads: rotary half 16 (32-byte swizzle, one K step)
+    "rope32": shrink(DS, batch=2, context=350, rope_dim=32, name="rope32"),
+    # 32 heads x 4 query tokens: causal inside the block, 128 rows
+    "heads32_q4": shrink(HYB, batch=3, context=500, num_heads=32, q_len=4, kv_lora_rank=512,
+                         name="heads32_q4"),
 }
 
 
