@@ -54,8 +54,8 @@ class GpuProblem:
             sin = np.broadcast_to(sin[None], (B,) + sin.shape)
             mla.mla_cache_append(self.dims, torch.stack([c[:n] for c, _ in ctx]).to(dev),
                                  torch.stack([k[:n] for _, k in ctx]).to(dev),
-                                 torch.from_numpy(np.array(cos, copy=True)).to(dev),
-                                 torch.from_numpy(np.array(sin, copy=True)).to(dev),
+                                 torch.from_numpy(np.array(cos, order="C")).to(dev),
+                                 torch.from_numpy(np.array(sin, order="C")).to(dev),
                                  self.block_table, torch.zeros(B, dtype=torch.int32, device=dev),
                                  self.cache, dev_error=self.err)
             for b, (c_kv, k_r) in enumerate(ctx):
