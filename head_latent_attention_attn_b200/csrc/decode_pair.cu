@@ -87,19 +87,17 @@ constexpr int kMiscInts = 32;
 
 struct PairLayout {
   uint32_t slot_bytes, rope_off, qrope_off, xs_off, xp_off, misc_off, bar_off, total;
-  int nb;   // TMA barriers per slot: one per latent block and one for the rotary block
 };
 
 __host__ __device__ inline uint32_t round_up_p(uint32_t x, uint32_t a) {
   return (x + a - 1) / a * a;
 }
 
-__host__ __device__ constexpr int pair_bars(int nslot, int nb) { return nslot * nb + nslot + 16; }
+__host__ __device__ constexpr int pair_bars(int nslot) { return 2 * nslot + 16; }
 
 __host__ __device__ inline PairLayout pair_layout(int r, int rope_half, int nslot) {
   PairLayout L;
   const int lb = r / 128;                         // 64-column latent blocks per CTA
-  L.nb = lb + 1;
   L.rope_off = uint32_t(lb) * kBlk;
   L.slot_bytes = round_up_p(L.rope_off + uint32_t(kDecodeTok) * rope_half * 2, 1024);
   uint32_t off = uint32_t(nslot) * L.slot_bytes;
@@ -112,7 +110,7 @@ __host__ __device__ inline PairLayout pair_layout(int r, int rope_half, int nslo
   L.misc_off = off;
   off += 4 * kMiscInts;
   L.bar_off = round_up_p(off, 8);
-  off = L.bar_off + 8 * pair_bars(nslot, L.nb);
+  off = L.bar_off + 8 * pair_bars(nslot);
   L.total = off + 1024;                           // slack for 1024-byte alignment
   return L;
 }
@@ -244,9 +242,10 @@ __global__ void __launch_bounds__(kThreads, 1)
   int* warp_sum = misc + 8;
   static_assert(8 + kThreads / 32 <= kMiscInts, "misc ints overflow into the mbarriers");
   uint64_t* bars = reinterpret_cast<uint64_t*>(base + lay.bar_off);
-  const int nb = lay.nb;
-  uint64_t* full = bars;                               // [slot][nb]
-  uint64_t* empty = full + p.nslot * nb;               // [slot]
+  // One barrier per slot for all of a page's TMA boxes: the S issuer needs every box before
+  // it starts, and each mbarrier operation here costs a few hundred cycles of latency.
+  uint64_t* full = bars;                               // [slot]
+  uint64_t* empty = full + p.nslot;                    // [slot]
   uint64_t* q_full = empty + p.nslot;                  // Q of the piece in TMEM and smem
   uint64_t* s_full = q_full + 1;                       // [2] S buffer computed
   uint64_t* s_free = s_full + 2;                       // [2] S buffer read by all readers
@@ -270,7 +269,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < p.nslot; ++s) {
-      for (int k = 0; k < nb; ++k) mbar_init(&full[s * nb + k], 1);
+      mbar_init(&full[s], 1);
       mbar_init(&empty[s], 1);
     }
     mbar_init(q_full, 6);                              // 4 owner + 2 sender warps
@@ -336,14 +335,11 @@ __global__ void __launch_bounds__(kThreads, 1)
             page = 0;
           }
           uint8_t* sbase = slots + slot * lay.slot_bytes;
-          for (int k = 0; k < lb; ++k) {
-            uint64_t* fb = &full[slot * nb + k];
-            mbar_arrive_expect_tx(fb, kBlk);
+          uint64_t* fb = &full[slot];
+          mbar_arrive_expect_tx(fb, uint32_t(lb) * kBlk + rope_bytes);
+          for (int k = 0; k < lb; ++k)
             tma_load_2d(sbase + k * kBlk, &p.tm_cache, int(rank) * rhalf + k * 64,
                         page * kDecodeTok, fb);
-          }
-          uint64_t* fb = &full[slot * nb + lb];
-          mbar_arrive_expect_tx(fb, rope_bytes);
           tma_load_2d(sbase + lay.rope_off, &p.tm_rope, r + int(rank) * rh, page * kDecodeTok,
                       fb);
           MLA_PTRACE(0, jj);
@@ -351,8 +347,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       // Drain: never leave while copies into this CTA's shared memory are in flight.
       for (int j = (jj > p.nslot ? jj - p.nslot : 0); j < jj; ++j)
-        for (int k = 0; k < nb; ++k)
-          mbar_wait_bounded(&full[(j % p.nslot) * nb + k], (j / p.nslot) & 1, 200000000ull);
+        mbar_wait_bounded(&full[j % p.nslot], (j / p.nslot) & 1, 200000000ull);
     }
     __syncwarp();
   } else if (warp == 1) {
@@ -377,9 +372,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           const int slot = jj % p.nslot;
           const int sb = jj & 1;
           // every block of the tile landed, then the S buffer free
-          for (int k = 0; ok && k <= lb; ++k)
-            ok = mbar_wait(&full[slot * nb + k], (jj / p.nslot) & 1, wc);
-          if (!ok) break;
+          if (!mbar_wait(&full[slot], (jj / p.nslot) & 1, wc)) { ok = false; break; }
           MLA_PTRACE(1, jj);
           if (jj >= 2 && (!mbar_wait(&s_free[sb], ((jj - 2) >> 1) & 1, wc) ||
                           !mbar_wait(&pv_done[sb], ((jj - 2) >> 1) & 1, wc))) {
