@@ -37,7 +37,7 @@ namespace mla {
 // Optional per-tile timeline of CTA 0 (compile with -DMLA_TRACE; read with mla_trace_read).
 // Events: 0 producer starts a tile, 1 S issued (all blocks landed), 2 S committed, 3 PV
 // committed, 4 softmax sees S, 5 after the vote barrier, 6 P buffer free, 7 P written
-// and PV about to be issued, 8 producer finished issuing the tile, 9 first block landed.
+// and PV about to be issued, 8 producer finished issuing the tile, 9 the whole page landed.
 #ifdef MLA_TRACE
 constexpr int kTraceTiles = 512;
 __device__ unsigned long long g_mla_trace[10 * kTraceTiles + 1];
@@ -70,7 +70,7 @@ struct DecodeLayout {
 
 __host__ __device__ inline uint32_t round_up(uint32_t x, uint32_t a) { return (x + a - 1) / a * a; }
 
-__host__ __device__ constexpr int num_bars(int nslot, int nblk) { return nslot * nblk + nslot + 8; }
+__host__ __device__ constexpr int num_bars(int nslot) { return 2 * nslot + 8; }
 
 __host__ __device__ inline DecodeLayout decode_layout(int ncol, int nblk, int slot_blocks,
                                                       int nslot, int npt) {
@@ -91,7 +91,7 @@ __host__ __device__ inline DecodeLayout decode_layout(int ncol, int nblk, int sl
   L.misc_off = off;                // int misc[kMiscInts], index map in the kernel
   off += 4 * kMiscInts;
   L.bar_off = round_up(off, 8);
-  off = L.bar_off + 8 * num_bars(nslot, nblk);
+  off = L.bar_off + 8 * num_bars(nslot);
   L.total = off + 1024;            // slack for 1024-byte alignment of the base
   return L;
 }
@@ -178,8 +178,11 @@ __global__ void __launch_bounds__(kThreads, 1)
   int* chg_flag = misc + 23;                           // [2] reference moved, per half
   static_assert(23 + 2 <= kMiscInts, "misc ints overflow into the mbarriers");
   uint64_t* bars = reinterpret_cast<uint64_t*>(base + lay.bar_off);
-  uint64_t* full = bars;                               // [slot][blk]
-  uint64_t* empty = full + p.nslot * p.nblk;           // [slot]
+  // One TMA barrier per slot for all boxes of a page: S^T starts once the whole page has
+  // landed. Every mbarrier operation on the S^T issuer's path costs a few hundred cycles, and
+  // one barrier per page measured faster than one per 64-column box.
+  uint64_t* full = bars;                               // [slot]
+  uint64_t* empty = full + p.nslot;                    // [slot]
   uint64_t* q_full = empty + p.nslot;
   uint64_t* q_empty = q_full + 1;
   uint64_t* s_full = q_empty + 1;                      // [2]
@@ -198,7 +201,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < p.nslot; ++s) {
-      for (int k = 0; k < p.nblk; ++k) mbar_init(&full[s * p.nblk + k], 1);
+      mbar_init(&full[s], 1);
       mbar_init(&empty[s], 1);
     }
     mbar_init(q_full, 1);
@@ -258,25 +261,23 @@ __global__ void __launch_bounds__(kThreads, 1)
             page = 0;
           }
           uint8_t* sbase = slots + slot * slot_bytes;
-          for (int k = 0; k < p.nblk; ++k) {
-            uint64_t* fb = &full[slot * p.nblk + k];
-            mbar_arrive_expect_tx(fb, kBlkBytes);
+          uint64_t* fb = &full[slot];
+          mbar_arrive_expect_tx(fb, uint32_t(p.nblk) * kBlkBytes);
+          for (int k = 0; k < p.nblk; ++k)
             tma_load_2d(sbase + k * kBlkBytes, &p.tm_cache, k * 64, page * kDecodeTok, fb);
-          }
           MLA_TRACE_AT(8, jj);
         }
       }
       // Drain: never leave while copies into this CTA's shared memory are in flight.
       if (pc > 0) mbar_wait_bounded(q_full, (pc - 1) & 1, 200000000ull);
       for (int j = (jj > p.nslot ? jj - p.nslot : 0); j < jj; ++j)
-        for (int k = 0; k < p.nblk; ++k)
-          mbar_wait_bounded(&full[(j % p.nslot) * p.nblk + k], (j / p.nslot) & 1, 200000000ull);
+        mbar_wait_bounded(&full[j % p.nslot], (j / p.nslot) & 1, 200000000ull);
     }
     __syncwarp();
   } else if (warp == 1) {
     // ================================ UMMA issuer for S^T ================================
-    // S^T(j) is issued one 64-column block at a time as the blocks land. The PV products
-    // are issued by the softmax warps themselves, the moment P(j) is written.
+    // S^T(j) is issued once the whole page has landed. The PV products are issued by the
+    // softmax warps themselves, the moment P(j) is written.
     if (has_work && elect_one()) {
       const uint32_t idesc_s = make_idesc_bf16(64, NCOL, 0, 0);
       const uint64_t a0 = make_sdesc(smem_u32(slots), 16, 1024, kSw128);
@@ -294,10 +295,10 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (jj >= 2 && !mbar_wait(&s_free[sb], ((jj - 2) >> 1) & 1, wc)) { ok = false; break; }
           tc_fence_after();
           const uint32_t soff = slot * slot_bytes;
+          if (!mbar_wait(&full[slot], (jj / p.nslot) & 1, wc)) { ok = false; break; }
+          tc_fence_after();
+          MLA_TRACE_AT(9, jj);
           for (int k = 0; k < p.nblk; ++k) {
-            if (!mbar_wait(&full[slot * p.nblk + k], (jj / p.nslot) & 1, wc)) { ok = false; break; }
-            tc_fence_after();
-            if (k == 0) MLA_TRACE_AT(9, jj);
             const int rem = p.D - k * 64;
             const int nkk = rem >= 64 ? 4 : (rem + 15) / 16;
             for (int kk = 0; kk < nkk; ++kk) {
@@ -306,7 +307,6 @@ __global__ void __launch_bounds__(kThreads, 1)
               umma_bf16(tmem + sb * NCOL, ad, bd, idesc_s, (k | kk) != 0 ? 1u : 0u);
             }
           }
-          if (!ok) break;
           MLA_TRACE_AT(1, jj);
           umma_commit(&s_full[sb]);
           MLA_TRACE_AT(2, jj);
