@@ -238,6 +238,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (blockIdx.x == 0) *p.range_len = per;
       UnitWalk w{sched[0], sched[1]};
       int jj = 0, pc = 0;
+      SlotRing ring(p.nslot);
       bool ok = true;
       for (; ok && w.s < r1; w.s += w.tiles, ++w.b, ++pc) {
         w.load(p, cg);
@@ -248,9 +249,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int k = 0; k < p.nblk; ++k)
           tma_load_3d(q_smem + k * kQBlk, &p.tm_q, k * 64, cg * NCOL, w.b, q_full);
         const int32_t* bt = p.block_table + int64_t(w.b) * p.max_pages;
-        for (int t = tb; t < te; ++t, ++jj) {
-          const int slot = jj % p.nslot;
-          if (jj >= p.nslot && !mbar_wait(&empty[slot], ((jj / p.nslot) - 1) & 1, wc)) {
+        for (int t = tb; t < te; ++t, ++jj, ring.next()) {
+          const int slot = ring.slot;
+          if (jj >= p.nslot && !mbar_wait(&empty[slot], (ring.round - 1) & 1, wc)) {
             ok = false;
             break;
           }
@@ -284,18 +285,19 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint64_t b0 = make_sdesc(smem_u32(q_smem), 16, 1024, kSw128);
       UnitWalk w{sched[0], sched[1]};
       int jj = 0, pc = 0;
+      SlotRing ring(p.nslot);
       bool ok = true;
       for (; ok && w.s < r1; w.s += w.tiles, ++w.b, ++pc) {
         w.load(p, cg);
         const int tb = max(w.s, r0), te = min(w.s + w.tiles, r1);
         if (!mbar_wait(q_full, pc & 1, wc)) { ok = false; break; }
-        for (int t = tb; ok && t < te; ++t, ++jj) {
-          const int slot = jj % p.nslot;
+        for (int t = tb; ok && t < te; ++t, ++jj, ring.next()) {
+          const int slot = ring.slot;
           const int sb = jj & 1;
           if (jj >= 2 && !mbar_wait(&s_free[sb], ((jj - 2) >> 1) & 1, wc)) { ok = false; break; }
           tc_fence_after();
           const uint32_t soff = slot * slot_bytes;
-          if (!mbar_wait(&full[slot], (jj / p.nslot) & 1, wc)) { ok = false; break; }
+          if (!mbar_wait(&full[slot], ring.round & 1, wc)) { ok = false; break; }
           tc_fence_after();
           MLA_TRACE_AT(9, jj);
           for (int k = 0; k < p.nblk; ++k) {
@@ -333,6 +335,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 
     UnitWalk w{sched[0], sched[1]};
     int jj = 0;
+    SlotRing ring(p.nslot), pring(p.npt);
     for (; w.s < r1; w.s += w.tiles, ++w.b) {
       w.load(p, cg);
       const int tb = max(w.s, r0), te = min(w.s + w.tiles, r1);
@@ -344,7 +347,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         m[j] = kRefInit;
         l[j] = 0.0f;
       }
-      for (int t = tb; t < te; ++t, ++jj) {
+      for (int t = tb; t < te; ++t, ++jj, ring.next(), pring.next()) {
         const int sb = jj & 1;
         const uint32_t s_addr = tmem + lane_base + sb * NCOL;
         const bool got = __all_sync(0xffffffffu, mbar_wait(&s_full[sb], (jj >> 1) & 1, wc));
@@ -460,8 +463,8 @@ __global__ void __launch_bounds__(kThreads, 1)
           l[j + 1] += p1;
           packed[j / 2] = cvt_bf16x2(p0, p1);
         }
-        const int slot = jj % p.nslot;
-        const int pbuf = jj % p.npt;
+        const int slot = ring.slot;
+        const int pbuf = pring.slot;
         {
           uint8_t* buf = pt + pbuf * kPtBytes;
           constexpr uint32_t kRowBytes = NCOL * 2;

@@ -317,15 +317,16 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (blockIdx.x == 0) *p.range_len = per;
       UnitWalk w{sched[0], sched[1]};
       int jj = 0;
+      SlotRing ring(p.nslot);
       bool ok = true;
       for (; ok && w.s < r1; w.s += w.tiles, ++w.b) {
         w.load(p, cg);
         if (rank == 0) p.unit_start[w.u] = w.s;   // same value from every cluster
         const int tb = max(w.s, r0), te = min(w.s + w.tiles, r1);
         const int32_t* bt = p.block_table + int64_t(w.b) * p.max_pages;
-        for (int t = tb; t < te; ++t, ++jj) {
-          const int slot = jj % p.nslot;
-          if (jj >= p.nslot && !mbar_wait(&empty[slot], ((jj / p.nslot) - 1) & 1, wc)) {
+        for (int t = tb; t < te; ++t, ++jj, ring.next()) {
+          const int slot = ring.slot;
+          if (jj >= p.nslot && !mbar_wait(&empty[slot], (ring.round - 1) & 1, wc)) {
             ok = false;
             break;
           }
@@ -362,17 +363,18 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint64_t aq0 = make_sdesc(smem_u32(qrope), 16, 8 * rh * 2, rope_swizzle(rh));
       UnitWalk w{sched[0], sched[1]};
       int jj = 0, pc = 0;
+      SlotRing ring(p.nslot);
       bool ok = true;
       for (; ok && w.s < r1; w.s += w.tiles, ++w.b, ++pc) {
         w.load(p, cg);
         const int tb = max(w.s, r0), te = min(w.s + w.tiles, r1);
         if (!mbar_wait(q_full, pc & 1, wc)) { ok = false; break; }
         tc_fence_after();
-        for (int t = tb; ok && t < te; ++t, ++jj) {
-          const int slot = jj % p.nslot;
+        for (int t = tb; ok && t < te; ++t, ++jj, ring.next()) {
+          const int slot = ring.slot;
           const int sb = jj & 1;
           // every block of the tile landed, then the S buffer free
-          if (!mbar_wait(&full[slot], (jj / p.nslot) & 1, wc)) { ok = false; break; }
+          if (!mbar_wait(&full[slot], ring.round & 1, wc)) { ok = false; break; }
           MLA_PTRACE(1, jj);
           if (jj >= 2 && (!mbar_wait(&s_free[sb], ((jj - 2) >> 1) & 1, wc) ||
                           !mbar_wait(&pv_done[sb], ((jj - 2) >> 1) & 1, wc))) {
@@ -406,25 +408,26 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint64_t pb0 = make_sdesc(smem_u32(slots), kBlk, 1024, kSw128);
       UnitWalk w{sched[0], sched[1]};
       int jj = 0;
+      SlotRing ring(p.nslot);
       bool ok = true;
       for (; ok && w.s < r1; w.s += w.tiles, ++w.b) {
         w.load(p, cg);
         const int tb = max(w.s, r0), te = min(w.s + w.tiles, r1);
-        for (int t = tb; t < te; ++t, ++jj) {
+        for (int t = tb; t < te; ++t, ++jj, ring.next()) {
           const int sb = jj & 1;
           if (!mbar_wait(&p_full[sb], (jj >> 1) & 1, wc)) { ok = false; break; }
           tc_fence_after();
           // the first tile of a piece overwrites O: the previous piece's epilogue read O
           // before its warps arrived on p_full for this tile
           const bool first = (t == tb);
-          const uint32_t soff = (jj % p.nslot) * lay.slot_bytes;
+          const uint32_t soff = ring.slot * lay.slot_bytes;
 #pragma unroll
           for (int kk = 0; kk < 4; ++kk)
             umma_bf16_ts(tmem + kColO, tmem + kColS + 64 * sb + kk * 8,
                          pb0 + ((soff + kk * 2048) >> 4), idesc_o,
                          (!first || kk > 0) ? 1u : 0u);
           umma_commit(&pv_done[sb]);
-          umma_commit(&empty[jj % p.nslot]);
+          umma_commit(&empty[ring.slot]);
           MLA_PTRACE(8, jj);
         }
       }
@@ -496,15 +499,16 @@ __global__ void __launch_bounds__(kThreads, 1)
       UnitWalk w{sched[0], sched[1]};
       w.load(p, cg);
       int jj = 0;
+      SlotRing ring(p.nslot);
       while (true) {
         const int tb = max(w.s, r0), te = min(w.s + w.tiles, r1);
         const int L = w.L;
         // last position row n sees (causal: L - q + i); rows past q*H see L - 1
         const int lim = min(L - 1, p.causal ? L - p.q_len + qi : L - 1);
         float mref = kRefInit, l = 0.0f, lt = 0.0f;   // the same in both threads of a row
-        for (int t = tb; t < te; ++t, ++jj) {
+        for (int t = tb; t < te; ++t, ++jj, ring.next()) {
           const int sb = jj & 1;                 // S buffer and partial buffer of this tile
-          const int slot = jj % p.nslot;
+          const int slot = ring.slot;
           const int tile_pos0 = (t - w.s) * kDecodeTok;
           const int pos0 = tile_pos0 + qt * kHalfTok;   // first token of this thread's half
           // ---- own partial scores ----

@@ -23,6 +23,20 @@ MLA_DEVICE int valid_len(const DecodeParams& p, int L) {
   return ok ? L : 0;
 }
 
+// Position of tile number j in a ring of n cache slots, kept incrementally: slot = j % n
+// and round = j / n without a division on the issue paths (an integer division by a
+// runtime value there measurably lengthens the per-tile loop).
+struct SlotRing {
+  int n, slot, round;
+  MLA_DEVICE explicit SlotRing(int nslot) : n(nslot), slot(0), round(0) {}
+  MLA_DEVICE void next() {
+    if (++slot == n) {
+      slot = 0;
+      ++round;
+    }
+  }
+};
+
 // The walk over the sequences a range touches; every role runs the same walk.
 struct UnitWalk {
   int b, s;       // sequence and the index of its first tile in this row block's tile space
