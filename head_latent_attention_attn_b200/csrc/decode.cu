@@ -251,12 +251,13 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int32_t* bt = p.block_table + int64_t(w.b) * p.max_pages;
         for (int t = tb; t < te; ++t, ++jj, ring.next()) {
           const int slot = ring.slot;
+          // the page id is read before the wait, so its round trip overlaps it
+          int32_t page = bt[t - w.s];
           if (jj >= p.nslot && !mbar_wait(&empty[slot], (ring.round - 1) & 1, wc)) {
             ok = false;
             break;
           }
           MLA_TRACE_AT(0, jj);
-          int32_t page = bt[t - w.s];
           if (page < 0 || page >= p.num_pages) {
             if (p.dev_error) atomicOr(p.dev_error, MLA_DEVERR_BOUNDS);
             page = 0;
