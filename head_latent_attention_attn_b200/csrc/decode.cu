@@ -284,6 +284,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint32_t idesc_s = make_idesc_bf16(64, NCOL, 0, 0);
       const uint64_t a0 = make_sdesc(smem_u32(slots), 16, 1024, kSw128);
       const uint64_t b0 = make_sdesc(smem_u32(q_smem), 16, 1024, kSw128);
+      const int nk16 = (p.D + 15) / 16;              // K steps over the row width
       UnitWalk w{sched[0], sched[1]};
       int jj = 0, pc = 0;
       SlotRing ring(p.nslot);
@@ -301,13 +302,17 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (!mbar_wait(&full[slot], ring.round & 1, wc)) { ok = false; break; }
           tc_fence_after();
           MLA_TRACE_AT(9, jj);
-          for (int k = 0; k < p.nblk; ++k) {
-            const int rem = p.D - k * 64;
-            const int nkk = rem >= 64 ? 4 : (rem + 15) / 16;
-            for (int kk = 0; kk < nkk; ++kk) {
-              const uint64_t ad = a0 + ((soff + k * kBlkBytes + kk * 32) >> 4);
-              const uint64_t bd = b0 + ((k * kQBlk + kk * 32) >> 4);
-              umma_bf16(tmem + sb * NCOL, ad, bd, idesc_s, (k | kk) != 0 ? 1u : 0u);
+          // K steps of 16 columns over the row width; the descriptors step 32 bytes within
+          // a 64-column block and to the next block's start after its fourth step
+          {
+            const uint32_t dS = tmem + sb * NCOL;
+            uint64_t ad = a0 + (soff >> 4), bd = b0;
+            umma_bf16(dS, ad, bd, idesc_s, 0u);
+            for (int i = 1; i < nk16; ++i) {
+              const bool next_blk = (i & 3) == 0;
+              ad += next_blk ? uint64_t((kBlkBytes - 96) >> 4) : uint64_t(2);
+              bd += next_blk ? uint64_t((kQBlk - 96) >> 4) : uint64_t(2);
+              umma_bf16(dS, ad, bd, idesc_s, 1u);
             }
           }
           MLA_TRACE_AT(1, jj);
