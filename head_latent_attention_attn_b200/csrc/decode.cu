@@ -504,13 +504,20 @@ __global__ void __launch_bounds__(kThreads, 1)
           const bool first = (t == tb);
           const uint32_t soff = slot * slot_bytes;
           const uint32_t poff = pbuf * kPtBytes;
-          // K-step outer, latent chunk inner: consecutive MMAs feed different accumulators
+          // K-step outer, latent chunk inner: consecutive MMAs feed different accumulators;
+          // descriptors stepped (16 tokens = 2 KB of C^T, 16 rows of P^T; 128 latent = 2 blocks)
+          {
+            const uint64_t ad0 = pa0 + (soff >> 4);
+            uint64_t bd = pb0 + (poff >> 4);
 #pragma unroll
-          for (int kk = 0; kk < 4; ++kk) {
-            const uint64_t bd = pb0 + ((poff + kk * 16 * NCOL * 2) >> 4);
-            for (int c = 0; c < p.nch; ++c) {
-              const uint64_t ad = pa0 + ((soff + 2 * c * kBlkBytes + kk * 2048) >> 4);
-              umma_bf16(tmem + (2 + c) * NCOL, ad, bd, idesc_o, (!first || kk > 0) ? 1u : 0u);
+            for (int kk = 0; kk < 4; ++kk) {
+              uint64_t ad = ad0 + uint64_t(kk * (2048 >> 4));
+              const uint32_t acc = (!first || kk > 0) ? 1u : 0u;
+              for (int c = 0; c < p.nch; ++c) {
+                umma_bf16(tmem + (2 + c) * NCOL, ad, bd, idesc_o, acc);
+                ad += uint64_t((2 * kBlkBytes) >> 4);
+              }
+              bd += uint64_t((16 * NCOL * 2) >> 4);
             }
           }
           umma_commit(&pv_done[jj & 1]);

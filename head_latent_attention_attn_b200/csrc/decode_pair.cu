@@ -386,15 +386,18 @@ __global__ void __launch_bounds__(kThreads, 1)
           tc_fence_after();
           const uint32_t dS = tmem + kColS + 64 * sb;
           const uint32_t soff = slot * lay.slot_bytes;
-          for (int k = 0; k < lb; ++k) {
-#pragma unroll
-            for (int kk = 0; kk < 4; ++kk)
-              umma_bf16_ts(dS, tmem + kColQ + (k * 4 + kk) * 8,
-                           b0 + ((soff + k * kBlk + kk * 32) >> 4), idesc_s,
-                           (k | kk) != 0 ? 1u : 0u);
+          // latent K steps: A = Q from TMEM (8 columns per step), B steps 32 bytes within a
+          // 64-column block and to the next block after its fourth step; then the rotary ones
+          {
+            uint64_t bd = b0 + (soff >> 4);
+            umma_bf16_ts(dS, tmem + kColQ, bd, idesc_s, 0u);
+            for (int i = 1; i < 4 * lb; ++i) {
+              bd += (i & 3) == 0 ? uint64_t((kBlk - 96) >> 4) : uint64_t(2);
+              umma_bf16_ts(dS, tmem + kColQ + i * 8, bd, idesc_s, 1u);
+            }
+            uint64_t ad = aq0, rd = br0 + (soff >> 4);
+            for (int kk = 0; kk < rh / 16; ++kk, ad += 2, rd += 2) umma_bf16(dS, ad, rd, idesc_s, 1u);
           }
-          for (int kk = 0; kk < rh / 16; ++kk)
-            umma_bf16(dS, aq0 + ((kk * 32) >> 4), br0 + ((soff + kk * 32) >> 4), idesc_s, 1u);
           umma_commit(&s_full[sb]);
           MLA_PTRACE(2, jj);
         }
