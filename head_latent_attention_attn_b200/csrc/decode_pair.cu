@@ -18,13 +18,12 @@
 // a 15-bit mantissa, relative error <= 2^-16, 4 values in 3 words) and 8.5 KB of weights,
 // and each CTA evaluates 64 x 64 exponentials instead of 128 x 64.
 //
-// TMEM (512 columns): O [0, r/2), two S buffers [256, 320) and [320, 384), the latent half
-// of Q [384, 384 + r/4) (bf16 pairs). The rotary half of Q is a shared-memory operand (the
-// S UMMA takes A from TMEM for the latent K steps and from shared memory for the rotary
-// ones), which frees the columns for the second S buffer. P of a tile (bf16 pairs) is
-// written over the first 32 columns of that tile's S buffer once its scores have been
-// read, so S of tile j + 2 waits for PV of tile j, while S of tile j + 1 is computed as soon
-// as its page has landed: the score exchange of one tile overlaps the softmax of the other.
+// TMEM (512 columns): O [0, r/2), two S buffers [256, 320) and [320, 384), two P buffers
+// (bf16 pairs) [384, 416) and [416, 448), and the first 128 latent elements of Q [448, 512)
+// (bf16 pairs). The rest of Q's latent half and its rotary half are shared-memory UMMA
+// operands (the S UMMA takes A from TMEM for the first K steps and from shared memory for
+// the others). With P in its own buffers, S of tile j + 2 waits only until the scores of
+// tile j have been read, not for PV of tile j.
 //
 // Roles (352 threads): warp 0 TMA producer, warp 1 S issuer and TMEM owner, warp 2 PV
 // issuer, warps 3-10 the rows. TMEM lane n holds row n and a warp reaches only the 32 lanes
@@ -78,7 +77,8 @@ constexpr uint32_t kXsWarpBytes = 32u * kPackWords * 4;        // one owner warp
 constexpr uint32_t kXsBytes = 4 * kXsWarpBytes;                // partials of 64 rows, 12 KB
 constexpr uint32_t kXpRowsBytes = 64u * kDecodeTok * 2;        // P of 64 rows (bf16), 8 KB
 constexpr uint32_t kXpBytes = kXpRowsBytes + 64u * 8;          // + (alpha, sum) per row
-constexpr uint32_t kColO = 0, kColS = 256, kColQ = 384, kTmemCols = 512;
+constexpr uint32_t kColO = 0, kColS = 256, kColP = 384, kColQ = 448, kTmemCols = 512;
+constexpr int kQTmem = 128;   // latent elements of each Q row held in TMEM (the rest: smem)
 constexpr float kLazyThreshold = 8.0f;   // log2 units; see decode.cu
 constexpr float kRefInit = -3.0e38f;
 constexpr float kLn2 = 0.69314718055994530942f;
@@ -86,7 +86,7 @@ constexpr float kLn2 = 0.69314718055994530942f;
 constexpr int kMiscInts = 32;
 
 struct PairLayout {
-  uint32_t slot_bytes, rope_off, qrope_off, xs_off, xp_off, misc_off, bar_off, total;
+  uint32_t slot_bytes, rope_off, qrope_off, qlat_off, xs_off, xp_off, misc_off, bar_off, total;
 };
 
 __host__ __device__ inline uint32_t round_up_p(uint32_t x, uint32_t a) {
@@ -103,6 +103,8 @@ __host__ __device__ inline PairLayout pair_layout(int r, int rope_half, int nslo
   uint32_t off = uint32_t(nslot) * L.slot_bytes;
   L.qrope_off = off;                              // rotary half of the 128 Q rows (swizzled)
   off += round_up_p(uint32_t(kPairRows) * rope_half * 2, 1024);
+  L.qlat_off = off;                               // latent Q past kQTmem, 64-column blocks
+  off += uint32_t(kPairRows) * uint32_t(r / 2 > kQTmem ? r / 2 - kQTmem : 0) * 2;
   L.xs_off = off;                                 // partner's partials for the own rows (x2)
   off += 2 * kXsBytes;
   L.xp_off = off;                                 // partner's P for its rows
@@ -143,6 +145,20 @@ MLA_DEVICE uint32_t swizzled_chunk(int row, int c, int pitch) {
   const uint32_t lin = uint32_t(row) * uint32_t(pitch) + uint32_t(c) * 16u;
   const uint32_t mask = uint32_t(pitch / 16 - 1);
   return lin ^ (((lin >> 7) & mask) << 4);
+}
+
+// Latent Q elements [e, e + 16) of row n (e a multiple of 16, counted from the first element
+// past the TMEM part) into the shared-memory A operand: 64-element K-major blocks of 128 rows,
+// 128-byte swizzle (the layout the S UMMA's descriptor reads).
+MLA_DEVICE void store_qlat(uint8_t* qlat, int n, int e, const uint32_t* v) {
+#pragma unroll
+  for (int i = 0; i < 2; ++i) {
+    const int el = e + 8 * i;
+    const uint32_t off = uint32_t(el / 64) * (kPairRows * 128) + uint32_t(n) * 128 +
+                         ((uint32_t((el % 64) / 8) ^ uint32_t(n & 7)) << 4);
+    *reinterpret_cast<uint4*>(qlat + off) =
+        make_uint4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
+  }
 }
 
 MLA_DEVICE void st_async_v2(uint32_t remote_addr, uint2 v, uint32_t remote_bar) {
@@ -233,6 +249,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   const PairLayout lay = pair_layout(r, rh, p.nslot);
   uint8_t* slots = base;
   uint8_t* qrope = base + lay.qrope_off;
+  uint8_t* qlat = base + lay.qlat_off;
   uint8_t* xs = base + lay.xs_off;
   uint8_t* xp = base + lay.xp_off;
   int* misc = reinterpret_cast<int*>(base + lay.misc_off);
@@ -354,14 +371,16 @@ __global__ void __launch_bounds__(kThreads, 1)
     __syncwarp();
   } else if (warp == 1) {
     // ============================ UMMA issuer for the partial S ==========================
-    // S of tile j goes to buffer j % 2: it waits for its page, for the readers of tile j - 2
-    // and for PV of tile j - 2 (whose P was written over that buffer).
+    // S of tile j goes to buffer j % 2: it waits for its page and for the readers of tile
+    // j - 2's scores (P has buffers of its own).
     if (has_work && elect_one()) {
       const uint32_t idesc_s = make_idesc_bf16(128, kDecodeTok, 0, 0);
       const uint64_t b0 = make_sdesc(smem_u32(slots), 16, 1024, kSw128);
       const uint64_t br0 =
           make_sdesc(smem_u32(slots + lay.rope_off), 16, 8 * rh * 2, rope_swizzle(rh));
       const uint64_t aq0 = make_sdesc(smem_u32(qrope), 16, 8 * rh * 2, rope_swizzle(rh));
+      const uint64_t aql0 = make_sdesc(smem_u32(qlat), 16, 1024, kSw128);
+      const int kt = 4 * (min(rhalf, kQTmem) / 64);   // latent K steps with A in TMEM
       UnitWalk w{sched[0], sched[1]};
       int jj = 0, pc = 0;
       SlotRing ring(p.nslot);
@@ -377,8 +396,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           // every block of the tile landed, then the S buffer free
           if (!mbar_wait(&full[slot], ring.round & 1, wc)) { ok = false; break; }
           MLA_PTRACE(1, jj);
-          if (jj >= 2 && (!mbar_wait(&s_free[sb], ((jj - 2) >> 1) & 1, wc) ||
-                          !mbar_wait(&pv_done[sb], ((jj - 2) >> 1) & 1, wc))) {
+          if (jj >= 2 && !mbar_wait(&s_free[sb], ((jj - 2) >> 1) & 1, wc)) {
             ok = false;
             break;
           }
@@ -386,14 +404,21 @@ __global__ void __launch_bounds__(kThreads, 1)
           tc_fence_after();
           const uint32_t dS = tmem + kColS + 64 * sb;
           const uint32_t soff = slot * lay.slot_bytes;
-          // latent K steps: A = Q from TMEM (8 columns per step), B steps 32 bytes within a
-          // 64-column block and to the next block after its fourth step; then the rotary ones
+          // latent K steps: A = Q from TMEM (8 columns per step) for the first kt steps and
+          // from shared memory after them; B steps 32 bytes within a 64-column block and to
+          // the next block after its fourth step; then the rotary steps
           {
             uint64_t bd = b0 + (soff >> 4);
             umma_bf16_ts(dS, tmem + kColQ, bd, idesc_s, 0u);
-            for (int i = 1; i < 4 * lb; ++i) {
+            for (int i = 1; i < kt; ++i) {
               bd += (i & 3) == 0 ? uint64_t((kBlk - 96) >> 4) : uint64_t(2);
               umma_bf16_ts(dS, tmem + kColQ + i * 8, bd, idesc_s, 1u);
+            }
+            uint64_t qd = aql0;
+            for (int i = kt; i < 4 * lb; ++i) {
+              bd += (i & 3) == 0 ? uint64_t((kBlk - 96) >> 4) : uint64_t(2);
+              if (i > kt) qd += (i & 3) == 0 ? uint64_t(((kPairRows * 128) - 96) >> 4) : uint64_t(2);
+              umma_bf16(dS, qd, bd, idesc_s, 1u);
             }
             uint64_t ad = aq0, rd = br0 + (soff >> 4);
             for (int kk = 0; kk < rh / 16; ++kk, ad += 2, rd += 2) umma_bf16(dS, ad, rd, idesc_s, 1u);
@@ -427,7 +452,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           const uint32_t soff = ring.slot * lay.slot_bytes;
 #pragma unroll
           for (int kk = 0; kk < 4; ++kk)
-            umma_bf16_ts(tmem + kColO, tmem + kColS + 64 * sb + kk * 8,
+            umma_bf16_ts(tmem + kColO, tmem + kColP + 32 * sb + kk * 8,
                          pb0 + ((soff + kk * 2048) >> 4), idesc_o,
                          (!first || kk > 0) ? 1u : 0u);
           umma_commit(&pv_done[sb]);
@@ -485,7 +510,8 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
             for (int i = 0; i < 8; ++i) v[i] = 0u;
           }
-          tm_st_x8_s8(trow + kColQ + c0 / 2, v);
+          if (c0 < kQTmem) tm_st_x8_s8(trow + kColQ + c0 / 2, v);
+          else store_qlat(qlat, n, c0 + 16 * qt - kQTmem, v);
         }
         for (int c = qt; c < rh / 8; c += 2) {
           const uint4 v = row_ok ? *reinterpret_cast<const uint4*>(q + r + int(rank) * rh + 8 * c)
@@ -609,7 +635,12 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
           l += sa + sc;
           lt = l + __shfl_xor_sync(0xffffffffu, l, 16);
-          tm_st_x16_s16(trow + kColS + 64 * sb, pk);
+          // this tile's P buffer held P of tile jj - 2: PV of that tile must have read it
+          if (jj >= 2) {
+            __all_sync(0xffffffffu, mbar_wait(&pv_done[sb], ((jj - 2) >> 1) & 1, wc));
+            tc_fence_after();
+          }
+          tm_st_x16_s16(trow + kColP + 32 * sb, pk);
           // ---- the same weights, the rescale factor and the running sum to the partner ----
           const bool pfree =
               __all_sync(0xffffffffu, jj == 0 || mbar_wait_cluster(xp_free, (jj - 1) & 1, wc));
@@ -727,7 +758,8 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
             for (int i = 0; i < 8; ++i) v[i] = 0u;
           }
-          tmem_st8(tq + kColQ + c0 / 2, v);
+          if (c0 < kQTmem) tmem_st8(tq + kColQ + c0 / 2, v);
+          else store_qlat(qlat, n, c0 - kQTmem, v);
         }
         for (int c = 0; c < rh / 8; ++c) {
           const uint4 v = row_ok ? *reinterpret_cast<const uint4*>(q + r + int(rank) * rh + 8 * c)
@@ -842,7 +874,11 @@ __global__ void __launch_bounds__(kThreads, 1)
               }
             }
           }
-          tmem_st32(tq + kColS + 64 * sb, pk);
+          if (jj >= 2) {
+            __all_sync(0xffffffffu, mbar_wait(&pv_done[sb], ((jj - 2) >> 1) & 1, wc));
+            tc_fence_after();
+          }
+          tmem_st32(tq + kColP + 32 * sb, pk);
           tmem_wait_st();
           tc_fence_before();
           __syncwarp();
