@@ -10,7 +10,7 @@
 // every Q row, and computes the partial scores S_k over its half of the row width. Each
 // page crosses HBM once per cluster.
 //
-// The softmax is split by rows. CTA k owns rows [64k, 64k + 64): it receives the partner's
+// The softmax is split by rows. CTA k owns 64 of the 128 rows: it receives the partner's
 // partial scores for those rows only, adds them to its own, runs the online softmax and
 // writes P for its rows into its TMEM; it also sends those weights (bf16), with the row's
 // rescale factor and running sum, to the partner, whose O half needs P for all 128 rows.
@@ -25,17 +25,17 @@
 // the others). With P in its own buffers, S of tile j + 2 waits only until the scores of
 // tile j have been read, not for PV of tile j.
 //
-// Roles (352 threads): warp 0 TMA producer, warp 1 S issuer and TMEM owner, warp 2 PV
-// issuer, warps 3-10 the rows. TMEM lane n holds row n and a warp reaches only the 32 lanes
-// of its sub-partition (warp % 4), so the rows of CTA k are the lanes of sub-partitions 2k
-// and 2k + 1:
-//   owners    (4 warps on the own sub-partitions; 16x32bx2 accesses, 16 rows per warp,
-//              lanes i and i + 16 take tokens 0-31 and 32-63 of row i): combine the two
-//              partials, softmax, P, the epilogue of the own rows;
-//   senders   (one warp per partner sub-partition, one row per lane): read the partner
-//              rows' partial scores and send them;
-//   receivers (one warp per partner sub-partition): take the partner's P and rescale
-//              factors for its rows into TMEM, the epilogue of those rows.
+// Roles (480 threads): warp 0 TMA producer, warp 1 S issuer and TMEM owner, warp 2 PV
+// issuer, warps 3-14 the rows. TMEM lane n holds row n and a warp reaches only the 32 lanes
+// of its sub-partition (warp % 4). CTA k owns the rows on lanes 16k..16k+15 of every
+// sub-partition, so each of the three row roles has one warp on every SM sub-partition
+// (its issue slots and MUFU units). With 16x32bx2 TMEM accesses a warp covers 16 lanes,
+// two threads per row (lanes i and i + 16: tokens 0-31 and 32-63):
+//   owners    (warps 3-6, this CTA's rows): combine the two partials, softmax, P, the
+//              epilogue and lse of the own rows;
+//   senders   (warps 7-10, the partner's rows): read their partial scores and send them;
+//   receivers (warps 11-14, the partner's rows): take the partner's P and rescale factors
+//              for those rows into TMEM, and their epilogue.
 #include <math.h>
 
 #include "decode_sched.cuh"
@@ -68,8 +68,8 @@ __device__ unsigned long long g_mla_pair_trace[kPairTraceEvents * kPairTraceTile
 namespace {
 
 constexpr int kPvWarp = 2;
-constexpr int kRowWarp0 = 3;                                   // first of the 8 row warps
-constexpr int kThreads = 32 * (kRowWarp0 + 8);
+constexpr int kRowWarp0 = 3;                                   // first of the 12 row warps
+constexpr int kThreads = 32 * (kRowWarp0 + 12);
 constexpr int kHalfTok = kDecodeTok / 2;                       // tokens per owner thread
 constexpr uint32_t kBlk = kDecodeTok * 128;                    // 64 x 64 bf16 block, 8 KB
 constexpr int kPackWords = kHalfTok * 3 / 4;                   // 24-bit values of a half row
@@ -289,17 +289,17 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&full[s], 1);
       mbar_init(&empty[s], 1);
     }
-    mbar_init(q_full, 6);                              // 4 owner + 2 sender warps
+    mbar_init(q_full, 8);                              // 4 owner + 4 sender warps
     for (int i = 0; i < 2; ++i) {
       mbar_init(&s_full[i], 1);
-      mbar_init(&s_free[i], 6);                        // 4 owner + 2 sender warps
+      mbar_init(&s_free[i], 8);                        // 4 owner + 4 sender warps
       mbar_init(&pv_done[i], 1);
-      mbar_init(&p_full[i], 6);                        // 4 owner + 2 receiver warps
+      mbar_init(&p_full[i], 8);                        // 4 owner + 4 receiver warps
       mbar_init(&xs_full[i], 1);
       mbar_init(&xs_free[i], 4);                       // the partner's 4 owner warps
     }
     mbar_init(xp_full, 1);
-    mbar_init(xp_free, 2);                             // the partner's 2 receiver warps
+    mbar_init(xp_free, 4);                             // the partner's 4 receiver warps
     *abort_flag = 0;
     fence_mbar_init();
     // the receive buffers expect their first messages
@@ -464,13 +464,25 @@ __global__ void __launch_bounds__(kThreads, 1)
     __syncwarp();
   } else if (has_work) {
     // ==================================== the 128 rows ====================================
-    const int wi = warp - kRowWarp0;          // 0..7
+    // Every row warp works on 16 TMEM lanes of its sub-partition with 16x32bx2 accesses:
+    // lanes i and i + 16 of the warp share row i and take tokens 0-31 and 32-63 (or the
+    // two 16-column halves of every 32 columns of O).
     const int sp = warp & 3;                  // TMEM sub-partition this warp reaches
-    const int hl = wi >> 2;                   // each sub-partition has two row warps
-    const bool owner = (sp >> 1) == int(rank);
+    const int role = (warp - kRowWarp0) >> 2; // 0 owner, 1 sender, 2 receiver
+    const int qt = lane >> 4;                 // token half of this thread
+    const int i16 = lane & 15;
+    // owners work on this CTA's rows, senders and receivers on the partner's
+    const uint32_t grp = uint32_t(32 * sp + 16 * int(role == 0 ? rank : peer));
+    const int n = int(grp) + i16;             // query row (TMEM lane)
+    const int m = 16 * sp + i16;              // row within its CTA's block of 64
+    const uint32_t trow = tmem + (grp << 16);
+    const int row = cg * kPairRows + n;       // row (i, h) of the sequence's q*H rows
+    const bool row_ok = row < p.qH;
     const float c_log2 = p.scale_log2;
     const bool vec_out = (reinterpret_cast<uintptr_t>(p.o_latent) & 15u) == 0;
     const int rpitch = rh * 2;                // bytes per Q rotary row in shared memory
+    const bool tr = (sp == 0 && lane == 0);
+    (void)tr;
     const uint32_t xs_s = smem_u32(xs), xp_s = smem_u32(xp);
     const uint32_t xs_r = map_to_rank(xs_s, peer), xp_r = map_to_rank(xp_s, peer);
     const uint32_t xs_full_r0 = map_to_rank(smem_u32(&xs_full[0]), peer);
@@ -480,51 +492,106 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t xp_full_r = map_to_rank(smem_u32(xp_full), peer);
     const uint32_t xp_free_r = map_to_rank(smem_u32(xp_free), peer);
 
-    if (owner) {
-      // ---------------- owner: rows of this CTA, 16 per warp, two threads per row --------
-      const int ow = 2 * hl + (sp & 1);       // owner warp index (block of the partial buffer)
-      const int qt = lane >> 4;               // token half of this thread
-      const int n = 32 * sp + 16 * hl + (lane & 15);   // query row (TMEM lane)
-      const int m = n & 63;                   // row within the own block
-      const uint32_t trow = tmem + (uint32_t(32 * sp + 16 * hl) << 16);
-      const int row = cg * kPairRows + n;     // row (i, h) of the sequence's q*H rows
-      const bool row_ok = row < p.qH;
-      const int qi = row / p.num_heads;
-      const bool tr = (ow == 0 && lane == 0);
-      (void)tr;
+    // This CTA's half of Q row n: the latent half into TMEM (16-element chunks dealt
+    // alternately to the two threads of the row), the rotary half into shared memory;
+    // zero rows past q*H. Ends with this warp's arrival on q_full (owners and senders).
+    auto load_q = [&](int b) {
+      const uint16_t* q = p.q_ext + (int64_t(b) * p.qH + row) * p.D;
+      for (int c0 = 0; c0 < rhalf; c0 += 32) {
+        const uint16_t* src = q + int(rank) * rhalf + c0 + 16 * qt;
+        uint32_t v[8];
+        if (row_ok) {
+          const uint4 a = *reinterpret_cast<const uint4*>(src);
+          const uint4 bb = *reinterpret_cast<const uint4*>(src + 8);
+          v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w;
+          v[4] = bb.x; v[5] = bb.y; v[6] = bb.z; v[7] = bb.w;
+        } else {
+#pragma unroll
+          for (int k = 0; k < 8; ++k) v[k] = 0u;
+        }
+        if (c0 < kQTmem) tm_st_x8_s8(trow + kColQ + c0 / 2, v);
+        else store_qlat(qlat, n, c0 + 16 * qt - kQTmem, v);
+      }
+      for (int c = qt; c < rh / 8; c += 2) {
+        const uint4 v = row_ok ? *reinterpret_cast<const uint4*>(q + r + int(rank) * rh + 8 * c)
+                               : make_uint4(0, 0, 0, 0);
+        *reinterpret_cast<uint4*>(qrope + swizzled_chunk(n, c, rpitch)) = v;
+      }
+      tmem_wait_st();
+      fence_proxy_async_smem();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(q_full);
+    };
 
-      // This CTA's half of Q row n: latent half into TMEM (16-element chunks dealt
-      // alternately to the two threads of the row), rotary half into shared memory; zero
-      // rows past q*H. Ends with this warp's arrival on q_full.
-      auto load_q = [&](int b) {
-        const uint16_t* q = p.q_ext + (int64_t(b) * p.qH + row) * p.D;
-        for (int c0 = 0; c0 < rhalf; c0 += 32) {
-          const uint16_t* src = q + int(rank) * rhalf + c0 + 16 * qt;
-          uint32_t v[8];
-          if (row_ok) {
-            const uint4 a = *reinterpret_cast<const uint4*>(src);
-            const uint4 bb = *reinterpret_cast<const uint4*>(src + 8);
-            v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w;
-            v[4] = bb.x; v[5] = bb.y; v[6] = bb.z; v[7] = bb.w;
+    // O rows of this warp times alpha (16 of every 32 columns per thread), once PV(jj - 1)
+    // has landed in O.
+    auto rescale_o = [&](int jj, float alpha) {
+      const bool pv_ok =
+          __all_sync(0xffffffffu, mbar_wait(&pv_done[(jj - 1) & 1], ((jj - 1) >> 1) & 1, wc));
+      tc_fence_after();
+      if (!pv_ok) return;
+      for (int c0 = 0; c0 < rhalf; c0 += 32) {
+        float o[16];
+        tm_ld_x16_s16(trow + kColO + c0, o);
+        tmem_wait_ld();
+#pragma unroll
+        for (int c = 0; c < 16; ++c) o[c] *= alpha;
+        tm_st_x16_s16(trow + kColO + c0, reinterpret_cast<const uint32_t*>(o));
+      }
+    };
+
+    // O rows of this warp divided by the row sum lt, to the outputs of piece (w, tb, te)
+    // whose last tile is jl: bf16 o_latent when the piece is the whole unit, else fp32 part_o.
+    auto write_o = [&](const UnitWalk& w, int tb, int te, int jl, float lt, bool* aborted_out) {
+      const bool fin = __all_sync(0xffffffffu, mbar_wait(&pv_done[jl & 1], (jl >> 1) & 1, wc));
+      tc_fence_after();
+      const bool aborted = __any_sync(0xffffffffu, !fin || *abort_flag != 0);
+      *aborted_out = aborted;
+      const bool whole = (tb == w.s) && (te == w.s + w.tiles);
+      const int64_t grow = int64_t(w.b) * p.qH + row;   // global (b, i, h) row
+      const int pslot = piece_slot(vc, w.s, per, p.col_groups, cg);
+      const float inv = (lt > 0.0f && !aborted) ? 1.0f / lt : 0.0f;
+      const int64_t lat0 = int64_t(rank) * rhalf + 16 * qt;   // this thread's 16 of every 32
+      for (int c0 = 0; c0 < rhalf; c0 += 32) {
+        float o[16];
+        if (!aborted) {
+          tm_ld_x16_s16(trow + kColO + c0, o);
+          tmem_wait_ld();
+        } else {
+#pragma unroll
+          for (int c = 0; c < 16; ++c) o[c] = 0.0f;
+        }
+        if (!row_ok) {
+          // padding row past q*H: nothing to write
+        } else if (whole) {
+          uint16_t* dst = p.o_latent + grow * r + lat0 + c0;
+          if (vec_out) {
+#pragma unroll
+            for (int c = 0; c < 16; c += 8)
+              *reinterpret_cast<uint4*>(dst + c) =
+                  make_uint4(cvt_bf16x2(o[c] * inv, o[c + 1] * inv),
+                             cvt_bf16x2(o[c + 2] * inv, o[c + 3] * inv),
+                             cvt_bf16x2(o[c + 4] * inv, o[c + 5] * inv),
+                             cvt_bf16x2(o[c + 6] * inv, o[c + 7] * inv));
           } else {
 #pragma unroll
-            for (int i = 0; i < 8; ++i) v[i] = 0u;
+            for (int c = 0; c < 16; ++c) dst[c] = f32_to_bf16_rne(o[c] * inv);
           }
-          if (c0 < kQTmem) tm_st_x8_s8(trow + kColQ + c0 / 2, v);
-          else store_qlat(qlat, n, c0 + 16 * qt - kQTmem, v);
+        } else {
+          float* dst = p.part_o + (int64_t(pslot) * kPairRows + n) * r + lat0 + c0;
+#pragma unroll
+          for (int c = 0; c < 16; c += 4)
+            *reinterpret_cast<float4*>(dst + c) =
+                make_float4(o[c] * inv, o[c + 1] * inv, o[c + 2] * inv, o[c + 3] * inv);
         }
-        for (int c = qt; c < rh / 8; c += 2) {
-          const uint4 v = row_ok ? *reinterpret_cast<const uint4*>(q + r + int(rank) * rh + 8 * c)
-                                 : make_uint4(0, 0, 0, 0);
-          *reinterpret_cast<uint4*>(qrope + swizzled_chunk(n, c, rpitch)) = v;
-        }
-        tmem_wait_st();
-        fence_proxy_async_smem();
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(q_full);
-      };
+      }
+      tc_fence_before();
+    };
 
+    if (role == 0) {
+      // ------------- owner: this CTA's 16 rows of sub-partition sp; softmax and P ---------
+      const int qi = row / p.num_heads;
       load_q(sched[0]);
       UnitWalk w{sched[0], sched[1]};
       w.load(p, cg);
@@ -567,7 +634,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             uint32_t wb[kPackWords];
 #pragma unroll
             for (int c = 0; c < kPackWords / 4; ++c) {
-              const uint4 v = ld_shared_v4(src + xs_offset(ow, lane, c));
+              const uint4 v = ld_shared_v4(src + xs_offset(sp, lane, c));
               wb[4 * c] = v.x; wb[4 * c + 1] = v.y; wb[4 * c + 2] = v.z; wb[4 * c + 3] = v.w;
             }
 #pragma unroll
@@ -575,7 +642,7 @@ __global__ void __launch_bounds__(kThreads, 1)
               float f[4];
               unpack_f24(wb + 3 * g, f);
 #pragma unroll
-              for (int i = 0; i < 4; ++i) s[4 * g + i] = rcv ? s[4 * g + i] + f[i] : 0.0f;
+              for (int k = 0; k < 4; ++k) s[4 * g + k] = rcv ? s[4 * g + k] + f[k] : 0.0f;
             }
           }
           __syncwarp();
@@ -583,7 +650,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           // release fence (which would wait for this warp's remote stores), and re-arm it for
           // tile jj + 2 (the partner sends that only after all four owner warps released it).
           if (lane == 1) mbar_arrive_remote_relaxed(sb ? xs_free_r1 : xs_free_r0);
-          if (ow == 0 && lane == 0 && rcv) mbar_arrive_expect_tx_relaxed(&xs_full[sb], kXsBytes);
+          if (sp == 0 && lane == 0 && rcv) mbar_arrive_expect_tx_relaxed(&xs_full[sb], kXsBytes);
 
           // ---- online softmax of row n over this tile (log2 domain, lazy reference) ----
           if (pos0 + kHalfTok - 1 > lim) {
@@ -606,22 +673,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             l *= alpha;
             mref = mx;
           }
-          // O rows of an earlier tile of the piece: rescale once PV(jj - 1) has landed
-          if (t > tb && __any_sync(0xffffffffu, alpha != 1.0f)) {
-            const bool pv_ok = __all_sync(
-                0xffffffffu, mbar_wait(&pv_done[(jj - 1) & 1], ((jj - 1) >> 1) & 1, wc));
-            tc_fence_after();
-            if (pv_ok) {
-              for (int c0 = 0; c0 < rhalf; c0 += 32) {
-                float o[16];
-                tm_ld_x16_s16(trow + kColO + c0, o);
-                tmem_wait_ld();
-#pragma unroll
-                for (int c = 0; c < 16; ++c) o[c] *= alpha;
-                tm_st_x16_s16(trow + kColO + c0, reinterpret_cast<const uint32_t*>(o));
-              }
-            }
-          }
+          // O rows of an earlier tile of the piece: rescale (the first tile overwrites O)
+          if (t > tb && __any_sync(0xffffffffu, alpha != 1.0f)) rescale_o(jj, alpha);
           // weights 2^(s * scale - m) over the S buffer (its scores are in registers)
           uint32_t pk[kHalfTok / 2];
           float sa = 0.0f, sc = 0.0f;
@@ -635,7 +688,6 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
           l += sa + sc;
           lt = l + __shfl_xor_sync(0xffffffffu, l, 16);
-          // this tile's P buffer held P of tile jj - 2: PV of that tile must have read it
           if (jj >= 2) {
             __all_sync(0xffffffffu, mbar_wait(&pv_done[sb], ((jj - 2) >> 1) & 1, wc));
             tc_fence_after();
@@ -646,9 +698,9 @@ __global__ void __launch_bounds__(kThreads, 1)
               __all_sync(0xffffffffu, jj == 0 || mbar_wait_cluster(xp_free, (jj - 1) & 1, wc));
           if (pfree) {
 #pragma unroll
-            for (int i = 0; i < 4; ++i)
-              st_async_v4(xp_r + xp_offset(m, 4 * qt + i),
-                          make_uint4(pk[4 * i], pk[4 * i + 1], pk[4 * i + 2], pk[4 * i + 3]),
+            for (int k = 0; k < 4; ++k)
+              st_async_v4(xp_r + xp_offset(m, 4 * qt + k),
+                          make_uint4(pk[4 * k], pk[4 * k + 1], pk[4 * k + 2], pk[4 * k + 3]),
                           xp_full_r);
             if (qt == 0)
               st_async_v2(xp_r + xp_scalars(m),
@@ -658,7 +710,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           // cache rows past the context may hold anything (even NaN): zero their latent half
           // so that 0-weight x garbage cannot reach O
           if (tile_pos0 + kDecodeTok > L) {
-            const int tid = ow * 32 + lane;      // 0..127
+            const int tid = sp * 32 + lane;      // 0..127
             const int tok = tid & (kDecodeTok - 1);
             if (tile_pos0 + tok >= L) {
               uint8_t* sbase = slots + slot * lay.slot_bytes;
@@ -676,103 +728,22 @@ __global__ void __launch_bounds__(kThreads, 1)
           __syncwarp();
           if (lane == 0) mbar_arrive(&p_full[sb]);
         }
-
-        // ------------------------- epilogue of this piece (own rows) -----------------------
-        const int jl = jj - 1;
-        const bool fin = __all_sync(0xffffffffu, mbar_wait(&pv_done[jl & 1], (jl >> 1) & 1, wc));
-        tc_fence_after();
-        const bool aborted = __any_sync(0xffffffffu, !fin || *abort_flag != 0);
-        const bool whole = (tb == w.s) && (te == w.s + w.tiles);
-        const int64_t grow = int64_t(w.b) * p.qH + row;   // global (b, i, h) row
-        const int pslot = piece_slot(vc, w.s, per, p.col_groups, cg);
-        const float lse = (lt > 0.0f && !aborted) ? (mref + __log2f(lt)) * kLn2 : -INFINITY;
+        // ---- epilogue of this piece: O and lse of the own rows ----
+        bool aborted = false;
+        write_o(w, tb, te, jj - 1, lt, &aborted);
         if (row_ok && qt == 0) {
-          if (whole) p.lse[grow] = lse;
-          else p.part_lse[int64_t(pslot) * kPairRows + n] = lse;
+          const float lse = (lt > 0.0f && !aborted) ? (mref + __log2f(lt)) * kLn2 : -INFINITY;
+          const bool whole = (tb == w.s) && (te == w.s + w.tiles);
+          if (whole) p.lse[int64_t(w.b) * p.qH + row] = lse;
+          else p.part_lse[int64_t(piece_slot(vc, w.s, per, p.col_groups, cg)) * kPairRows + n] = lse;
         }
-        const float inv = (lt > 0.0f && !aborted) ? 1.0f / lt : 0.0f;
-        const int64_t lat0 = int64_t(rank) * rhalf + 16 * qt;   // this thread's 16 of every 32
-        for (int c0 = 0; c0 < rhalf; c0 += 32) {
-          float o[16];
-          if (!aborted) {
-            tm_ld_x16_s16(trow + kColO + c0, o);
-            tmem_wait_ld();
-          } else {
-#pragma unroll
-            for (int c = 0; c < 16; ++c) o[c] = 0.0f;
-          }
-          if (!row_ok) {
-            // padding row past q*H: nothing to write
-          } else if (whole) {
-            uint16_t* dst = p.o_latent + grow * r + lat0 + c0;
-            if (vec_out) {
-#pragma unroll
-              for (int c = 0; c < 16; c += 8)
-                *reinterpret_cast<uint4*>(dst + c) =
-                    make_uint4(cvt_bf16x2(o[c] * inv, o[c + 1] * inv),
-                               cvt_bf16x2(o[c + 2] * inv, o[c + 3] * inv),
-                               cvt_bf16x2(o[c + 4] * inv, o[c + 5] * inv),
-                               cvt_bf16x2(o[c + 6] * inv, o[c + 7] * inv));
-            } else {
-#pragma unroll
-              for (int c = 0; c < 16; ++c) dst[c] = f32_to_bf16_rne(o[c] * inv);
-            }
-          } else {
-            float* dst = p.part_o + (int64_t(pslot) * kPairRows + n) * r + lat0 + c0;
-#pragma unroll
-            for (int c = 0; c < 16; c += 4)
-              *reinterpret_cast<float4*>(dst + c) =
-                  make_float4(o[c] * inv, o[c + 1] * inv, o[c + 2] * inv, o[c + 3] * inv);
-          }
-        }
-        tc_fence_before();
         w.s += w.tiles;
         ++w.b;
         if (w.s >= r1) break;
         w.load(p, cg);
       }
-    } else if (hl == 0) {
-      // ---------------- sender: the partner rows' partial scores, one row per lane ---------
-      const int n = 32 * sp + lane;           // query row (TMEM lane)
-      const uint32_t tq = tmem + (uint32_t(32 * sp) << 16);
-      const int row = cg * kPairRows + n;
-      const bool row_ok = row < p.qH;
-      // where the partner's owner threads of this row read: warp 2 (lane / 16) + (sp & 1),
-      // lanes (lane % 16) and (lane % 16) + 16 for the two token halves
-      const int ow_o = 2 * (lane >> 4) + (sp & 1);
-      const bool tr = ((sp & 1) == 0 && lane == 0);
-      (void)tr;
-
-      // This CTA's half of Q row n (one thread per row), as the owners' load_q.
-      auto load_q = [&](int b) {
-        const uint16_t* q = p.q_ext + (int64_t(b) * p.qH + row) * p.D;
-        for (int c0 = 0; c0 < rhalf; c0 += 16) {
-          const uint16_t* src = q + int(rank) * rhalf + c0;
-          uint32_t v[8];
-          if (row_ok) {
-            const uint4 a = *reinterpret_cast<const uint4*>(src);
-            const uint4 bb = *reinterpret_cast<const uint4*>(src + 8);
-            v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w;
-            v[4] = bb.x; v[5] = bb.y; v[6] = bb.z; v[7] = bb.w;
-          } else {
-#pragma unroll
-            for (int i = 0; i < 8; ++i) v[i] = 0u;
-          }
-          if (c0 < kQTmem) tmem_st8(tq + kColQ + c0 / 2, v);
-          else store_qlat(qlat, n, c0 - kQTmem, v);
-        }
-        for (int c = 0; c < rh / 8; ++c) {
-          const uint4 v = row_ok ? *reinterpret_cast<const uint4*>(q + r + int(rank) * rh + 8 * c)
-                                 : make_uint4(0, 0, 0, 0);
-          *reinterpret_cast<uint4*>(qrope + swizzled_chunk(n, c, rpitch)) = v;
-        }
-        tmem_wait_st();
-        fence_proxy_async_smem();
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(q_full);
-      };
-
+    } else if (role == 1) {
+      // ------------- sender: the partner's 16 rows of sub-partition sp, partial scores ----
       load_q(sched[0]);
       UnitWalk w{sched[0], sched[1]};
       int jj = 0;
@@ -781,53 +752,42 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int tb = max(w.s, r0), te = min(w.s + w.tiles, r1);
         for (int t = tb; t < te; ++t, ++jj) {
           const int sb = jj & 1;
-          float x[kDecodeTok];
+          float x[kHalfTok];
           const bool got = __all_sync(0xffffffffu, mbar_wait(&s_full[sb], (jj >> 1) & 1, wc));
           tc_fence_after();
           if (got) {
-            tmem_ld32(tq + kColS + 64 * sb, x);
-            tmem_ld32(tq + kColS + 64 * sb + 32, x + 32);
+            tm_ld_x32_s32(trow + kColS + 64 * sb, x);
             tmem_wait_ld();
           } else {
 #pragma unroll
-            for (int c = 0; c < kDecodeTok; ++c) x[c] = 0.0f;
+            for (int c = 0; c < kHalfTok; ++c) x[c] = 0.0f;
           }
           if (tr) MLA_PTRACE(3, jj);
           tc_fence_before();
           __syncwarp();
           if (lane == 0) mbar_arrive(&s_free[sb]);
           if (t == te - 1 && w.s + w.tiles < r1) load_q(w.b + 1);
-          uint32_t pw[2 * kPackWords];
+          uint32_t pw[kPackWords];
 #pragma unroll
-          for (int g = 0; g < kDecodeTok / 4; ++g) pack_f24(x + 4 * g, pw + 3 * g);
+          for (int g = 0; g < kHalfTok / 4; ++g) pack_f24(x + 4 * g, pw + 3 * g);
           // into the partner's buffer sb once its owners consumed tile jj - 2 from it: stores
-          // from registers over the SM-to-SM network, completing on the partner's mbarrier
+          // from registers over the SM-to-SM network, completing on the partner's mbarrier.
+          // The partner's owner thread of this (row, half) is the same lane of its warp sp.
           const bool free_ok = __all_sync(
               0xffffffffu, jj < 2 || mbar_wait_cluster(&xs_free[sb], ((jj - 2) >> 1) & 1, wc));
           if (free_ok) {
             const uint32_t dst = xs_r + sb * kXsBytes;
             const uint32_t rb = sb ? xs_full_r1 : xs_full_r0;
 #pragma unroll
-            for (int h = 0; h < 2; ++h)
-#pragma unroll
-              for (int c = 0; c < kPackWords / 4; ++c) {
-                const uint32_t* wp = pw + kPackWords * h + 4 * c;
-                st_async_v4(dst + xs_offset(ow_o, (lane & 15) + 16 * h, c),
-                            make_uint4(wp[0], wp[1], wp[2], wp[3]), rb);
-              }
+            for (int c = 0; c < kPackWords / 4; ++c)
+              st_async_v4(dst + xs_offset(sp, lane, c),
+                          make_uint4(pw[4 * c], pw[4 * c + 1], pw[4 * c + 2], pw[4 * c + 3]), rb);
           }
           if (tr) MLA_PTRACE(4, jj);
         }
       }
     } else {
-      // ---------------- receiver: the partner's weights for its rows; their epilogue ------
-      const int n = 32 * sp + lane;           // query row (TMEM lane)
-      const int m = n & 63;                   // row within the partner's block
-      const uint32_t tq = tmem + (uint32_t(32 * sp) << 16);
-      const int row = cg * kPairRows + n;
-      const bool row_ok = row < p.qH;
-      const bool tr = ((sp & 1) == 0 && lane == 0);
-      (void)tr;
+      // ------------- receiver: the partner's weights for its 16 rows of sub-partition sp --
       UnitWalk w{sched[0], sched[1]};
       w.load(p, cg);
       int jj = 0;
@@ -838,98 +798,42 @@ __global__ void __launch_bounds__(kThreads, 1)
           const int sb = jj & 1;
           const bool rcv = __all_sync(0xffffffffu, mbar_wait_cluster(xp_full, jj & 1, wc));
           if (tr) MLA_PTRACE(7, jj);
-          uint32_t pk[kDecodeTok / 2];
+          uint32_t pk[kHalfTok / 2];
           float alpha = 1.0f;
           if (rcv) {
 #pragma unroll
-            for (int c = 0; c < kDecodeTok / 8; ++c) {
-              const uint4 v = ld_shared_v4(xp_s + xp_offset(m, c));
-              pk[4 * c] = v.x; pk[4 * c + 1] = v.y; pk[4 * c + 2] = v.z; pk[4 * c + 3] = v.w;
+            for (int k = 0; k < 4; ++k) {
+              const uint4 v = ld_shared_v4(xp_s + xp_offset(m, 4 * qt + k));
+              pk[4 * k] = v.x; pk[4 * k + 1] = v.y; pk[4 * k + 2] = v.z; pk[4 * k + 3] = v.w;
             }
-            const uint2 sc = ld_shared_v2(xp_s + xp_scalars(m));
-            alpha = __uint_as_float(sc.x);
-            lt = __uint_as_float(sc.y);
+            const uint2 sv = ld_shared_v2(xp_s + xp_scalars(m));
+            alpha = __uint_as_float(sv.x);
+            lt = __uint_as_float(sv.y);
           } else {
 #pragma unroll
-            for (int c = 0; c < kDecodeTok / 2; ++c) pk[c] = 0u;
+            for (int c = 0; c < kHalfTok / 2; ++c) pk[c] = 0u;
             lt = 0.0f;
           }
           __syncwarp();
           // consumed into registers: release the buffer (relaxed) and re-arm it for tile jj + 1
           if (lane == 1) mbar_arrive_remote_relaxed(xp_free_r);
-          if ((sp & 1) == 0 && lane == 0 && rcv) mbar_arrive_expect_tx_relaxed(xp_full, kXpBytes);
+          if (sp == 0 && lane == 0 && rcv) mbar_arrive_expect_tx_relaxed(xp_full, kXpBytes);
           // the owner moved its reference: rescale these rows of this CTA's O half the same way
-          if (t > tb && __any_sync(0xffffffffu, alpha != 1.0f)) {
-            const bool pv_ok = __all_sync(
-                0xffffffffu, mbar_wait(&pv_done[(jj - 1) & 1], ((jj - 1) >> 1) & 1, wc));
-            tc_fence_after();
-            if (pv_ok) {
-              for (int c0 = 0; c0 < rhalf; c0 += 32) {
-                float o[32];
-                tmem_ld32(tq + kColO + c0, o);
-                tmem_wait_ld();
-#pragma unroll
-                for (int c = 0; c < 32; ++c) o[c] *= alpha;
-                tmem_st32(tq + kColO + c0, reinterpret_cast<const uint32_t*>(o));
-              }
-            }
-          }
+          if (t > tb && __any_sync(0xffffffffu, alpha != 1.0f)) rescale_o(jj, alpha);
           if (jj >= 2) {
             __all_sync(0xffffffffu, mbar_wait(&pv_done[sb], ((jj - 2) >> 1) & 1, wc));
             tc_fence_after();
           }
-          tmem_st32(tq + kColP + 32 * sb, pk);
+          tm_st_x16_s16(trow + kColP + 32 * sb, pk);
           tmem_wait_st();
           tc_fence_before();
           __syncwarp();
           if (lane == 0) mbar_arrive(&p_full[sb]);
           if (tr) MLA_PTRACE(11, jj);
         }
-
-        // ---------------------- epilogue of this piece (the partner's rows) ----------------
-        const int jl = jj - 1;
-        const bool fin = __all_sync(0xffffffffu, mbar_wait(&pv_done[jl & 1], (jl >> 1) & 1, wc));
-        tc_fence_after();
-        const bool aborted = __any_sync(0xffffffffu, !fin || *abort_flag != 0);
-        const bool whole = (tb == w.s) && (te == w.s + w.tiles);
-        const int64_t grow = int64_t(w.b) * p.qH + row;
-        const int pslot = piece_slot(vc, w.s, per, p.col_groups, cg);
-        const float inv = (lt > 0.0f && !aborted) ? 1.0f / lt : 0.0f;
-        const int64_t lat0 = int64_t(rank) * rhalf;
-        for (int c0 = 0; c0 < rhalf; c0 += 32) {
-          float o[32];
-          if (!aborted) {
-            tmem_ld32(tq + kColO + c0, o);
-            tmem_wait_ld();
-          } else {
-#pragma unroll
-            for (int c = 0; c < 32; ++c) o[c] = 0.0f;
-          }
-          if (!row_ok) {
-            // padding row past q*H: nothing to write
-          } else if (whole) {
-            uint16_t* dst = p.o_latent + grow * r + lat0 + c0;
-            if (vec_out) {
-#pragma unroll
-              for (int c = 0; c < 32; c += 8)
-                *reinterpret_cast<uint4*>(dst + c) =
-                    make_uint4(cvt_bf16x2(o[c] * inv, o[c + 1] * inv),
-                               cvt_bf16x2(o[c + 2] * inv, o[c + 3] * inv),
-                               cvt_bf16x2(o[c + 4] * inv, o[c + 5] * inv),
-                               cvt_bf16x2(o[c + 6] * inv, o[c + 7] * inv));
-            } else {
-#pragma unroll
-              for (int c = 0; c < 32; ++c) dst[c] = f32_to_bf16_rne(o[c] * inv);
-            }
-          } else {
-            float* dst = p.part_o + (int64_t(pslot) * kPairRows + n) * r + lat0 + c0;
-#pragma unroll
-            for (int c = 0; c < 32; c += 4)
-              *reinterpret_cast<float4*>(dst + c) =
-                  make_float4(o[c] * inv, o[c + 1] * inv, o[c + 2] * inv, o[c + 3] * inv);
-          }
-        }
-        tc_fence_before();
+        // ---- epilogue of this piece: O of the partner's rows (this CTA's latent half) ----
+        bool aborted = false;
+        write_o(w, tb, te, jj - 1, lt, &aborted);
         w.s += w.tiles;
         ++w.b;
         if (w.s >= r1) break;
