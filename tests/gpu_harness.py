@@ -126,6 +126,27 @@ class GpuProblem:
                                       self.cfg.softmax_scale, causal=self.cfg.causal)
 
 
+    def oracle_heads(self, b: int, heads) -> dict:
+        """The oracle for sequence b restricted to some heads: {h: {"o", "o_latent", "lse"}}
+        with arrays over the q query rows. Heads are independent in the oracle, so the
+        inputs are sliced per key group (the heads of one group see one k_r slice)."""
+        import oracle.mla_oracle as O  # test infrastructure only
+        wl, cfg = self.wl, self.cfg
+        c_kv, k_r = wl.context(b)
+        g_of = O.group_of_head(cfg.num_heads, cfg.num_kv_groups)
+        out = {}
+        for g in sorted({int(g_of[h]) for h in heads}):
+            hs = [int(h) for h in heads if int(g_of[h]) == g]
+            bias = None if wl.bias is None else wl.bias[hs]
+            ref = O.mla_decode_reference(wl.q_nope[b][:, hs], wl.q_pe[b][:, hs], c_kv,
+                                         k_r[:, g:g + 1], wl.w_uk[hs], wl.w_uv[hs], bias,
+                                         wl.theta[g:g + 1], wl.query_positions()[b],
+                                         cfg.softmax_scale, causal=cfg.causal)
+            for j, h in enumerate(hs):
+                out[h] = {k: ref[k][:, j] for k in ("o", "o_latent", "lse")}
+        return out
+
+
 def max_rel_err(got: np.ndarray, ref: np.ndarray) -> float:
     """max|got - ref| / max|ref| (the tolerance measure of the parity tests)."""
     return float(np.max(np.abs(got - ref)) / max(np.max(np.abs(ref)), 1e-30))
