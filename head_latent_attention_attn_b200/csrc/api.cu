@@ -256,7 +256,9 @@ mla_status mla_absorb_q(const mla_dims* dims, const void* q_nope, const void* q_
   p.rope_sin = rope_sin;
   p.groups = dims->num_kv_groups;
   p.rope_dim = dims->rope_dim;
-  return launch_wgemm(p, nr, as_stream(stream)) == cudaSuccess ? MLA_OK : MLA_ERR_CUDA;
+  p.rope_vec = (dims->rope_dim % 8 == 0 && aligned(q_pe, 8) && aligned(rope_cos, 16) &&
+                aligned(rope_sin, 16)) ? 1 : 0;
+  return launch_wgemm(p, nr, num_sms(), as_stream(stream)) == cudaSuccess ? MLA_OK : MLA_ERR_CUDA;
 }
 
 mla_status mla_out_up(const mla_dims* dims, const void* o_latent, const void* w_uv,
@@ -298,7 +300,7 @@ mla_status mla_out_up(const mla_dims* dims, const void* o_latent, const void* w_
   p.heads = H;
   p.a_mn = 0;
   p.q_pe = nullptr;
-  return launch_wgemm(p, nr, as_stream(stream)) == cudaSuccess ? MLA_OK : MLA_ERR_CUDA;
+  return launch_wgemm(p, nr, num_sms(), as_stream(stream)) == cudaSuccess ? MLA_OK : MLA_ERR_CUDA;
 }
 
 size_t mla_decode_workspace_size(const mla_dims* dims, int32_t batch, int32_t q_len,

@@ -39,8 +39,10 @@ struct WGemmParams {
   const float* rope_cos;     // [rows, G, d_r/2]
   const float* rope_sin;
   int32_t groups, rope_dim;
+  int32_t rope_vec;          // 1: q_pe 8-byte, cos/sin 16-byte aligned and d_r/2 % 4 == 0
 };
-cudaError_t launch_wgemm(const WGemmParams& p, int nr, cudaStream_t stream);
+// max_ctas: the persistent grid's size limit (one CTA per SM)
+cudaError_t launch_wgemm(const WGemmParams& p, int nr, int max_ctas, cudaStream_t stream);
 
 // ---- mla_decode_attn -----------------------------------------------------------------------
 constexpr int kDecodeTok = 64;        // tokens per tile = one cache page

@@ -89,3 +89,31 @@ def test_packed_kv_b_proj_view():
     mla.mla_out_up(dims, o_lat, kvb.view(-1)[dn * r:], o1, w_uv_head_stride=(dn + dv) * r)
     mla.mla_out_up(dims, o_lat, wl.w_uv.cuda(), o2)
     assert torch.equal(o1, o2)
+
+
+def _offset_copy(t: torch.Tensor) -> torch.Tensor:
+    """The same values in a contiguous tensor whose start is one element past an aligned
+    allocation (so 2 or 4 bytes off every wider boundary)."""
+    buf = torch.empty(t.numel() + 1, dtype=t.dtype, device=t.device)
+    out = buf[1:].view(t.shape)
+    out.copy_(t)
+    return out
+
+
+@pytest.mark.parametrize("name", ["deepseek_v2", "qwen3_30b_a3b", "hybrid_q4"])
+def test_absorb_rope_unaligned_inputs(name):
+    """q_pe, cos and sin off their vector alignment take the scalar rotary path; q_ext is
+    bit-identical to the aligned call's."""
+    cfg = CASES[name]
+    wl = make_workload(cfg)
+    dims = dims_of(cfg)
+    B, q, H, D = cfg.batch, cfg.q_len, cfg.num_heads, cfg.row_width
+    cos, sin = wl.rope_table(wl.query_positions())
+    q_pe, cos_t, sin_t = wl.q_pe.cuda(), torch.from_numpy(cos).cuda(), torch.from_numpy(sin).cuda()
+    outs = []
+    for qp, c, s in ((q_pe, cos_t, sin_t),
+                     (_offset_copy(q_pe), _offset_copy(cos_t), _offset_copy(sin_t))):
+        q_ext = torch.full((B, q, H, D), float("nan"), dtype=torch.bfloat16, device="cuda")
+        mla.mla_absorb_q(dims, wl.q_nope.cuda(), qp, c, s, wl.w_uk.cuda(), q_ext)
+        outs.append(q_ext.view(torch.int16).cpu())
+    assert torch.equal(outs[0], outs[1])
