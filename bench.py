@@ -26,6 +26,7 @@ import os
 import statistics
 import subprocess
 import sys
+import tempfile
 import time
 
 import numpy as np
@@ -93,7 +94,8 @@ class ClockSampler:
     """SM clock, power and clock-event (throttle) reasons of this GPU during the timed region:
     a child process polls NVML as fast as it answers (a timed region of a few milliseconds
     still gets samples); nvidia-smi every 200 ms when NVML is not importable. Only samples
-    between mark_start() and mark_end() count. Rows go to gpurun_out/clocks_rank<R>.csv."""
+    between mark_start() and mark_end() count. Rows go to the file MLA_BENCH_CLOCKS_CSV names
+    (with the rank appended before .csv), else to a temporary file."""
     Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
          "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
          "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
@@ -107,15 +109,24 @@ class ClockSampler:
         self.kind = None   # "nvml" or "nvidia-smi"
         self.path = None
         self.rows = None   # (time, sm_mhz, max_mhz, power_w, reasons bitmask) for "nvml"
+        self.tmp = False   # the sample file is a temporary file of ours (removed after use)
         self.t0 = self.t1 = None
 
     def __enter__(self):
         try:
-            out_dir = os.path.join(ROOT, "gpurun_out")
-            os.makedirs(out_dir, exist_ok=True)
-            self.path = os.path.join(out_dir, f"clocks_rank{os.environ.get('RANK', '0')}.csv")
-            if os.path.exists(self.path):
-                os.remove(self.path)
+            rank = os.environ.get("RANK", "0")
+            want = os.environ.get("MLA_BENCH_CLOCKS_CSV")
+            if want:
+                root, ext = os.path.splitext(want)
+                self.path = f"{root}_rank{rank}{ext or '.csv'}"
+                os.makedirs(os.path.dirname(os.path.abspath(self.path)), exist_ok=True)
+                if os.path.exists(self.path):
+                    os.remove(self.path)
+            else:
+                fd, self.path = tempfile.mkstemp(prefix=f"mla_clocks_rank{rank}_", suffix=".csv")
+                os.close(fd)
+                self.tmp = True
+                os.remove(self.path)   # the sampler creates it; its size tells it has started
         except Exception:
             self.path = None
             return self
@@ -178,6 +189,15 @@ class ClockSampler:
                 pass
 
     def summary(self):
+        out = self._summary()
+        if self.tmp and self.path is not None:
+            try:
+                os.remove(self.path)
+            except OSError:
+                pass
+        return out
+
+    def _summary(self):
         if self.kind == "nvml":
             rows = [r for r in (self.rows or [])
                     if self.t0 is None or self.t1 is None or self.t0 <= r[0] <= self.t1]
