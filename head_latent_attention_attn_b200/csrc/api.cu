@@ -143,8 +143,8 @@ mla_status plan_decode(const mla_dims* d, int32_t batch, int32_t q_len, int32_t 
   off = align256(off + size_t(units) * sizeof(int32_t));
   P->part_lse_off = off;                         // two partial slots per range
   off = align256(off + size_t(g) * 2 * P->ncol * sizeof(float));
-  P->part_o_off = off;
-  off += size_t(g) * 2 * P->ncol * size_t(r) * sizeof(float);
+  P->part_o_off = off;                           // bf16: one rounding more than o_latent's
+  off += size_t(g) * 2 * P->ncol * size_t(r) * sizeof(uint16_t);
   P->ws_bytes = off;
   return MLA_OK;
 }
@@ -362,7 +362,7 @@ mla_status mla_decode_attn(const mla_dims* dims, const void* q_ext, const void* 
   p.o_latent = static_cast<uint16_t*>(o_latent);
   p.lse = lse;
   p.part_lse = reinterpret_cast<float*>(ws + P.part_lse_off);
-  p.part_o = reinterpret_cast<float*>(ws + P.part_o_off);
+  p.part_o = reinterpret_cast<uint16_t*>(ws + P.part_o_off);
   p.unit_start = reinterpret_cast<int32_t*>(ws + P.unit_start_off);
   p.range_len = reinterpret_cast<int32_t*>(ws + P.range_off);
   p.dev_error = reinterpret_cast<int32_t*>(ws);

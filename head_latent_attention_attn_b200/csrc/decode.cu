@@ -15,8 +15,8 @@
 // ceil(L_b / 64) page tiles. The units' tiles are laid end to end and cut into gridDim.x
 // equal ranges, one per CTA, so ragged lengths balance. A CTA walks the units its range
 // touches; a unit it holds whole is written straight to o_latent / lse, a unit cut
-// between CTAs leaves one normalised fp32 partial (o, lse) per piece, merged afterwards
-// by mla_combine_kernel with the log-sum-exp identity.
+// between CTAs leaves one normalised partial per piece (o in bf16, lse in fp32), merged
+// afterwards by mla_combine_kernel with the log-sum-exp identity.
 //
 // Roles (192 threads): warp 0 TMA producer, warp 1 UMMA issuer and TMEM owner, warps 2-5
 // softmax and epilogue. In the M=64 accumulator layout rows 16*sp..16*sp+15 sit in lanes
@@ -586,8 +586,8 @@ __global__ void __launch_bounds__(kThreads, 1)
               const int col = n0 + n;
               if (col < cols_here) {
                 const float v = o[n] * inv[n];
-                if (whole) p.o_latent[(row0 + col) * p.r + lat] = f32_to_bf16_rne(v);
-                else p.part_o[(int64_t(pslot) * NCOL + col) * p.r + lat] = v;
+                if (whole) p.o_latent[(row0 + col) * p.r + lat] = cvt_bf16(v);
+                else p.part_o[(int64_t(pslot) * NCOL + col) * p.r + lat] = cvt_bf16(v);
               }
             }
           }
@@ -604,7 +604,9 @@ __global__ void __launch_bounds__(kThreads, 1)
 
 // ---- merge of cut units: lse = log sum_i e^{lse_i}, o = sum_i e^{lse_i - lse} o_i ------
 // One block per (unit, query row): warp 0 reduces the pieces' lse, then the 4 warps split
-// the pieces and every lane accumulates up to 16 latents; shared memory adds the warps.
+// the pieces and every lane accumulates up to 16 latents (8 x lane + 256 k + 0..7: one
+// 16-byte load of a piece's bf16 row per k; two pieces' loads in flight per step); shared
+// memory adds the warps.
 __global__ void __launch_bounds__(128) mla_combine_kernel(const CombineParams p) {
   __shared__ float part[4][512];
   __shared__ float lse_s;
@@ -643,22 +645,42 @@ __global__ void __launch_bounds__(128) mla_combine_kernel(const CombineParams p)
   float acc[16];
 #pragma unroll
   for (int j = 0; j < 16; ++j) acc[j] = 0.0f;
-  for (int i = i0 + warp; i <= i1; i += 4) {
+  // latents 8 * lane + 256 * k + e of a piece's row: 16-byte aligned (r % 8 == 0)
+  auto add_piece = [&](int i) {
     const int64_t sl = piece_slot(i, s, per, G, cg);
     const float li = p.part_lse[sl * p.ncol + n];
-    if (li == -INFINITY) continue;
-    const float wgt = expf(li - lse);
-    const float* row = p.part_o + (sl * p.ncol + n) * p.r;
+    const uint16_t* row = p.part_o + (sl * p.ncol + n) * p.r;
+    uint4 v[2];
 #pragma unroll
-    for (int j = 0; j < 16; ++j) {
-      const int lat = lane + 32 * j;
-      if (lat < p.r) acc[j] += wgt * row[lat];
+    for (int k = 0; k < 2; ++k) {
+      const int lat = 8 * lane + 256 * k;
+      v[k] = (lat < p.r && li != -INFINITY) ? *reinterpret_cast<const uint4*>(row + lat)
+                                            : make_uint4(0u, 0u, 0u, 0u);
     }
-  }
+    const float wgt = li == -INFINITY ? 0.0f : expf(li - lse);
 #pragma unroll
-  for (int j = 0; j < 16; ++j) {
-    const int lat = lane + 32 * j;
-    if (lat < p.r) part[warp][lat] = acc[j];
+    for (int k = 0; k < 2; ++k) {
+      const uint32_t w[4] = {v[k].x, v[k].y, v[k].z, v[k].w};
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        acc[8 * k + 2 * e] += wgt * __uint_as_float(w[e] << 16);
+        acc[8 * k + 2 * e + 1] += wgt * __uint_as_float(w[e] & 0xFFFF0000u);
+      }
+    }
+  };
+  int i = i0 + warp;
+  for (; i + 4 <= i1; i += 8) {
+    add_piece(i);
+    add_piece(i + 4);
+  }
+  if (i <= i1) add_piece(i);
+#pragma unroll
+  for (int k = 0; k < 2; ++k) {
+    const int lat = 8 * lane + 256 * k;
+    if (lat < p.r) {
+#pragma unroll
+      for (int e = 0; e < 8; ++e) part[warp][lat + e] = acc[8 * k + e];
+    }
   }
   __syncthreads();
   uint16_t* out = p.o_latent + (int64_t(b) * p.qH + f) * p.r;
@@ -668,8 +690,10 @@ __global__ void __launch_bounds__(128) mla_combine_kernel(const CombineParams p)
 }
 
 // The same merge with one warp per (unit, query row), four rows per block: for units cut
-// into a few pieces. Lanes own latents 4 * lane + 128 k + {0..3}: every load of a piece's
-// row is one 512-byte coalesced segment per warp.
+// into a few pieces. Up to 32 pieces, lane i reads piece i0 + i's lse once and the maximum,
+// the sum and each piece's weight come from shuffles; more pieces take a loop over global
+// memory. Lanes own latents 4 * lane + 128 k + {0..3}: every load of a piece's bf16 row is
+// one 256-byte coalesced segment per warp.
 __global__ void __launch_bounds__(128) mla_combine_rows_kernel(const CombineParams p) {
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int64_t gw = int64_t(blockIdx.x) * 4 + warp;
@@ -688,15 +712,25 @@ __global__ void __launch_bounds__(128) mla_combine_rows_kernel(const CombinePara
   const int s = p.unit_start[u];
   const int i0 = s / per, i1 = (s + tiles - 1) / per;
   if (i0 == i1) return;   // held whole by one range: already written
-  float mx = -INFINITY;
-  for (int i = i0 + lane; i <= i1; i += 32)
-    mx = fmaxf(mx, p.part_lse[int64_t(piece_slot(i, s, per, G, cg)) * p.ncol + n]);
+  const int np = i1 - i0 + 1;
+  const bool few = np <= 32;
+  // this lane's piece (few pieces) and the row's max and log-sum-exp
+  const float my_l = (few && lane < np)
+                         ? p.part_lse[int64_t(piece_slot(i0 + lane, s, per, G, cg)) * p.ncol + n]
+                         : -INFINITY;
+  float mx = my_l;
+  if (!few)
+    for (int i = i0 + lane; i <= i1; i += 32)
+      mx = fmaxf(mx, p.part_lse[int64_t(piece_slot(i, s, per, G, cg)) * p.ncol + n]);
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
-  float den = 0.0f;
-  for (int i = i0 + lane; i <= i1; i += 32) {
-    const float li = p.part_lse[int64_t(piece_slot(i, s, per, G, cg)) * p.ncol + n];
-    den += li == -INFINITY ? 0.0f : expf(li - mx);
+  float den = my_l == -INFINITY ? 0.0f : expf(my_l - mx);
+  if (!few) {
+    den = 0.0f;
+    for (int i = i0 + lane; i <= i1; i += 32) {
+      const float li = p.part_lse[int64_t(piece_slot(i, s, per, G, cg)) * p.ncol + n];
+      den += li == -INFINITY ? 0.0f : expf(li - mx);
+    }
   }
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) den += __shfl_xor_sync(0xffffffffu, den, o);
@@ -706,19 +740,19 @@ __global__ void __launch_bounds__(128) mla_combine_rows_kernel(const CombinePara
   for (int k = 0; k < 4; ++k) acc[k] = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
   for (int i = i0; i <= i1; ++i) {
     const int64_t sl = piece_slot(i, s, per, G, cg);
-    const float li = p.part_lse[sl * p.ncol + n];
+    const float li = few ? __shfl_sync(0xffffffffu, my_l, i - i0) : p.part_lse[sl * p.ncol + n];
     if (li == -INFINITY) continue;
     const float wgt = expf(li - lse);
-    const float* row = p.part_o + (sl * p.ncol + n) * p.r;
+    const uint16_t* row = p.part_o + (sl * p.ncol + n) * p.r;
 #pragma unroll
     for (int k = 0; k < 4; ++k) {
       const int lat = 4 * lane + 128 * k;
       if (lat < p.r) {
-        const float4 v = *reinterpret_cast<const float4*>(row + lat);
-        acc[k].x += wgt * v.x;
-        acc[k].y += wgt * v.y;
-        acc[k].z += wgt * v.z;
-        acc[k].w += wgt * v.w;
+        const uint2 v = *reinterpret_cast<const uint2*>(row + lat);   // r % 4 == 0: 8-byte aligned
+        acc[k].x += wgt * __uint_as_float(v.x << 16);
+        acc[k].y += wgt * __uint_as_float(v.x & 0xFFFF0000u);
+        acc[k].z += wgt * __uint_as_float(v.y << 16);
+        acc[k].w += wgt * __uint_as_float(v.y & 0xFFFF0000u);
       }
     }
   }

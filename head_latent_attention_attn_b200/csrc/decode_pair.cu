@@ -542,7 +542,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     };
 
     // O rows of this warp divided by the row sum lt, to the outputs of piece (w, tb, te)
-    // whose last tile is jl: bf16 o_latent when the piece is the whole unit, else fp32 part_o.
+    // whose last tile is jl: bf16 o_latent when the piece is the whole unit, else the bf16 partial part_o.
     auto write_o = [&](const UnitWalk& w, int tb, int te, int jl, float lt, bool* aborted_out) {
       const bool fin = __all_sync(0xffffffffu, mbar_wait(&pv_done[jl & 1], (jl >> 1) & 1, wc));
       tc_fence_after();
@@ -579,11 +579,15 @@ __global__ void __launch_bounds__(kThreads, 1)
             for (int c = 0; c < 16; ++c) dst[c] = f32_to_bf16_rne(o[c] * inv);
           }
         } else {
-          float* dst = p.part_o + (int64_t(pslot) * kPairRows + n) * r + lat0 + c0;
+          // bf16 partial (16-byte aligned: r % 8 == 0 and lat0 + c0 a multiple of 16)
+          uint16_t* dst = p.part_o + (int64_t(pslot) * kPairRows + n) * r + lat0 + c0;
 #pragma unroll
-          for (int c = 0; c < 16; c += 4)
-            *reinterpret_cast<float4*>(dst + c) =
-                make_float4(o[c] * inv, o[c + 1] * inv, o[c + 2] * inv, o[c + 3] * inv);
+          for (int c = 0; c < 16; c += 8)
+            *reinterpret_cast<uint4*>(dst + c) =
+                make_uint4(cvt_bf16x2(o[c] * inv, o[c + 1] * inv),
+                           cvt_bf16x2(o[c + 2] * inv, o[c + 3] * inv),
+                           cvt_bf16x2(o[c + 4] * inv, o[c + 5] * inv),
+                           cvt_bf16x2(o[c + 6] * inv, o[c + 7] * inv));
         }
       }
       tc_fence_before();

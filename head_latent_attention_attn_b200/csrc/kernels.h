@@ -56,7 +56,7 @@ struct DecodeParams {
   const int32_t* seq_lens;
   uint16_t* o_latent;        // [B, q, H, r]
   float* lse;                // [B, q, H]
-  float* part_o;             // [grid, 2, NCOL, r]  partial outputs of cut units
+  uint16_t* part_o;          // [grid, 2, NCOL, r]  partial outputs of cut units (bf16)
   float* part_lse;           // [grid, 2, NCOL]
   int32_t* unit_start;       // [units] first tile of each unit in its row block (for the merge)
   int32_t* range_len;        // [1] tiles per CTA range (for the merge)
@@ -87,7 +87,7 @@ cudaError_t launch_decode_pair(const DecodeParams& p, dim3 grid, size_t smem,
 
 // Merge of the per-piece partials of units cut between CTAs (log-sum-exp identity).
 struct CombineParams {
-  const float* part_o;
+  const uint16_t* part_o;    // bf16
   const float* part_lse;
   const int32_t* unit_start;
   const int32_t* range_len;

@@ -414,6 +414,14 @@ __host__ __device__ __forceinline__ uint16_t f32_to_bf16_rne(float f) {
 
 MLA_DEVICE float bf16_bits_to_f32(uint16_t b) { return __uint_as_float(uint32_t(b) << 16); }
 
+// fp32 -> bf16 bits, hardware round-to-nearest-even (one instruction; a NaN may come out
+// with another payload than f32_to_bf16_rne's).
+MLA_DEVICE uint16_t cvt_bf16(float x) {
+  uint16_t r;
+  asm("cvt.rn.bf16.f32 %0, %1;" : "=h"(r) : "f"(x));
+  return r;
+}
+
 // Two fp32 -> packed bf16x2 (lo in the low half), hardware round-to-nearest-even.
 MLA_DEVICE uint32_t cvt_bf16x2(float lo, float hi) {
   uint32_t r;

@@ -104,24 +104,25 @@ def test_workspace_size(mla_lib):
     a256 = lambda x: (x + 255) // 256 * 256  # noqa: E731
     # 128 heads, q = 1: one block of 128 query rows per sequence on a cluster of two CTAs
     # that split the latent; 64 units, n ranges (clusters) per unit, two partial slots each
+    # (bf16 partial o, fp32 partial lse)
     d = _dims()
     for n in (1, 4):
         ranges = 64 * n
         off = a256(256 + 256 + 64 * 4)                  # error word, range, unit starts
         off = a256(off + ranges * 2 * 128 * 4)          # partial lse
-        assert mla.mla_decode_workspace_size(d, 64, 1, 8192, n) == off + ranges * 2 * 128 * 512 * 4
+        assert mla.mla_decode_workspace_size(d, 64, 1, 8192, n) == off + ranges * 2 * 128 * 512 * 2
     # 32 heads, q = 1: blocks of 32 rows, one CTA per range
     d32 = _dims(num_heads=32)
     for n in (1, 3):
         ranges = 64 * n
         off = a256(256 + 256 + 64 * 4)
         off = a256(off + ranges * 2 * 32 * 4)
-        assert mla.mla_decode_workspace_size(d32, 64, 1, 8192, n) == off + ranges * 2 * 32 * 512 * 4
+        assert mla.mla_decode_workspace_size(d32, 64, 1, 8192, n) == off + ranges * 2 * 32 * 512 * 2
     # 128 heads of rank 320 (not a multiple of 128): two blocks of 64 rows instead
     d320 = _dims(kv_lora_rank=320)
     off = a256(256 + 256 + 128 * 4)
     off = a256(off + 128 * 2 * 64 * 4)
-    assert mla.mla_decode_workspace_size(d320, 64, 1, 8192, 1) == off + 128 * 2 * 64 * 320 * 4
+    assert mla.mla_decode_workspace_size(d320, 64, 1, 8192, 1) == off + 128 * 2 * 64 * 320 * 2
     assert mla.mla_decode_workspace_size(d, 64, 0, 8192, 1) == 0        # invalid q_len
     assert mla.mla_decode_workspace_size(_dims(page_size=16), 1, 1, 64, 1) == 0
 
