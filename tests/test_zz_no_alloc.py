@@ -51,13 +51,14 @@ def test_noalloc_matches_workspace_decode(name):
 
 
 def test_noalloc_rejects_problems_beyond_the_scratch():
-    """64 sequences x 128 heads x rank 512 need more partial-result room than the scratch
-    holds even with one work range per (sequence, row block): refused, nothing launched."""
+    """256 sequences x 128 heads x rank 512 need more partial-result room than the scratch
+    holds even with one work range per (sequence, row block): 256 x 2 slots x 128 rows x 512
+    bf16 = 64 MiB > 32 MiB. Refused, nothing launched."""
     cfg = CONFIGS["deepseek_v2"]
     dims = dims_of(cfg)
     fake = ctypes.c_void_p(0x10000)
     st = mla.lib().mla_decode_attn_noalloc(ctypes.byref(dims), fake, fake, 100000, fake, 128,
-                                           fake, cfg.batch, 1, cfg.context, 1, fake, fake, fake,
+                                           fake, 256, 1, cfg.context, 1, fake, fake, fake,
                                            None)
     assert st == mla.MLA_ERR_WORKSPACE
     st = mla.lib().mla_decode_attn_noalloc(ctypes.byref(dims_of(cfg.with_(page_size=32))), fake,
