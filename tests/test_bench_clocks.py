@@ -48,3 +48,46 @@ def test_all_reason_bits():
 def test_no_samples_in_window():
     s = _sampler([(0.0, 1965, 1965, 250.0, 0)], 1.0, 2.0).summary()
     assert s["reasons"] == ["unsampled"]
+
+
+def test_sample_file_location(tmp_path, monkeypatch):
+    """MLA_BENCH_CLOCKS_CSV names the sample file (rank appended); without it the samples go
+    to a temporary file that summary() removes."""
+    b = _bench()
+    monkeypatch.setenv("MLA_BENCH_CLOCKS_CSV", str(tmp_path / "clk.csv"))
+    monkeypatch.setenv("RANK", "3")
+    s = b.ClockSampler("0")
+    s.__enter__()
+    assert s.path == str(tmp_path / "clk_rank3.csv") and not s.tmp
+    s._stop()
+    monkeypatch.delenv("MLA_BENCH_CLOCKS_CSV")
+    s = b.ClockSampler("0")
+    s.__enter__()
+    assert s.tmp and s.path is not None
+    s._stop()
+    open(s.path, "a").close()            # as if the sampler had written it
+    s.kind, s.rows = "nvml", []
+    s.summary()
+    assert not os.path.exists(s.path)
+
+
+def test_traffic_is_keyed_to_the_kernel_source(tmp_path, monkeypatch):
+    """roofline.traffic comes from the committed record only while its source hash matches
+    the decode kernel's current sources; otherwise it is null."""
+    import json
+    b = _bench()
+    from mla_inputs import CONFIGS
+    cfg = CONFIGS["deepseek_v2"]
+    prof = tmp_path / "profiles"
+    prof.mkdir()
+    monkeypatch.setattr(b, "ROOT", str(tmp_path))
+    csrc = tmp_path / "head_latent_attention_attn_b200" / "csrc"
+    csrc.mkdir(parents=True)
+    for f in ("decode_pair.cu", "decode.cu", "decode_sched.cuh", "ptx.cuh", "kernels.h"):
+        (csrc / f).write_text(f"// {f}\n")
+    h = b._source_hash(cfg)
+    (prof / "decode_traffic.json").write_text(json.dumps(
+        {"deepseek_v2": {"source_hash": h, "dram_bytes_per_launch": 123}}))
+    assert b._traffic(cfg) == 123
+    (csrc / "decode_pair.cu").write_text("// changed\n")
+    assert b._traffic(cfg) is None
