@@ -264,6 +264,16 @@ def _traffic(cfg):
     return e.get("dram_bytes_per_launch")
 
 
+def max_over_ranks(values, dist, device):
+    """Element-wise maximum of `values` over all ranks (each rank's own list when `dist` is
+    None). Every rank must call it with the same length, in the same order."""
+    import torch
+    vec = torch.tensor([float(v) for v in values], dtype=torch.float64, device=device)
+    if dist is not None:
+        dist.all_reduce(vec, op=dist.ReduceOp.MAX)
+    return [float(x) for x in vec.tolist()]
+
+
 def cpu_oracle_sample(cfg, wl, budget_s=12.0, max_seqs=None):
     """Time the fp64 oracle on whole sequences of the workload until ``budget_s`` is spent."""
     import oracle.mla_oracle as O
@@ -427,10 +437,7 @@ def run_gpu(args, cfg, rank, world, dist):
     t_e2e = sum(e2e_ms) / len(e2e_ms)
 
     # ---- max over ranks -------------------------------------------------------------------
-    vec = torch.tensor([t_step, t_dec, t_e2e], dtype=torch.float64, device=dev)
-    if dist is not None:
-        dist.all_reduce(vec, op=dist.ReduceOp.MAX)
-    t_step, t_dec, t_e2e = [float(x) for x in vec.tolist()]
+    t_step, t_dec, t_e2e = max_over_ranks([t_step, t_dec, t_e2e], dist, dev)
     if rank != 0:
         return
     peaks = _peaks()
