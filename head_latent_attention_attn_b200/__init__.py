@@ -34,7 +34,7 @@ STATUS_NAMES = {0: "MLA_OK", 1: "MLA_ERR_INVALID_ARG", 2: "MLA_ERR_UNSUPPORTED",
 # Public C symbols (kept in sync with include/mla.h; a CPU test checks both ways).
 C_SYMBOLS = ("mla_row_width", "mla_status_string", "mla_cache_append", "mla_absorb_q",
              "mla_decode_workspace_size", "mla_decode_attn", "mla_out_up",
-             "mla_get_device_status", "mla_decode_attn_noalloc")
+             "mla_get_device_status", "mla_decode_attn_noalloc", "mla_selftest_wait_timeout")
 
 
 class MlaError(RuntimeError):
@@ -96,6 +96,8 @@ def lib() -> ctypes.CDLL:
     L.mla_decode_attn_noalloc.argtypes = [D, _P, _P, _I64, _P, _I32, _P, _I32, _I32, _I32, _I32,
                                           _P, _P, _P, _P]
     L.mla_decode_attn_noalloc.restype = _I32
+    L.mla_selftest_wait_timeout.argtypes = [_P, _P]
+    L.mla_selftest_wait_timeout.restype = _I32
     _lib = L
     return L
 
@@ -270,6 +272,14 @@ def mla_get_device_status(dev_error, reset: bool = False, stream=None) -> int:
     if dev_error.device.type != "cuda":
         raise MlaError("dev_error must be on a CUDA device", MLA_ERR_INVALID_ARG)
     return int(lib().mla_get_device_status(_ptr(dev_error), 1 if reset else 0, _stream(stream)))
+
+
+def mla_selftest_wait_timeout(dev_error, stream=None) -> None:
+    """Launch the device error path's self-test: a bounded wait that nothing completes, which
+    sets MLA_DEVERR_TIMEOUT in dev_error (an int32 CUDA tensor) after about 2 s."""
+    _need(dev_error, "dev_error", torch.int32)
+    _check(lib().mla_selftest_wait_timeout(_ptr(dev_error), _stream(stream)),
+           "mla_selftest_wait_timeout")
 
 
 def mla_decode_step(dims: MlaDims, *, c_kv_new, k_r_new, cos_new, sin_new, start_pos,

@@ -413,6 +413,11 @@ mla_status mla_decode_attn(const mla_dims* dims, const void* q_ext, const void* 
   return MLA_OK;
 }
 
+mla_status mla_selftest_wait_timeout(int32_t* dev_error, void* stream) {
+  if (!dev_error) return MLA_ERR_INVALID_ARG;
+  return launch_selftest_wait(dev_error, as_stream(stream)) == cudaSuccess ? MLA_OK : MLA_ERR_CUDA;
+}
+
 mla_status mla_get_device_status(const int32_t* dev_error, int32_t reset, void* stream) {
   if (!dev_error) return MLA_ERR_INVALID_ARG;
   cudaStream_t s = as_stream(stream);

@@ -222,6 +222,16 @@ mla_status mla_decode_attn_noalloc(const mla_dims* dims, const void* q_ext, cons
  */
 mla_status mla_get_device_status(const int32_t* dev_error, int32_t reset, void* stream);
 
+/*
+ * Self-test of the device error path. Launches one CTA on `stream` that waits on an
+ * mbarrier nothing arrives on, with the same bounded wait every kernel here uses (2 s).
+ * The wait gives up, ORs MLA_DEVERR_TIMEOUT into the caller's int32 error word `dev_error`
+ * and the kernel returns, so the context stays usable. Returns MLA_OK once launched
+ * (MLA_ERR_INVALID_ARG for a null word, MLA_ERR_CUDA if the launch fails); read the word
+ * with mla_get_device_status.
+ */
+mla_status mla_selftest_wait_timeout(int32_t* dev_error, void* stream);
+
 #ifdef __cplusplus
 }
 #endif
