@@ -7,10 +7,28 @@
 
 #include "host_common.h"
 #include "kernels.h"
+#include "ptx.cuh"
 
 using namespace mla;
 
 namespace {
+
+// Self-test of the device error path: one warp waits, with the bounded wait of every kernel
+// here, on an mbarrier that nothing arrives on; the wait gives up, sets the CTA's abort flag
+// and ORs MLA_DEVERR_TIMEOUT into the error word, and the kernel returns.
+__global__ void __launch_bounds__(32) mla_selftest_wait_kernel(int32_t* dev_error) {
+  __shared__ uint64_t bar;
+  __shared__ int abort_flag;
+  if (threadIdx.x == 0) {
+    mbar_init(&bar, 1);
+    abort_flag = 0;
+    fence_mbar_init();
+  }
+  __syncthreads();
+  const WaitCtx wc{&abort_flag, dev_error};
+  if (threadIdx.x == 0) (void)mbar_wait(&bar, 0, wc);   // phase 0 never completes
+  __syncthreads();
+}
 
 constexpr int kMaxSmem = 232448;  // 227 KB opt-in dynamic shared memory per CTA
 
@@ -415,7 +433,8 @@ mla_status mla_decode_attn(const mla_dims* dims, const void* q_ext, const void* 
 
 mla_status mla_selftest_wait_timeout(int32_t* dev_error, void* stream) {
   if (!dev_error) return MLA_ERR_INVALID_ARG;
-  return launch_selftest_wait(dev_error, as_stream(stream)) == cudaSuccess ? MLA_OK : MLA_ERR_CUDA;
+  mla_selftest_wait_kernel<<<1, 32, 0, as_stream(stream)>>>(dev_error);
+  return cudaGetLastError() == cudaSuccess ? MLA_OK : MLA_ERR_CUDA;
 }
 
 mla_status mla_get_device_status(const int32_t* dev_error, int32_t reset, void* stream) {

@@ -782,28 +782,6 @@ extern "C" int mla_trace_read(unsigned long long* host, int n) {
 }
 #endif
 
-// Self-test of the device error path: one warp waits, with the bounded wait of every kernel
-// here, on an mbarrier that nothing arrives on; the wait gives up, sets the CTA's abort flag
-// and ORs MLA_DEVERR_TIMEOUT into the error word, and the kernel returns.
-__global__ void __launch_bounds__(32) mla_selftest_wait_kernel(int32_t* dev_error) {
-  __shared__ uint64_t bar;
-  __shared__ int abort_flag;
-  if (threadIdx.x == 0) {
-    mbar_init(&bar, 1);
-    abort_flag = 0;
-    fence_mbar_init();
-  }
-  __syncthreads();
-  const WaitCtx wc{&abort_flag, dev_error};
-  if (threadIdx.x == 0) (void)mbar_wait(&bar, 0, wc);   // phase 0 never completes
-  __syncthreads();
-}
-
-cudaError_t launch_selftest_wait(int32_t* dev_error, cudaStream_t stream) {
-  mla_selftest_wait_kernel<<<1, 32, 0, stream>>>(dev_error);
-  return cudaGetLastError();
-}
-
 cudaError_t launch_combine(const CombineParams& p, cudaStream_t stream) {
   const int64_t rows = int64_t(p.units) * p.ncol;
   if (rows <= 0 || rows > 0x7fffffffLL || p.r > 512 || p.r % 4 != 0) return cudaErrorInvalidValue;

@@ -44,9 +44,6 @@ struct WGemmParams {
 // max_ctas: the persistent grid's size limit (one CTA per SM)
 cudaError_t launch_wgemm(const WGemmParams& p, int nr, int max_ctas, cudaStream_t stream);
 
-// The device error path's self-test (one bounded wait that nothing completes).
-cudaError_t launch_selftest_wait(int32_t* dev_error, cudaStream_t stream);
-
 // ---- mla_decode_attn -----------------------------------------------------------------------
 constexpr int kDecodeTok = 64;        // tokens per tile = one cache page
 constexpr int kDecodeMaxBlk = 10;     // D <= 640 -> at most 10 64-column blocks
