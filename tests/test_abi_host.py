@@ -141,6 +141,7 @@ def test_absorb_and_out_up_validation(mla_lib):
     st = L.mla_out_up(ctypes.byref(d), FAKE, FAKE, 128 * 512, None, 0, FAKE, None)
     assert st == mla.MLA_OK
     assert L.mla_get_device_status(None, 0, None) == mla.MLA_ERR_INVALID_ARG
+    assert L.mla_selftest_wait_timeout(None, None) == mla.MLA_ERR_INVALID_ARG   # no launch
 
 
 def test_binding_fails_loudly_without_library(monkeypatch, tmp_path):
