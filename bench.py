@@ -329,23 +329,70 @@ def _config_json(cfg):
             "parallelism": "replicas"}
 
 
+def roofline_of(cfg, seq_lens, t_ms, peaks):
+    """Roofline object of one mla_decode_attn launch of `t_ms` milliseconds."""
+    nbytes, flops = algorithmic_work(cfg, seq_lens)
+    gbs = nbytes / (t_ms * 1e-3) / 1e9
+    tfl = flops / (t_ms * 1e-3) / 1e12
+    t_hbm = nbytes / (peaks["hbm_gbs"] * 1e9)
+    t_tc = flops / (peaks["bf16_tflops"] * 1e12)
+    if t_hbm >= t_tc:
+        roof = {"bound": "hbm", "achieved": gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                "frac": gbs / peaks["hbm_gbs"]}
+    else:
+        roof = {"bound": "tensor", "achieved": tfl, "peak": peaks["bf16_tflops"],
+                "unit": "TFLOP/s", "frac": tfl / peaks["bf16_tflops"]}
+    roof.update({"traffic": _traffic(cfg), "peak_source": peaks["source"],
+                 "kernel": decode_kernel_name(cfg) + " (+ merge of cut units when the work is split)",
+                 "algorithmic_bytes_per_launch": nbytes, "algorithmic_flops_per_launch": flops,
+                 "achieved_gbs": gbs, "achieved_tflops": tfl,
+                 "roofline_time_us": 1e6 * max(t_hbm, t_tc),
+                 "pct_of_roofline": 100.0 * max(t_hbm, t_tc) / (t_ms * 1e-3)})
+    return roof
+
+
+def time_decode(prob, cfg, n, stream, flush=None):
+    """Per-launch times (ms) of `n` back-to-back mla_decode_attn calls, CUDA events on the
+    launching stream; an L2 flush between launches when `flush` is given."""
+    import torch
+
+    import head_latent_attention_attn_b200 as mla
+    evs = []
+    for _ in range(n):
+        if flush is not None:
+            flush.zero_()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        mla.mla_decode_attn(prob.dims, prob.q_ext, prob.cache, prob.block_table, prob.seq_lens,
+                            prob.max_seq_len, prob.workspace, prob.o_latent, prob.lse,
+                            causal=cfg.causal, num_splits=prob.num_splits, stream=stream)
+        b.record(stream)
+        evs.append((a, b))
+    torch.cuda.synchronize()
+    return [a.elapsed_time(b) for a, b in evs]
+
+
+# Workloads timed after the headline in the default run: every other decode shape.
+PER_CONFIG = ("tiny", "qwen25_7b", "qwen3_30b_a3b", "hybrid_1m_q1", "hybrid_1m_q4",
+              "hybrid_256k_q1", "hybrid_256k_q4")
+DECODE_BLOCK = 60   # decode launches timed back to back for the roofline figure
+
+
 def run_gpu(args, cfg, rank, world, dist):
     import torch
 
     import head_latent_attention_attn_b200 as mla
-    from mla_inputs import make_workload
-    sys.path.insert(0, os.path.join(ROOT, "tests"))
-    from tests.gpu_harness import GpuProblem
+    from mla_inputs import CONFIGS, make_workload
+    from mla_inputs.device import DeviceProblem
 
     local = int(os.environ.get("LOCAL_RANK", "0"))
     torch.cuda.set_device(local)
     dev = torch.device("cuda", local)
     mla.lib()
     wl = make_workload(cfg)
-    prob = GpuProblem(wl, num_splits=args.splits, device=str(dev))
+    prob = DeviceProblem(wl, num_splits=args.splits, device=str(dev))
     stream = torch.cuda.current_stream()
-    nbytes, flops = algorithmic_work(cfg, wl.seq_lens)
-    cache_bytes = nbytes
+    cache_bytes, _ = algorithmic_work(cfg, wl.seq_lens)
     flush = None
     if cache_bytes < 2 * L2_BYTES:
         flush = torch.empty(4 * L2_BYTES // 4, dtype=torch.float32, device=dev)
@@ -377,6 +424,7 @@ def run_gpu(args, cfg, rank, world, dist):
         if flush is not None:
             flush.zero_()
         one_step(mk())
+    time_decode(prob, cfg, 3, stream, flush)
     barrier()
     evs = []
     with ClockSampler(_gpu_id(local)) as clk:
@@ -388,100 +436,157 @@ def run_gpu(args, cfg, rank, world, dist):
             e = mk()
             one_step(e)
             evs.append(e)
+        # the decode alone, back to back: the roofline figure (median of DECODE_BLOCK launches)
+        dec_block = time_decode(prob, cfg, DECODE_BLOCK, stream, flush)
         barrier()
         clk.mark_end()
     step_ms = [e[0].elapsed_time(e[3]) for e in evs]
     dec_ms = [e[1].elapsed_time(e[2]) for e in evs]
-    t_step = sum(step_ms) / len(step_ms)
-    t_dec = sum(dec_ms) / len(dec_ms)
+    t_step = statistics.mean(step_ms)
+    t_dec_step = statistics.mean(dec_ms)
+    t_dec = statistics.median(dec_block)
+    t_dec_mean = statistics.mean(dec_block)
     status = mla.mla_get_device_status(prob.workspace.view(torch.int32)[:1])
     if status != mla.MLA_OK:
         raise RuntimeError(f"device error word set: {mla.STATUS_NAMES[status]}")
 
     # ---- end to end through the public API with pinned host buffers ------------------------
-    host_in = {k: getattr(prob, k).detach().cpu().pin_memory()
-               for k in ("c_new", "k_new", "cos_q", "sin_q", "start_pos", "q_nope", "q_pe")}
-    host_o = torch.empty(prob.o.shape, dtype=prob.o.dtype).pin_memory()
-    host_lse = torch.empty(prob.lse.shape, dtype=prob.lse.dtype).pin_memory()
-    h2d = sum(t.numel() * t.element_size() for t in host_in.values())
-    d2h = host_o.numel() * host_o.element_size() + host_lse.numel() * host_lse.element_size()
+    # Every step copies its inputs from pinned host memory and reads its outputs back. Two
+    # buffer sets and three streams let step k's host->device copy, step k-1's compute and
+    # step k-2's device->host copy run at once, as a serving loop would.
+    in_names = ("c_new", "k_new", "cos_q", "sin_q", "start_pos", "q_nope", "q_pe")
+    host_in = [{k: getattr(prob, k).detach().cpu().pin_memory() for k in in_names}
+               for _ in range(2)]
+    dev_in = [{k: getattr(prob, k) for k in in_names},
+              {k: torch.empty_like(getattr(prob, k)) for k in in_names}]
+    dev_o = [prob.o, torch.empty_like(prob.o)]
+    dev_lse = [prob.lse, torch.empty_like(prob.lse)]
+    host_o = [torch.empty(prob.o.shape, dtype=prob.o.dtype).pin_memory() for _ in range(2)]
+    host_lse = [torch.empty(prob.lse.shape, dtype=prob.lse.dtype).pin_memory() for _ in range(2)]
+    h2d = sum(t.numel() * t.element_size() for t in host_in[0].values())
+    d2h = host_o[0].numel() * host_o[0].element_size() + host_lse[0].numel() * host_lse[0].element_size()
+    s_h2d, s_d2h = torch.cuda.Stream(), torch.cuda.Stream()
+    ev_in = [torch.cuda.Event() for _ in range(2)]      # inputs of a set copied in
+    ev_comp = [torch.cuda.Event() for _ in range(2)]    # a set's step computed
+    ev_out = [torch.cuda.Event() for _ in range(2)]     # a set's outputs copied out
 
-    def e2e_step():
-        for k, t in host_in.items():
-            getattr(prob, k).copy_(t, non_blocking=True)
-        mla.mla_decode_step(prob.dims, c_kv_new=prob.c_new, k_r_new=prob.k_new,
-                            cos_new=prob.cos_q, sin_new=prob.sin_q, start_pos=prob.start_pos,
-                            q_nope=prob.q_nope, q_pe=prob.q_pe, cos_q=prob.cos_q, sin_q=prob.sin_q,
-                            w_uk=prob.w_uk, w_uv=prob.w_uv, bias=prob.bias, cache=prob.cache,
-                            block_table=prob.block_table, seq_lens=prob.seq_lens,
-                            max_seq_len=prob.max_seq_len, q_ext=prob.q_ext,
-                            workspace=prob.workspace, o_latent=prob.o_latent, lse=prob.lse,
-                            o=prob.o, causal=cfg.causal, num_splits=args.splits, stream=stream)
-        host_o.copy_(prob.o, non_blocking=True)
-        host_lse.copy_(prob.lse, non_blocking=True)
+    def e2e_steps(n):
+        for k in range(n):
+            s = k % 2
+            with torch.cuda.stream(s_h2d):
+                s_h2d.wait_event(ev_comp[s])            # step k-2 finished reading the set
+                for name in in_names:
+                    dev_in[s][name].copy_(host_in[s][name], non_blocking=True)
+                ev_in[s].record(s_h2d)
+            stream.wait_event(ev_in[s])
+            stream.wait_event(ev_out[s])                # step k-2's outputs already read back
+            d = dev_in[s]
+            mla.mla_decode_step(prob.dims, c_kv_new=d["c_new"], k_r_new=d["k_new"],
+                                cos_new=d["cos_q"], sin_new=d["sin_q"], start_pos=d["start_pos"],
+                                q_nope=d["q_nope"], q_pe=d["q_pe"], cos_q=d["cos_q"],
+                                sin_q=d["sin_q"], w_uk=prob.w_uk, w_uv=prob.w_uv, bias=prob.bias,
+                                cache=prob.cache, block_table=prob.block_table,
+                                seq_lens=prob.seq_lens, max_seq_len=prob.max_seq_len,
+                                q_ext=prob.q_ext, workspace=prob.workspace,
+                                o_latent=prob.o_latent, lse=dev_lse[s], o=dev_o[s],
+                                causal=cfg.causal, num_splits=args.splits, stream=stream)
+            ev_comp[s].record(stream)
+            with torch.cuda.stream(s_d2h):
+                s_d2h.wait_event(ev_comp[s])
+                host_o[s].copy_(dev_o[s], non_blocking=True)
+                host_lse[s].copy_(dev_lse[s], non_blocking=True)
+                ev_out[s].record(s_d2h)
 
-    for _ in range(args.warmup):
-        e2e_step()
+    for e in ev_comp + ev_out:
+        e.record(stream)
+    e2e_steps(max(args.warmup, 2))
     barrier()
-    e2e_ms = []
-    for _ in range(args.steps):
-        if flush is not None:
-            flush.zero_()
-        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        a.record(stream)
-        e2e_step()
-        b.record(stream)
-        b.synchronize()
-        e2e_ms.append(a.elapsed_time(b))
+    t0 = torch.cuda.Event(enable_timing=True)
+    t1 = torch.cuda.Event(enable_timing=True)
+    t0.record(s_h2d)
+    e2e_steps(args.steps)
+    t1.record(s_d2h)       # after the last read-back in stream order
     barrier()
-    t_e2e = sum(e2e_ms) / len(e2e_ms)
+    t_e2e = t0.elapsed_time(t1) / args.steps
+    # the outputs read back match the device-resident step's
+    if not (torch.equal(host_o[0], prob.o.cpu()) and torch.equal(host_lse[0], prob.lse.cpu())):
+        raise RuntimeError("end-to-end outputs differ from the device-resident step")
 
     # ---- max over ranks -------------------------------------------------------------------
-    t_step, t_dec, t_e2e = max_over_ranks([t_step, t_dec, t_e2e], dist, dev)
-    if rank != 0:
-        return
+    t_step, t_dec, t_dec_mean, t_dec_step, t_e2e = max_over_ranks(
+        [t_step, t_dec, t_dec_mean, t_dec_step, t_e2e], dist, dev)
     peaks = _peaks()
     tokens = cfg.batch * cfg.q_len
     value = world * tokens / (t_step * 1e-3)
-    gbs = nbytes / (t_dec * 1e-3) / 1e9
-    tfl = flops / (t_dec * 1e-3) / 1e12
-    t_hbm = nbytes / (peaks["hbm_gbs"] * 1e9)
-    t_tc = flops / (peaks["bf16_tflops"] * 1e12)
-    bound = "hbm" if t_hbm >= t_tc else "tensor"
-    if bound == "hbm":
-        roof = {"bound": "hbm", "achieved": gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
-                "frac": gbs / peaks["hbm_gbs"]}
-    else:
-        roof = {"bound": "tensor", "achieved": tfl, "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
-                "frac": tfl / peaks["bf16_tflops"]}
-    roof["traffic"] = _traffic(cfg)
-    roof["peak_source"] = peaks["source"]
-    roof["kernel"] = decode_kernel_name(cfg) + " (+ merge of cut units when the work is split)"
-    roof["algorithmic_bytes_per_launch"] = nbytes
-    roof["algorithmic_flops_per_launch"] = flops
-    roof["roofline_time_us"] = 1e6 * max(t_hbm, t_tc)
-    roof["pct_of_roofline"] = 100.0 * max(t_hbm, t_tc) / (t_dec * 1e-3)
+    roof = roofline_of(cfg, wl.seq_lens, t_dec, peaks)
     # append, absorb, decode, out_up (+ the split combine when the plan has > 1 split;
     # a one-split plan needs only the 256-byte error-word workspace)
-    launches_per_step = 4 + (1 if plan_splits_ws > 256 else 0)
+    merge = 1 if plan_splits_ws > 256 else 0
+    launches = (4 + merge) * args.steps + (1 + merge) * DECODE_BLOCK
     line = {
         "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": t_step,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
         "data": "synthetic",
         "config": dict(_config_json(cfg), l2=("cache > L2, no flush" if flush is None
-                                              else "L2 flushed between steps (512 MB write)")),
-        "decode_us": 1e3 * t_dec, "decode_gbs": gbs, "decode_tflops": tfl,
+                                              else "L2 flushed between launches (504 MB write)")),
+        "decode_us": 1e3 * t_dec, "decode_us_mean": 1e3 * t_dec_mean,
+        "decode_launches_timed": DECODE_BLOCK, "decode_us_in_step_mean": 1e3 * t_dec_step,
+        "decode_gbs": roof["achieved_gbs"], "decode_tflops": roof["achieved_tflops"],
         "roofline": roof,
         "e2e": {"value": world * tokens / (t_e2e * 1e-3), "unit": "tokens/s",
                 "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
-                "ms_per_step": t_e2e},
-        "gpu_launches": launches_per_step * args.steps,
+                "ms_per_step": t_e2e,
+                "method": "pinned host inputs copied in and outputs read back every step; "
+                          "copies of neighbouring steps overlap the compute on separate streams"},
+        "gpu_launches": launches,
         "clocks": clk.summary(),
     }
+    del prob, flush
+    torch.cuda.empty_cache()
+    if not args.no_per_config:
+        line["per_config"] = per_config_block(args, cfg, dev, stream, dist, peaks)
+    if rank != 0:
+        return
     if world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_oracle_sample(cfg, wl, budget_s=args.cpu_budget)
     print(json.dumps(line), flush=True)
+
+
+def per_config_block(args, head_cfg, dev, stream, dist, peaks):
+    """mla_decode_attn on every other decode workload, in the same process: the median of
+    DECODE_BLOCK launches, its roofline and the clocks seen while it ran. Every rank runs
+    the same workloads (the timings are maxed over ranks)."""
+    import torch
+
+    from mla_inputs import CONFIGS, make_workload
+    from mla_inputs.device import DeviceProblem
+    out = {}
+    for name in PER_CONFIG:
+        if name == head_cfg.name:
+            continue
+        cfg = CONFIGS[name]
+        wl = make_workload(cfg)
+        prob = DeviceProblem(wl, device=str(dev))
+        prob.step()
+        nbytes, _ = algorithmic_work(cfg, wl.seq_lens)
+        flush = (torch.empty(4 * L2_BYTES // 4, dtype=torch.float32, device=dev)
+                 if nbytes < 2 * L2_BYTES else None)
+        time_decode(prob, cfg, 3, stream, flush)
+        with ClockSampler(_gpu_id(dev.index or 0)) as clk:
+            clk.mark_start()
+            ms = time_decode(prob, cfg, DECODE_BLOCK, stream, flush)
+            clk.mark_end()
+        t_med, t_mean = max_over_ranks([statistics.median(ms), statistics.mean(ms)], dist, dev)
+        out[name] = {"decode_us": 1e3 * t_med, "decode_us_mean": 1e3 * t_mean,
+                     "launches": DECODE_BLOCK,
+                     "tokens_per_s": cfg.batch * cfg.q_len / (t_med * 1e-3),
+                     "roofline": roofline_of(cfg, wl.seq_lens, t_med, peaks),
+                     "l2": "cache > L2, no flush" if flush is None else "L2 flushed between launches",
+                     "clocks": clk.summary()}
+        del prob, flush, wl
+        torch.cuda.empty_cache()
+    return out
 
 
 def _gpu_id(local: int) -> str:
@@ -503,6 +608,8 @@ def main():
     ap.add_argument("--splits", type=int, default=0, help="KV splits per sequence (0 = auto)")
     ap.add_argument("--cpu-budget", type=float, default=12.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-per-config", action="store_true",
+                    help="time only the headline workload")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
 

@@ -65,9 +65,10 @@ extern "C" mla_status mla_decode_attn(const mla_dims*, const void*, const void*,
                                       void*);
 
 // The decode of mla_decode_attn with its workspace carved out of the fixed scratch array.
-// The number of work ranges is the largest one (at most one per SM) whose partial results
-// fit in the scratch; a problem that does not fit even with one range per (sequence, row
-// block) is rejected with MLA_ERR_WORKSPACE before anything is launched.
+// The automatic plan is used: it has at most one work range per SM, and no explicit split
+// count gives fewer ranges once there are more (sequence, row block) units than SMs, so a
+// problem whose automatic plan does not fit is rejected with MLA_ERR_WORKSPACE before
+// anything is launched.
 extern "C" mla_status mla_decode_attn_noalloc(const mla_dims* dims, const void* q_ext,
                                               const void* cache, int64_t num_pages,
                                               const int32_t* block_table,
@@ -77,39 +78,30 @@ extern "C" mla_status mla_decode_attn_noalloc(const mla_dims* dims, const void* 
                                               int32_t* dev_error, void* o_latent, float* lse,
                                               void* stream) {
   if (dev_error == nullptr) return MLA_ERR_INVALID_ARG;
-  if (batch == 0) return MLA_OK;
-  // Largest grid (ranges per unit, as in mla_decode_attn's num_splits) that fits.
-  const size_t auto_ws = mla_decode_workspace_size(dims, batch, q_len, max_seq_len, 0);
-  if (auto_ws == 0) {
-    // invalid or unsupported problem: report what mla_decode_attn's validation reports
-    // (it fails before looking at the workspace, so nothing is launched)
+  const size_t need = mla_decode_workspace_size(dims, batch, q_len, max_seq_len, 0);
+  if (need == 0 || batch == 0) {
+    // invalid or unsupported problem, or nothing to do: report what mla_decode_attn's
+    // validation reports (it returns before looking at the workspace and launches nothing)
     return mla_decode_attn(dims, q_ext, cache, num_pages, block_table, max_pages_per_seq,
                            seq_lens, batch, q_len, max_seq_len, causal, 0, nullptr, 0, o_latent,
                            lse, stream);
   }
-  int32_t splits = 0;
-  size_t need = auto_ws;
-  if (need > kScratchBytes) {
-    splits = -1;
-    for (int32_t s = 1; s <= 64; ++s) {
-      const size_t w = mla_decode_workspace_size(dims, batch, q_len, max_seq_len, s);
-      if (w == 0 || w > kScratchBytes) break;
-      splits = s;
-      need = w;
-    }
-    if (splits < 0) return MLA_ERR_WORKSPACE;
-  }
+  if (need > kScratchBytes) return MLA_ERR_WORKSPACE;
   void* scratch = nullptr;
   mla_status st = scratch_address(&scratch);
   if (st != MLA_OK) return st;
   // The scratch is used exactly like a workspace: its first int32 is the decode's error
-  // word (cleared by every call below), the rest is fully rewritten by every call.
+  // word, the rest is fully rewritten by every call.
   unsigned char* ws = static_cast<unsigned char*>(scratch);
   st = mla_decode_attn(dims, q_ext, cache, num_pages, block_table, max_pages_per_seq, seq_lens,
-                       batch, q_len, max_seq_len, causal, splits, ws, round256(need), o_latent,
-                       lse, stream);
-  if (st != MLA_OK) return st;
+                       batch, q_len, max_seq_len, causal, 0, ws, round256(need), o_latent, lse,
+                       stream);
+  if (st != MLA_OK && st != MLA_ERR_CUDA) return st;   // rejected before any launch
+  // After any launch (even one followed by a failed launch) move the bits the decode left in
+  // the scratch's error word into the caller's word and clear it, so no call inherits them.
   fold_error_word<<<1, 1, 0, static_cast<cudaStream_t>(stream)>>>(reinterpret_cast<int32_t*>(ws),
                                                                   dev_error);
-  return cudaGetLastError() == cudaSuccess ? MLA_OK : MLA_ERR_CUDA;
+  const cudaError_t le = cudaGetLastError();
+  if (st != MLA_OK) return st;
+  return le == cudaSuccess ? MLA_OK : MLA_ERR_CUDA;
 }

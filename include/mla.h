@@ -202,9 +202,12 @@ mla_status mla_out_up(const mla_dims* dims, const void* o_latent, const void* w_
  *   rewrites what it reads, so nothing has to be cleared between calls. Calls whose
  *   execution overlaps on the GPU (different streams, or different host threads without
  *   ordering) race on the array and must not be used.
- * - The number of work ranges is the largest that fits in the array (at most one per SM);
- *   a problem whose partial results cannot fit even with one range per (sequence, block of
- *   query rows) returns MLA_ERR_WORKSPACE and launches nothing.
+ * - The call uses mla_decode_attn's automatic plan (num_splits = 0: at most one work range
+ *   per SM), which needs the least workspace of all plans once there are more (sequence,
+ *   block of query rows) units than SMs, and fits the array whenever there are fewer. A
+ *   problem whose plan does not fit (millions of sequences, or many more row blocks than
+ *   SMs) returns MLA_ERR_WORKSPACE and launches nothing.
+ * - Validation is that of mla_decode_attn, done before anything else (batch == 0 included).
  */
 #define MLA_NOALLOC_SCRATCH_BYTES ((size_t)32 << 20)
 mla_status mla_decode_attn_noalloc(const mla_dims* dims, const void* q_ext, const void* cache,

@@ -48,6 +48,7 @@ class MLAConfig:
     rope_ref_dim: int = 0      # denominator of the RoPE frequency exponent
     rope_index_pool: int = 0   # > 0: per-group frequency indices drawn from range(pool)
     with_bias: bool = False    # W_UV bias (the up_v.bias of the MLAfied checkpoints)
+    identity_weights: bool = False   # W_UK = W_UV = I (needs d_n = d_v = r): plain MQA on c_kv
 
     @property
     def row_width(self) -> int:

@@ -11,6 +11,7 @@ Recipe (all drawn in fp32 from ``torch.Generator('cpu')`` and rounded to bf16):
   from its own generator, so any one sequence can be rebuilt without the others;
 * token l of a sequence sits at position l; query row i of sequence b sits at
   position L_b - q + i (the last q tokens are the ones appended in the decode step);
+* ``identity_weights`` replaces W_UK and W_UV by identity matrices (drawn values unused);
 * RoPE frequencies are theta[g, j] = base ** (-2 * idx[g, j] / ref_dim); cos/sin
   tables handed to the GPU are the fp64 cosine/sine of theta * position rounded
   to fp32.
@@ -132,6 +133,11 @@ def make_workload(cfg: MLAConfig, q_scale: float = 1.0, spare_pages: int = 0,
 
     w_uk = _randn(gen, (H, dn, r), r)
     w_uv = _randn(gen, (H, dv, r), r)
+    if cfg.identity_weights:
+        # the special case in which the method is multi-query attention over c_kv itself
+        assert dn == r and dv == r, "identity weights need d_n = d_v = r"
+        w_uk = torch.eye(r, dtype=torch.bfloat16).expand(H, r, r).contiguous()
+        w_uv = w_uk.clone()
     bias = _randn(gen, (H, dv), dv) if cfg.with_bias else None
     qn = torch.randn(B, q, H, dn, generator=gen, dtype=torch.float32) / math.sqrt(dn)
     qp = torch.randn(B, q, H, dr, generator=gen, dtype=torch.float32) / math.sqrt(max(dr, 1))

@@ -149,3 +149,28 @@ def test_binding_fails_loudly_without_library(monkeypatch, tmp_path):
     monkeypatch.setattr(mla, "LIB_PATH", str(tmp_path / "libmla.so"))
     with pytest.raises(mla.MlaError):
         mla.lib()
+
+
+def _noalloc(d, **kw):
+    a = dict(q=FAKE, cache=FAKE, npages=100000, table=FAKE, maxp=4, lens=FAKE, batch=2, qlen=1,
+             maxlen=256, causal=1, err=FAKE, o=FAKE, lse=FAKE)
+    a.update(kw)
+    return mla.lib().mla_decode_attn_noalloc(ctypes.byref(d), a["q"], a["cache"], a["npages"],
+                                             a["table"], a["maxp"], a["lens"], a["batch"],
+                                             a["qlen"], a["maxlen"], a["causal"], a["err"],
+                                             a["o"], a["lse"], None)
+
+
+def test_noalloc_validation_before_launch(mla_lib):
+    """The no-allocation decode validates exactly like mla_decode_attn, batch 0 included,
+    and refuses a plan larger than its scratch array before any launch or CUDA call."""
+    assert _noalloc(_dims(), err=None) == mla.MLA_ERR_INVALID_ARG      # error word required
+    assert _noalloc(_dims(page_size=32), batch=0) == mla.MLA_ERR_UNSUPPORTED
+    assert _noalloc(_dims(), batch=0, causal=2) == mla.MLA_ERR_INVALID_ARG
+    assert _noalloc(_dims(), batch=0, qlen=0) == mla.MLA_ERR_INVALID_ARG
+    assert _noalloc(_dims(), batch=0) == mla.MLA_OK                     # valid, nothing to do
+    # four million one-page sequences: the per-sequence schedule alone is 16 MB and the
+    # automatic plan (the smallest one) no longer fits the 32 MiB array
+    d = _dims()
+    assert mla.mla_decode_workspace_size(d, 4_000_000, 1, 64, 0) > 32 << 20
+    assert _noalloc(d, batch=4_000_000, maxlen=64, maxp=1) == mla.MLA_ERR_WORKSPACE

@@ -48,14 +48,20 @@ def test_noalloc_matches_workspace_decode(name):
         assert max_rel_err(got_o, ref_o) <= O_TOL, f"call {call}: o_latent differs"
         assert float(np.max(np.abs(got_l - ref_l))) <= LSE_TOL, f"call {call}: lse differs"
     assert mla.mla_get_device_status(err) == mla.MLA_OK
+    # and the no-allocation output against the fp64 oracle itself, sequence by sequence
+    for b in range(cfg.batch):
+        ref = prob.oracle(b)
+        assert max_rel_err(o[b].float().cpu().numpy(), ref["o_latent"]) <= O_TOL, f"seq {b}"
+        assert float(np.max(np.abs(lse[b].cpu().numpy() - ref["lse"]))) <= LSE_TOL, f"seq {b}"
 
 
 def test_noalloc_refusals_launch_nothing():
     """Host-side refusals of the no-allocation decode: an unsupported page size and a
     missing error word are rejected before anything is launched (the pointers here are not
     device memory, so only calls that return before a launch may use them). The automatic
-    plan of the largest supported shapes fits the scratch: with bf16 partial outputs a plan
-    holds at most 148 ranges x 2 slots x 128 rows x 512 bf16 = 19.4 MB of partials."""
+    plan of the benchmark shapes fits the scratch: with bf16 partial outputs it holds at
+    most 148 one-CTA ranges of up to 64 rows, or 74 two-CTA ranges of 128 rows, each
+    x 2 slots x r <= 512 bf16 = 19.4 MB of partials, plus 4 bytes per sequence."""
     cfg = CONFIGS["deepseek_v2"]
     dims = dims_of(cfg)
     fake = ctypes.c_void_p(0x10000)
