@@ -34,7 +34,9 @@ STATUS_NAMES = {0: "MLA_OK", 1: "MLA_ERR_INVALID_ARG", 2: "MLA_ERR_UNSUPPORTED",
 # Public C symbols (kept in sync with include/mla.h; a CPU test checks both ways).
 C_SYMBOLS = ("mla_row_width", "mla_status_string", "mla_cache_append", "mla_absorb_q",
              "mla_decode_workspace_size", "mla_decode_attn", "mla_out_up",
-             "mla_get_device_status", "mla_decode_attn_noalloc", "mla_selftest_wait_timeout")
+             "mla_get_device_status", "mla_decode_attn_noalloc", "mla_selftest_wait_timeout",
+             "mla_kv_shared_decode_dims", "mla_kv_shared_query", "mla_kv_shared_output",
+             "mla_down_kv_append")
 
 
 class MlaError(RuntimeError):
@@ -98,6 +100,14 @@ def lib() -> ctypes.CDLL:
     L.mla_decode_attn_noalloc.restype = _I32
     L.mla_selftest_wait_timeout.argtypes = [_P, _P]
     L.mla_selftest_wait_timeout.restype = _I32
+    L.mla_kv_shared_decode_dims.argtypes = [D, D]
+    L.mla_kv_shared_decode_dims.restype = _I32
+    for fn in (L.mla_kv_shared_query, L.mla_kv_shared_output):
+        fn.argtypes = [D, _P, _P, _P, _I32, _I32, _P, _P]
+        fn.restype = _I32
+    L.mla_down_kv_append.argtypes = [D, _P, _I32, _P, _P, _P, _P, _I32, _P, _I32, _I32, _P,
+                                     _I64, _P, _P, _P]
+    L.mla_down_kv_append.restype = _I32
     _lib = L
     return L
 
@@ -162,6 +172,37 @@ def mla_cache_append(dims: MlaDims, c_kv, k_r, rope_cos, rope_sin, block_table, 
                                 block_table.shape[1], _ptr(start_pos), B, n, _ptr(cache),
                                 cache.shape[0], _ptr(dev_error), _stream(stream))
     _check(st, "mla_cache_append")
+
+
+def mla_down_kv_append(dims: MlaDims, hidden, w_dkv, rope_cos, rope_sin, block_table,
+                       start_pos, cache, dev_error=None, kv_out=None, stream=None) -> None:
+    """[c_kv ; k_r] = w_dkv @ hidden (bf16) for hidden [B, n, hidden_dim], written into cache
+    [P, ps, D] exactly as mla_cache_append would; kv_out [B, n, D] optionally receives the
+    projection before the rotation."""
+    B, n, hid = hidden.shape
+    G, dr, D = dims.num_kv_groups, dims.rope_dim, dims.row_width
+    _need(hidden, "hidden", torch.bfloat16)
+    _need(w_dkv, "w_dkv", torch.bfloat16, (D, hid))
+    if dr > 0:
+        _need(rope_cos, "rope_cos", torch.float32, (B, n, G, dr // 2))
+        _need(rope_sin, "rope_sin", torch.float32, (B, n, G, dr // 2))
+    _need(block_table, "block_table", torch.int32)
+    _need(start_pos, "start_pos", torch.int32, (B,))
+    _need(cache, "cache", torch.bfloat16)
+    if cache.dim() != 3 or cache.shape[1] != dims.page_size or cache.shape[2] != D:
+        raise MlaError(f"cache shape {tuple(cache.shape)} does not match dims", MLA_ERR_INVALID_ARG)
+    if block_table.dim() != 2 or block_table.shape[0] != B:
+        raise MlaError("block_table must be [B, max_pages]", MLA_ERR_INVALID_ARG)
+    if dev_error is not None:
+        _need(dev_error, "dev_error", torch.int32)
+    if kv_out is not None:
+        _need(kv_out, "kv_out", torch.bfloat16, (B, n, D))
+    st = lib().mla_down_kv_append(ctypes.byref(dims), _ptr(hidden), hid, _ptr(w_dkv),
+                                  _ptr(rope_cos if dr > 0 else None),
+                                  _ptr(rope_sin if dr > 0 else None), _ptr(block_table),
+                                  block_table.shape[1], _ptr(start_pos), B, n, _ptr(cache),
+                                  cache.shape[0], _ptr(dev_error), _ptr(kv_out), _stream(stream))
+    _check(st, "mla_down_kv_append")
 
 
 def mla_absorb_q(dims: MlaDims, q_nope, q_pe, rope_cos, rope_sin, w_uk, q_ext,
@@ -267,6 +308,38 @@ def mla_out_up(dims: MlaDims, o_latent, w_uv, o, bias=None,
     _check(st, "mla_out_up")
 
 
+def mla_kv_shared_decode_dims(dims: MlaDims) -> MlaDims:
+    """Decode view of a K = V layout: the whole cache row is the latent (rank D, no rotary
+    slot), so mla_decode_attn with these dims returns o_latent = sum_l p_l row_l."""
+    out = MlaDims()
+    _check(lib().mla_kv_shared_decode_dims(ctypes.byref(dims), ctypes.byref(out)),
+           "mla_kv_shared_decode_dims")
+    return out
+
+
+def _kv_shared_rotate(fn, what, dims: MlaDims, x, rope_cos, rope_sin, out, stream) -> None:
+    B, q = x.shape[0], x.shape[1]
+    D = dims.row_width
+    _need(x, what + " input", torch.bfloat16, (B, q, dims.num_heads, D))
+    _need(out, what + " output", torch.bfloat16, (B, q, dims.num_heads, D))
+    _need(rope_cos, "rope_cos", torch.float32, (B, q, 1, dims.rope_dim // 2))
+    _need(rope_sin, "rope_sin", torch.float32, (B, q, 1, dims.rope_dim // 2))
+    _check(fn(ctypes.byref(dims), _ptr(x), _ptr(rope_cos), _ptr(rope_sin), B, q, _ptr(out),
+              _stream(stream)), what)
+
+
+def mla_kv_shared_query(dims: MlaDims, q, rope_cos, rope_sin, q_ext, stream=None) -> None:
+    """q_ext [B, q, H, D] = q with its last d_r dims rotated to the query positions."""
+    _kv_shared_rotate(lib().mla_kv_shared_query, "mla_kv_shared_query", dims, q, rope_cos,
+                      rope_sin, q_ext, stream)
+
+
+def mla_kv_shared_output(dims: MlaDims, o_latent, rope_cos, rope_sin, o, stream=None) -> None:
+    """o [B, q, H, D] = o_latent with its last d_r dims rotated back from the query positions."""
+    _kv_shared_rotate(lib().mla_kv_shared_output, "mla_kv_shared_output", dims, o_latent,
+                      rope_cos, rope_sin, o, stream)
+
+
 def mla_get_device_status(dev_error, reset: bool = False, stream=None) -> int:
     """Synchronise and read a device error word (an int32 tensor, or a decode workspace)."""
     if dev_error.device.type != "cuda":
@@ -297,5 +370,5 @@ def mla_decode_step(dims: MlaDims, *, c_kv_new, k_r_new, cos_new, sin_new, start
 
 __all__ = ["MlaDims", "MlaError", "make_dims", "lib", "mla_row_width", "mla_cache_append",
            "mla_absorb_q", "mla_decode_workspace_size", "mla_decode_attn", "mla_out_up",
-           "mla_decode_attn_noalloc",
-           "mla_get_device_status", "mla_decode_step", "C_SYMBOLS", "STATUS_NAMES"]
+           "mla_decode_attn_noalloc", "mla_kv_shared_decode_dims", "mla_kv_shared_query",
+           "mla_kv_shared_output", "mla_down_kv_append", "mla_get_device_status", "mla_decode_step", "C_SYMBOLS", "STATUS_NAMES"]

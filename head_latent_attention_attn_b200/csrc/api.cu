@@ -321,6 +321,69 @@ mla_status mla_out_up(const mla_dims* dims, const void* o_latent, const void* w_
   return launch_wgemm(p, nr, num_sms(), as_stream(stream)) == cudaSuccess ? MLA_OK : MLA_ERR_CUDA;
 }
 
+mla_status mla_down_kv_append(const mla_dims* dims, const void* hidden, int32_t hidden_dim,
+                              const void* w_dkv, const float* rope_cos, const float* rope_sin,
+                              const int32_t* block_table, int32_t max_pages_per_seq,
+                              const int32_t* start_pos, int32_t batch, int32_t n_new, void* cache,
+                              int64_t num_pages, int32_t* dev_error, void* kv_out, void* stream) {
+  mla_status st = check_dims(dims);
+  if (st != MLA_OK) return st;
+  if (batch < 0 || n_new < 0 || hidden_dim <= 0 || hidden_dim % 8 != 0 ||
+      max_pages_per_seq <= 0 || num_pages <= 0 || num_pages > INT32_MAX)
+    return MLA_ERR_INVALID_ARG;
+  if (batch == 0 || n_new == 0) return MLA_OK;
+  const int r = dims->kv_lora_rank, R = dims->num_kv_groups * dims->rope_dim;
+  if (!hidden || !w_dkv || !block_table || !start_pos || !cache) return MLA_ERR_INVALID_ARG;
+  if (R > 0 && (!rope_cos || !rope_sin)) return MLA_ERR_INVALID_ARG;
+  if (!aligned(hidden, 16) || !aligned(w_dkv, 16) || !aligned(cache, 16) ||
+      (kv_out && !aligned(kv_out, 16)))
+    return MLA_ERR_INVALID_ARG;
+  if (R > 128) return MLA_ERR_UNSUPPORTED;        // the rotary features share one tile
+  const int64_t rows = int64_t(batch) * n_new;
+  if (rows > int64_t(65535) * 128) return MLA_ERR_UNSUPPORTED;
+  const int D = row_width(dims);
+  WGemmParams p{};
+  {
+    const uint64_t dims3[3] = {uint64_t(hidden_dim), uint64_t(D), 1};
+    const uint64_t str[2] = {uint64_t(hidden_dim) * 2, uint64_t(D) * hidden_dim * 2};
+    const uint32_t box[3] = {64, 128, 1};
+    if (!encode_bf16_map(&p.tm_w, w_dkv, 3, dims3, str, box, CU_TENSOR_MAP_SWIZZLE_128B))
+      return MLA_ERR_CUDA;
+  }
+  const int nr = pick_nr(rows);
+  {
+    const uint64_t dims3[3] = {uint64_t(hidden_dim), 1, uint64_t(rows)};
+    const uint64_t str[2] = {uint64_t(hidden_dim) * 2, uint64_t(hidden_dim) * 2};
+    const uint32_t box[3] = {64, 1, uint32_t(nr)};
+    if (!encode_bf16_map(&p.tm_x, hidden, 3, dims3, str, box, CU_TENSOR_MAP_SWIZZLE_128B))
+      return MLA_ERR_CUDA;
+  }
+  p.out = nullptr;
+  p.bias = nullptr;
+  p.dev_error = dev_error;
+  p.M = D;
+  p.K = hidden_dim;
+  p.rows = int32_t(rows);
+  p.heads = 1;
+  p.a_mn = 0;
+  p.q_pe = nullptr;
+  p.rope_cos = rope_cos;
+  p.rope_sin = rope_sin;
+  p.groups = dims->num_kv_groups;
+  p.rope_dim = dims->rope_dim;
+  p.cache = static_cast<uint16_t*>(cache);
+  p.block_table = block_table;
+  p.start_pos = start_pos;
+  p.kv_out = static_cast<uint16_t*>(kv_out);
+  p.num_pages = num_pages;
+  p.max_pages = max_pages_per_seq;
+  p.n_new = n_new;
+  p.page_size = dims->page_size;
+  p.lat_r = r;
+  p.lat_tiles = (r + 127) / 128;
+  return launch_wgemm(p, nr, num_sms(), as_stream(stream)) == cudaSuccess ? MLA_OK : MLA_ERR_CUDA;
+}
+
 size_t mla_decode_workspace_size(const mla_dims* dims, int32_t batch, int32_t q_len,
                                  int32_t max_seq_len, int32_t num_splits) {
   DecodePlan P;
@@ -429,6 +492,74 @@ mla_status mla_decode_attn(const mla_dims* dims, const void* q_ext, const void* 
     if (launch_combine(c, s) != cudaSuccess) return MLA_ERR_CUDA;
   }
   return MLA_OK;
+}
+
+}  // extern "C"
+
+namespace {
+
+// The K = V form takes one key group, a query whose nope part is already in the latent
+// space (d_n = r) and an output as wide as the cache row (d_v = r + d_r).
+mla_status check_kv_shared(const mla_dims* d) {
+  mla_status st = check_dims(d);
+  if (st != MLA_OK) return st;
+  if (d->num_kv_groups != 1 || d->rope_dim <= 0 || d->qk_nope_dim != d->kv_lora_rank ||
+      d->v_head_dim != row_width(d))
+    return MLA_ERR_INVALID_ARG;
+  return MLA_OK;
+}
+
+mla_status kv_shared_rotate(const mla_dims* dims, const void* in, const float* rope_cos,
+                            const float* rope_sin, int32_t batch, int32_t q_len, void* out,
+                            int inverse, void* stream) {
+  mla_status st = check_kv_shared(dims);
+  if (st != MLA_OK) return st;
+  if (batch < 0 || q_len <= 0) return MLA_ERR_INVALID_ARG;
+  if (batch == 0) return MLA_OK;
+  if (!in || !out || !rope_cos || !rope_sin) return MLA_ERR_INVALID_ARG;
+  if (!aligned(in, 16) || !aligned(out, 16) || !aligned(rope_cos, 4) || !aligned(rope_sin, 4))
+    return MLA_ERR_INVALID_ARG;
+  KvSharedParams p{};
+  p.in = static_cast<const uint16_t*>(in);
+  p.out = static_cast<uint16_t*>(out);
+  p.rope_cos = rope_cos;
+  p.rope_sin = rope_sin;
+  p.rows = int64_t(batch) * q_len * dims->num_heads;
+  p.heads = dims->num_heads;
+  p.r = dims->kv_lora_rank;
+  p.rope_dim = dims->rope_dim;
+  p.inverse = inverse;
+  if (p.rows > (int64_t(1) << 36)) return MLA_ERR_UNSUPPORTED;
+  return launch_kv_shared_rotate(p, as_stream(stream)) == cudaSuccess ? MLA_OK : MLA_ERR_CUDA;
+}
+
+}  // namespace
+
+extern "C" {
+
+mla_status mla_kv_shared_decode_dims(const mla_dims* dims, mla_dims* decode_dims) {
+  mla_status st = check_kv_shared(dims);
+  if (st != MLA_OK) return st;
+  if (!decode_dims) return MLA_ERR_INVALID_ARG;
+  const int32_t D = row_width(dims);
+  *decode_dims = *dims;
+  decode_dims->kv_lora_rank = D;
+  decode_dims->qk_nope_dim = D;
+  decode_dims->rope_dim = 0;
+  decode_dims->v_head_dim = D;
+  return MLA_OK;
+}
+
+mla_status mla_kv_shared_query(const mla_dims* dims, const void* q, const float* rope_cos,
+                               const float* rope_sin, int32_t batch, int32_t q_len, void* q_ext,
+                               void* stream) {
+  return kv_shared_rotate(dims, q, rope_cos, rope_sin, batch, q_len, q_ext, 0, stream);
+}
+
+mla_status mla_kv_shared_output(const mla_dims* dims, const void* o_latent, const float* rope_cos,
+                                const float* rope_sin, int32_t batch, int32_t q_len, void* o,
+                                void* stream) {
+  return kv_shared_rotate(dims, o_latent, rope_cos, rope_sin, batch, q_len, o, 1, stream);
 }
 
 mla_status mla_selftest_wait_timeout(int32_t* dev_error, void* stream) {

@@ -22,6 +22,18 @@ struct AppendParams {
 };
 cudaError_t launch_cache_append(const AppendParams& p, cudaStream_t stream);
 
+// ---- the single-latent K = V form: rotary slice of the query / inverse rotation of o ---
+struct KvSharedParams {
+  const uint16_t* in;        // [rows, r + d_r] bf16
+  uint16_t* out;             // [rows, r + d_r] bf16 (may equal `in`)
+  const float* rope_cos;     // [rows / heads, d_r / 2]
+  const float* rope_sin;
+  int64_t rows;              // B * q * H
+  int32_t heads, r, rope_dim;
+  int32_t inverse;           // 0: rotate by +pos (query), 1: by -pos (output)
+};
+cudaError_t launch_kv_shared_rotate(const KvSharedParams& p, cudaStream_t stream);
+
 // ---- per-head weight GEMM (mla_absorb_q, mla_out_up) --------------------------------------
 // For every head h and activation row n: out[n, h, m] = sum_k W_h[m, k] * x[n, h, k] (+ bias).
 // The weight tile is the UMMA A operand (M = output features), the activation rows are B.
@@ -40,8 +52,18 @@ struct WGemmParams {
   const float* rope_sin;
   int32_t groups, rope_dim;
   int32_t rope_vec;          // 1: q_pe 8-byte, cos/sin 16-byte aligned and d_r/2 % 4 == 0
+  // fused cache append (mla_down_kv_append; cache == nullptr otherwise): the outputs are the
+  // D = r + G*d_r features of each token's [c_kv ; k_r], written as cache rows. Features
+  // come in ceil(r/128) latent tiles [128 t, 128 t + 128) and one rotary tile [r, D).
+  uint16_t* cache;           // [num_pages, page_size, D]
+  const int32_t* block_table;   // [B, max_pages]
+  const int32_t* start_pos;     // [B]
+  uint16_t* kv_out;          // [rows, D] bf16 GEMM output before the rotation, or null
+  int64_t num_pages;
+  int32_t max_pages, n_new, page_size, lat_r, lat_tiles;
 };
-// max_ctas: the persistent grid's size limit (one CTA per SM)
+// max_ctas: the persistent grid's size limit (one CTA per SM). With p.cache set the
+// output goes into the paged cache (see WGemmParams) instead of p.out.
 cudaError_t launch_wgemm(const WGemmParams& p, int nr, int max_ctas, cudaStream_t stream);
 
 // ---- mla_decode_attn -----------------------------------------------------------------------
@@ -76,8 +98,9 @@ cudaError_t launch_decode(const DecodeParams& p, int ncol, dim3 grid, size_t sme
 
 // Blocks of up to 128 query rows: a cluster of two CTAs splits the latent (decode_pair.cu).
 constexpr int kPairRows = 128;
-// Cache slots per CTA of the pair kernel. More TMA tiles in flight per SM lengthened each
-// tile's load latency by more than they added bandwidth (measured on B200: 4 slots beat 5).
+// Cache slots per CTA of the pair kernel. A fifth slot (room made by holding all of Q in
+// TMEM and single-buffering S) measured no faster than four on B200: the kernel is bound by
+// its per-tile hand-offs, not by the bytes in flight.
 constexpr int kPairMaxSlots = 4;
 size_t decode_pair_smem_bytes(int r, int rope_half, int nslot);
 // Clusters of two that can be resident at once with `smem` bytes each (0 if unknown).

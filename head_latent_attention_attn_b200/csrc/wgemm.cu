@@ -1,8 +1,11 @@
-// wgemm.cu - per-head weight GEMM on tcgen05 for mla_absorb_q and mla_out_up.
+// wgemm.cu - per-head weight GEMM on tcgen05 for mla_absorb_q, mla_out_up and
+// mla_down_kv_append.
 //
-// Both steps are "one small weight matrix per head times a few activation rows":
+// All three steps are "one small weight matrix per head times a few activation rows":
 //   absorb:  q_c[n, h, :]  = W_UK[h]^T q_nope[n, h, :]   (W_UK[h] stored [d_n][r])
 //   out_up:  o[n, h, :]    = W_UV[h]   o_latent[n, h, :] (W_UV[h] stored [d_v][r])
+//   down_kv: [c_kv ; k_r][n, :] = W_DKV x[n, :]          (one "head", W_DKV stored [D][hidden])
+// and the last one writes its output straight into the paged cache (mla_down_kv_append).
 // The weights dominate the bytes, so the output features are the UMMA M dimension
 // (128 per work item) and the activation rows the N dimension; D[m, n] lives in TMEM with
 // one output feature per lane, so the epilogue writes consecutive features per warp.
@@ -40,17 +43,33 @@ MLA_DEVICE uint8_t* align1024(uint8_t* p) {
   return reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(p) + 1023) & ~uintptr_t(1023));
 }
 
-// Work item `it` -> (head, first output feature, first activation row).
+// Work item `it` -> (head, first output feature, first activation row). For the fused
+// append the last feature tile is the rotary one and starts at feature r (all of a
+// group's rotation pairs then sit in one tile); the others are 128-aligned latent tiles.
 struct WgItem {
-  int h, m0, n0;
-  MLA_DEVICE WgItem(int it, int n_mt, int n_nt, int nr) {
+  int h, m0, n0, mt;
+  MLA_DEVICE WgItem(int it, int n_mt, int n_nt, int nr, int rope_tile_m0) {
     const int nt = it % n_nt;
     const int hm = it / n_nt;
     h = hm / n_mt;
-    m0 = (hm % n_mt) * 128;
+    mt = hm % n_mt;
+    m0 = (rope_tile_m0 >= 0 && mt == n_mt - 1) ? rope_tile_m0 : mt * 128;
     n0 = nt * nr;
   }
 };
+
+// Physical cache row of activation row `row` (token t of sequence b) for the fused append,
+// or -1 when its position or page is out of range (the caller sets the error word).
+MLA_DEVICE int64_t append_slot(const WGemmParams& p, int row) {
+  const int b = row / p.n_new;
+  const int t = row - b * p.n_new;
+  const int64_t pos = int64_t(p.start_pos[b]) + t;
+  const int64_t lp = pos >= 0 ? pos / p.page_size : -1;
+  if (pos < 0 || lp >= p.max_pages) return -1;
+  const int32_t page = p.block_table[int64_t(b) * p.max_pages + lp];
+  if (page < 0 || page >= p.num_pages) return -1;
+  return int64_t(page) * p.page_size + pos % p.page_size;
+}
 
 // One rotary chunk: outputs j..j+3 and j+half..j+half+3 of the (n, h, group) slice `seg`
 // (c = j / 4). Split into an address/load step and a compute/store step so that a thread
@@ -163,6 +182,85 @@ MLA_DEVICE void write_rope_slots(const WGemmParams& p, int tid, int nthreads) {
 }
 }  // namespace
 
+// Epilogue of the fused down-projection + cache append, run by the four epilogue warps for
+// one item: the accumulator (feature m0 + lane of each TMEM lane, one column per token) is
+// rounded to bf16 into a [NR tokens][128 features] staging tile, the accumulator is handed
+// back, and the tile is written as cache rows: latent features as 16-byte copies, rotary
+// features rotated in fp32 (separately rounded products and sums, from the rounded bf16
+// values, exactly as mla_cache_append) and rounded to bf16 with ties to even.
+// All four warps pass both named barriers whatever their accumulator wait returned (`ok`);
+// a failed wait leaves the CTA's abort flag set, and then no warp writes the tile.
+template <int NR>
+MLA_DEVICE void append_epilogue(const WGemmParams& p, const WgItem& w, int buf, uint32_t tmem,
+                                int sp, int lane, uint16_t* stage, uint64_t* acc_empty, bool ok,
+                                volatile int* abort_flag) {
+  const int m_loc = sp * 32 + lane;
+  const int nrows = min(NR, p.rows - w.n0);
+  if (ok) {
+#pragma unroll 1
+    for (int c0 = 0; c0 < NR; c0 += 16) {
+      float v[16];
+      tmem_ld16(tmem + (uint32_t(sp * 32) << 16) + uint32_t(buf * NR + c0), v);
+      tmem_wait_ld();
+#pragma unroll
+      for (int j = 0; j < 16; ++j) stage[(c0 + j) * 128 + m_loc] = f32_to_bf16_rne(v[j]);
+    }
+  }
+  tc_fence_before();
+  __syncwarp();
+  if (lane == 0) mbar_arrive(acc_empty);
+  named_bar_sync(1, kWgEpiThreads);               // the staging tile is complete
+  if (*abort_flag != 0) {
+    named_bar_sync(1, kWgEpiThreads);
+    return;
+  }
+  const int tid = m_loc;                          // 0..127
+  const int D = p.lat_r + p.groups * p.rope_dim;
+  if (w.m0 < p.lat_r) {
+    // latent tile: features [m0, min(m0 + 128, r)) of every token, 8 per 16-byte chunk
+    const int chunks = (min(128, p.lat_r - w.m0)) / 8;
+    for (int idx = tid; idx < nrows * chunks; idx += kWgEpiThreads) {
+      const int n = idx / chunks, c = idx - (idx / chunks) * chunks;
+      const int row = w.n0 + n;
+      const uint4 v = *reinterpret_cast<const uint4*>(stage + n * 128 + c * 8);
+      if (p.kv_out) *reinterpret_cast<uint4*>(p.kv_out + int64_t(row) * D + w.m0 + c * 8) = v;
+      const int64_t slot = append_slot(p, row);
+      if (slot < 0) {
+        if (c == 0 && p.dev_error) atomicOr(p.dev_error, MLA_DEVERR_BOUNDS);
+        continue;
+      }
+      *reinterpret_cast<uint4*>(p.cache + slot * D + w.m0 + c * 8) = v;
+    }
+  } else {
+    // rotary tile: features [r, D), pair j of group g = (x_j, x_{j + d_r/2})
+    const int half = p.rope_dim / 2;
+    const int pairs = p.groups * half;
+    for (int idx = tid; idx < nrows * pairs; idx += kWgEpiThreads) {
+      const int n = idx / pairs, pi = idx - (idx / pairs) * pairs;
+      const int g = pi / half, j = pi - (pi / half) * half;
+      const int row = w.n0 + n;
+      const int f = g * p.rope_dim + j;           // feature within the rotary tile
+      const uint16_t b0 = stage[n * 128 + f], b1 = stage[n * 128 + f + half];
+      if (p.kv_out) {
+        p.kv_out[int64_t(row) * D + p.lat_r + f] = b0;
+        p.kv_out[int64_t(row) * D + p.lat_r + f + half] = b1;
+      }
+      const int64_t slot = append_slot(p, row);
+      if (slot < 0) {
+        if (pi == 0 && p.dev_error) atomicOr(p.dev_error, MLA_DEVERR_BOUNDS);
+        continue;
+      }
+      const float x0 = bf16_bits_to_f32(b0), x1 = bf16_bits_to_f32(b1);
+      const int64_t ci = (int64_t(row) * p.groups + g) * half + j;
+      const float cj = p.rope_cos[ci], sj = p.rope_sin[ci];
+      uint16_t* dst = p.cache + slot * D + p.lat_r + f;
+      dst[0] = f32_to_bf16_rne(__fsub_rn(__fmul_rn(x0, cj), __fmul_rn(x1, sj)));
+      dst[half] = f32_to_bf16_rne(__fadd_rn(__fmul_rn(x1, cj), __fmul_rn(x0, sj)));
+    }
+  }
+  named_bar_sync(1, kWgEpiThreads);               // the staging tile may be reused
+}
+
 template <int NR>
 __global__ void __launch_bounds__(kWgThreads, 1) wgemm_kernel(const __grid_constant__ WGemmParams p) {
   using Lay = WgLayout<NR>;
@@ -178,7 +276,9 @@ __global__ void __launch_bounds__(kWgThreads, 1) wgemm_kernel(const __grid_const
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-  const int n_mt = (p.M + 127) / 128;
+  const bool append = p.cache != nullptr;
+  const int rope_m0 = (append && p.groups * p.rope_dim > 0) ? p.lat_r : -1;
+  const int n_mt = append ? p.lat_tiles + (rope_m0 >= 0 ? 1 : 0) : (p.M + 127) / 128;
   const int n_nt = (p.rows + NR - 1) / NR;
   const int items = n_mt * p.heads * n_nt;
   const int nk = (p.K + 63) / 64;
@@ -215,7 +315,7 @@ __global__ void __launch_bounds__(kWgThreads, 1) wgemm_kernel(const __grid_const
       int g = 0;   // stages issued
       bool ok = true;
       for (int it = blockIdx.x; ok && it < items; it += gridDim.x) {
-        const WgItem w(it, n_mt, n_nt, NR);
+        const WgItem w(it, n_mt, n_nt, NR, rope_m0);
         for (int kb = 0; kb < nk; ++kb, ++g, ring.next()) {
           if (g >= S && !mbar_wait(&empty[ring.slot], (ring.round - 1) & 1, wc)) {
             ok = false;
@@ -281,10 +381,16 @@ __global__ void __launch_bounds__(kWgThreads, 1) wgemm_kernel(const __grid_const
                        int(gridDim.x) * kWgEpiThreads);
     int li = 0;
     for (int it = blockIdx.x; it < items; it += gridDim.x, ++li) {
-      const WgItem w(it, n_mt, n_nt, NR);
+      const WgItem w(it, n_mt, n_nt, NR, rope_m0);
       const int buf = li & 1;
       const bool ok = __all_sync(0xffffffffu, mbar_wait(&acc_full[buf], (li >> 1) & 1, wc));
       tc_fence_after();
+      if (append) {
+        append_epilogue<NR>(p, w, buf, tmem, sp, lane,
+                            reinterpret_cast<uint16_t*>(base + Lay::kBars + 256), &acc_empty[buf],
+                            ok, abort_flag);
+        continue;
+      }
       if (ok) {
         const int m = w.m0 + sp * 32 + lane;   // output feature of this thread's TMEM lane
         const float bias = (p.bias != nullptr && m < p.M)
@@ -321,11 +427,15 @@ __global__ void __launch_bounds__(kWgThreads, 1) wgemm_kernel(const __grid_const
 
 template <int NR>
 static cudaError_t launch_wgemm_nr(const WGemmParams& p, int max_ctas, cudaStream_t stream) {
-  const int smem = WgLayout<NR>::kTotal;
+  const bool append = p.cache != nullptr;
+  // the fused append stages one [NR][128] bf16 tile after the barriers
+  const int smem = WgLayout<NR>::kTotal + (append ? NR * 128 * 2 : 0);
   cudaError_t e = cudaFuncSetAttribute(wgemm_kernel<NR>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
-  const int64_t items = int64_t((p.M + 127) / 128) * p.heads * ((p.rows + NR - 1) / NR);
+  const int64_t n_mt = append ? p.lat_tiles + (p.groups * p.rope_dim > 0 ? 1 : 0)
+                              : (p.M + 127) / 128;
+  const int64_t items = n_mt * p.heads * ((p.rows + NR - 1) / NR);
   const int grid = int(items < max_ctas ? items : max_ctas);
   wgemm_kernel<NR><<<grid, kWgThreads, smem, stream>>>(p);
   return cudaGetLastError();

@@ -103,6 +103,33 @@ mla_status mla_cache_append(const mla_dims* dims, const void* c_kv, const void* 
                             void* stream);
 
 /*
+ * mla_down_kv_append - the KV down-projection of new tokens, written straight into the
+ * paged cache: one tcgen05 GEMM whose epilogue is mla_cache_append.
+ *
+ * The MLAfication page (wzjinhao.cn) sends the hidden state X through down_kv to the
+ * latent c_kv (all the cache keeps of K/V) and through k_r_proj to the rotary key; the
+ * DeepSeek-V2 page does both with kv_a_proj_with_mqa, eq. (41), split into
+ * [kv_lora_rank, qk_rope_head_dim].
+ *
+ *   hidden      bf16 [B, n_new, hidden_dim]   hidden_dim a multiple of 8
+ *   w_dkv       bf16 [D, hidden_dim]          rows 0..r-1: down_kv; rows r + g*d_r + j:
+ *                                             group g's k_r_proj (no bias)
+ *   rope_cos/sin, block_table, start_pos, cache, num_pages, dev_error: as mla_cache_append
+ *   kv_out      bf16 [B, n_new, D] or NULL    if given, also receives the GEMM's bf16
+ *                                             output [c_kv ; k_r] before the rotation
+ *
+ * For each token: [c_kv ; k_r] = bf16_rne(fp32 sum over hidden of w_dkv * x), then exactly
+ * what mla_cache_append writes for that c_kv and k_r (the same cache bytes). Requires
+ * G*d_r <= 128 (MLA_ERR_UNSUPPORTED otherwise). Bounds faults as mla_cache_append.
+ */
+mla_status mla_down_kv_append(const mla_dims* dims, const void* hidden, int32_t hidden_dim,
+                              const void* w_dkv, const float* rope_cos, const float* rope_sin,
+                              const int32_t* block_table, int32_t max_pages_per_seq,
+                              const int32_t* start_pos, int32_t batch, int32_t n_new,
+                              void* cache, int64_t num_pages, int32_t* dev_error, void* kv_out,
+                              void* stream);
+
+/*
  * mla_absorb_q - fold W_UK into the query and rotate its RoPE part.
  *
  * The "W^{UK} is absorbed by q_nope" step of the DeepSeek-V2 page:
@@ -180,6 +207,43 @@ mla_status mla_decode_attn(const mla_dims* dims, const void* q_ext, const void* 
 mla_status mla_out_up(const mla_dims* dims, const void* o_latent, const void* w_uv,
                       int64_t w_uv_head_stride, const void* bias, int32_t rows, void* o,
                       void* stream);
+
+/*
+ * The single-latent K = V form (nanowhale-100m page, cnnetsun.cn: "single KV head, many
+ * query heads", "applying RoPE" and "efficient attention", where
+ * scaled_dot_product_attention(q, kv_expanded, kv_expanded) uses one head_dim vector per
+ * token as both key and value, RoPE on its last d_r dims, and the output's rotary dims are
+ * rotated back afterwards).
+ *
+ * dims describe that form: num_kv_groups = 1, kv_lora_rank = r = the unrotated width,
+ * qk_nope_dim = r, rope_dim = d_r > 0, v_head_dim = r + d_r = D (the head_dim). The cache is
+ * the ordinary latent cache written by mla_cache_append with these dims (row = [kv_nope |
+ * RoPE(kv_pe)]). One decode step is then:
+ *   mla_kv_shared_query   q_ext = [q[:r] ; R(pos) q[r:]]                (bf16 [B, q, H, D])
+ *   mla_decode_attn       with the dims from mla_kv_shared_decode_dims (the whole row is
+ *                         the "latent": rank D, no separate rotary slot), giving
+ *                         o_latent = sum_l p_l row_l  [B, q, H, D] and lse
+ *   mla_kv_shared_output  o = [o_latent[:r] ; R(-pos) o_latent[r:]]    (bf16 [B, q, H, D])
+ * R(pos) rotates the pairs (x_j, x_{j+d_r/2}) by the caller's angles: rope_cos/sin fp32
+ * [B, q, 1, d_r/2] at each query row's position (the same tables for both calls). The
+ * rotation is fp32 with separately rounded products and sums, then bf16 round to nearest
+ * even. A model whose rotary embedding pairs adjacent dims (complex form) permutes its
+ * rotary dims once to this half-split layout; attention and the inverse rotation commute
+ * with that permutation.
+ *
+ * mla_kv_shared_decode_dims: writes the decode view of `dims` ({H, 1, D, D, 0, D, ps,
+ * scale}) to `decode_dims`; MLA_ERR_INVALID_ARG if `dims` is not a K = V layout.
+ * mla_kv_shared_query / _output: q / o_latent and q_ext / o are [B, q, H, D] bf16, 16-byte
+ * aligned; in place allowed (in == out). MLA_ERR_INVALID_ARG on a non-K = V layout, a null
+ * or misaligned pointer, batch < 0 or q_len <= 0; batch == 0 launches nothing.
+ */
+mla_status mla_kv_shared_decode_dims(const mla_dims* dims, mla_dims* decode_dims);
+mla_status mla_kv_shared_query(const mla_dims* dims, const void* q, const float* rope_cos,
+                               const float* rope_sin, int32_t batch, int32_t q_len, void* q_ext,
+                               void* stream);
+mla_status mla_kv_shared_output(const mla_dims* dims, const void* o_latent,
+                                const float* rope_cos, const float* rope_sin, int32_t batch,
+                                int32_t q_len, void* o, void* stream);
 
 /*
  * mla_decode_attn_noalloc - mla_decode_attn for callers that cannot allocate device memory.

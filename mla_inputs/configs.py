@@ -15,6 +15,13 @@ Shapes come from the pages' models:
   KV groups, rank 512, 8 RoPE dims per KV group, ragged context lengths.
 * hybrid_*: the MLA layers of the zebra hybrid model (trdm.cn page):
   16 heads, kv_lora_rank 256, context extended to 1,048,576 tokens.
+* nanowhale_kv_shared: the single-latent K = V layer of nanowhale-100m (cnnetsun.cn
+  page): 8 heads, one 512-d key/value vector per token with RoPE on its last 64 dims.
+
+Model widths (``hidden_size``, the input of the KV down-projection): DeepSeek-V2 5120
+(the dtcms.com page's o_proj is [128*128, 5120]), Qwen3-1.7B 2048 (trdm.cn page's
+config table), nanowhale-100m 320 (cnnetsun.cn page). The pages print none for
+Qwen2.5-7B or Qwen3-30B-A3B; reading: those models' published widths, 3584 and 2048.
 
 This module holds shapes and seeds only; it does none of the method's
 arithmetic.
@@ -49,6 +56,7 @@ class MLAConfig:
     rope_index_pool: int = 0   # > 0: per-group frequency indices drawn from range(pool)
     with_bias: bool = False    # W_UV bias (the up_v.bias of the MLAfied checkpoints)
     identity_weights: bool = False   # W_UK = W_UV = I (needs d_n = d_v = r): plain MQA on c_kv
+    hidden_size: int = 256     # model width feeding the KV down-projection (mla_down_kv_append)
 
     @property
     def row_width(self) -> int:
@@ -82,26 +90,37 @@ TINY = _cfg(name="tiny", index=0, batch=1, q_len=1, num_heads=4, num_kv_groups=1
 
 QWEN25_7B = _cfg(name="qwen25_7b", index=1, batch=32, q_len=1, num_heads=28,
                  num_kv_groups=4, kv_lora_rank=128, qk_nope_dim=128, rope_dim=8,
-                 v_head_dim=128, context=4096, rope_ref_dim=128, rope_index_pool=64)
+                 v_head_dim=128, context=4096, rope_ref_dim=128, rope_index_pool=64,
+                 hidden_size=3584)
 
 DEEPSEEK_V2 = _cfg(name="deepseek_v2", index=2, batch=64, q_len=1, num_heads=128,
                    num_kv_groups=1, kv_lora_rank=512, qk_nope_dim=128, rope_dim=64,
-                   v_head_dim=128, context=8192, softmax_scale=1.0 / math.sqrt(192.0))
+                   v_head_dim=128, context=8192, softmax_scale=1.0 / math.sqrt(192.0),
+                   hidden_size=5120)
 
 QWEN3_30B_A3B = _cfg(name="qwen3_30b_a3b", index=3, batch=128, q_len=1, num_heads=32,
                      num_kv_groups=4, kv_lora_rank=512, qk_nope_dim=128, rope_dim=8,
                      v_head_dim=128, lens_range=(1024, 32768), rope_ref_dim=128,
-                     rope_index_pool=64)
+                     rope_index_pool=64, hidden_size=2048)
 
 _HYB = dict(index=4, num_heads=16, num_kv_groups=1, kv_lora_rank=256, qk_nope_dim=128,
-            rope_dim=64, v_head_dim=128, softmax_scale=1.0 / math.sqrt(192.0))
+            rope_dim=64, v_head_dim=128, softmax_scale=1.0 / math.sqrt(192.0), hidden_size=2048)
 HYBRID_1M_Q1 = _cfg(name="hybrid_1m_q1", batch=1, q_len=1, context=1 << 20, **_HYB)
 HYBRID_1M_Q4 = _cfg(name="hybrid_1m_q4", batch=1, q_len=4, context=1 << 20, **_HYB)
 HYBRID_256K_Q1 = _cfg(name="hybrid_256k_q1", batch=4, q_len=1, context=1 << 18, **_HYB)
 HYBRID_256K_Q4 = _cfg(name="hybrid_256k_q4", batch=4, q_len=4, context=1 << 18, **_HYB)
 
+# The single-latent K = V layer of nanowhale-100m (cnnetsun.cn page): 8 query heads over one
+# KV head of head_dim 512 = 448 unrotated + 64 rotary dims, context 2,048. In the library's
+# terms r = 448 and d_r = 64 with one key group; the output is the whole 512-d row.
+NANOWHALE_KV_SHARED = _cfg(name="nanowhale_kv_shared", index=5, batch=128, q_len=1,
+                           num_heads=8, num_kv_groups=1, kv_lora_rank=448, qk_nope_dim=448,
+                           rope_dim=64, v_head_dim=512, context=2048,
+                           softmax_scale=1.0 / math.sqrt(512.0), hidden_size=320)
+
 CONFIGS = {c.name: c for c in (TINY, QWEN25_7B, DEEPSEEK_V2, QWEN3_30B_A3B, HYBRID_1M_Q1,
-                               HYBRID_1M_Q4, HYBRID_256K_Q1, HYBRID_256K_Q4)}
+                               HYBRID_1M_Q4, HYBRID_256K_Q1, HYBRID_256K_Q4,
+                               NANOWHALE_KV_SHARED)}
 
 
 def shrink(cfg: MLAConfig, batch: Optional[int] = None, context: Optional[int] = None,

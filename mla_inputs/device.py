@@ -121,3 +121,31 @@ class DeviceProblem:
         a = mla.mla_get_device_status(self.err)
         b = mla.mla_get_device_status(self.workspace.view(torch.int32)[:1])
         return max(a, b)
+
+    # ---- the single-latent K = V form ------------------------------------------------------
+    def kv_shared_step(self, stream=None, num_splits=None) -> None:
+        """One step of the K = V form on this problem's cache: append the last q tokens,
+        rotate the query's rotary slice, decode over whole rows (the decode view of the dims)
+        and rotate the output's rotary slice back. Output in ``self.o_kv`` [B, q, H, D]."""
+        cfg = self.cfg
+        B, q, H, D = cfg.batch, cfg.q_len, cfg.num_heads, cfg.row_width
+        ns = self.num_splits if num_splits is None else num_splits
+        if not hasattr(self, "o_kv"):
+            self.kv_dims = mla.mla_kv_shared_decode_dims(self.dims)
+            self.q_kv = torch.cat([self.q_nope, self.q_pe], dim=-1).contiguous()
+            self.q_ext_kv = torch.empty((B, q, H, D), dtype=torch.bfloat16, device=self.dev)
+            self.o_lat_kv = torch.empty((B, q, H, D), dtype=torch.bfloat16, device=self.dev)
+            self.lse_kv = torch.empty((B, q, H), dtype=torch.float32, device=self.dev)
+            self.o_kv = torch.empty((B, q, H, D), dtype=torch.bfloat16, device=self.dev)
+            ws = mla.mla_decode_workspace_size(self.kv_dims, B, q, self.max_seq_len, ns)
+            self.ws_kv = torch.zeros(ws, dtype=torch.uint8, device=self.dev)
+        mla.mla_cache_append(self.dims, self.c_new, self.k_new, self.cos_q, self.sin_q,
+                             self.block_table, self.start_pos, self.cache,
+                             dev_error=self.ws_kv.view(torch.int32)[:1], stream=stream)
+        mla.mla_kv_shared_query(self.dims, self.q_kv, self.cos_q, self.sin_q, self.q_ext_kv,
+                                stream=stream)
+        mla.mla_decode_attn(self.kv_dims, self.q_ext_kv, self.cache, self.block_table,
+                            self.seq_lens, self.max_seq_len, self.ws_kv, self.o_lat_kv,
+                            self.lse_kv, causal=cfg.causal, num_splits=ns, stream=stream)
+        mla.mla_kv_shared_output(self.dims, self.o_lat_kv, self.cos_q, self.sin_q, self.o_kv,
+                                 stream=stream)

@@ -146,3 +146,14 @@ def make_workload(cfg: MLAConfig, q_scale: float = 1.0, spare_pages: int = 0,
     return Workload(cfg=cfg, seq_lens=lens, rope_index=idx, theta=theta, w_uk=w_uk, w_uv=w_uv,
                     bias=bias, q_nope=q_nope, q_pe=q_pe, block_table=table,
                     num_pages=num_pages, spare_pages=spare)
+
+
+def make_down_kv_inputs(cfg: MLAConfig, n_new: int) -> Tuple[torch.Tensor, torch.Tensor]:
+    """Inputs of the KV down-projection for ``cfg``: hidden states [B, n_new, hidden] ~ N(0, 1)
+    and the stacked projection [r + G*d_r, hidden] ~ N(0, 1) / sqrt(hidden) (down_kv rows,
+    then each group's k_r_proj rows), both rounded to bf16, from their own seeded generator."""
+    gen = torch.Generator("cpu")
+    gen.manual_seed(cfg.seed * 31 + 17)
+    hidden = torch.randn(cfg.batch, n_new, cfg.hidden_size, generator=gen).to(torch.bfloat16)
+    w_dkv = _randn(gen, (cfg.row_width, cfg.hidden_size), cfg.hidden_size)
+    return hidden, w_dkv

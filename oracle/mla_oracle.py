@@ -16,6 +16,14 @@ What it computes, and where the pages define it
   It also returns o_latent = sum_l p_l c_kv[l], the intermediate of einsum (4).
 * ``absorb_reference`` / ``out_up_reference``: the absorb einsum and einsum (5) on their
   own, for checking the two projection steps separately.
+* ``mla_decode_absorbed``: the same attention in the absorbed order (a second CPU
+  baseline; equal to the unabsorbed definition by associativity).
+* ``down_kv_reference``: the hidden -> [c_kv ; k_r] projection whose output the cache
+  stores (down_kv / k_r_proj of the MLAfication page, kv_a_proj_with_mqa of the
+  DeepSeek-V2 page).
+* ``kv_shared_reference``: the single-latent K = V form of the nanowhale-100m page
+  (cnnetsun.cn): one rotated head_dim vector per token serves as key and value, and the
+  output's rotary dims are rotated back by the query position.
 * ``rope_rotate``: RoPE on a rotary slice, pairs (x_j, x_{j+d/2}) rotated by theta_j * pos
   (the rotate-half convention of ``apply_rotary_pos_emb`` used on that page), angles in fp64.
 * ``cache_append_emulate``: the byte-exact result of writing new tokens into the paged
@@ -219,3 +227,101 @@ def cache_append_emulate(cache_bits: np.ndarray, c_kv_bits: np.ndarray, k_r_bits
             y = rotate_fp32(x, cos32[b], sin32[b])                         # [n, G, d_r]
             out[pages, rows, r:] = f32_to_bf16_bits(y).reshape(n, G * dr)
     return out
+
+
+# ----------------------------------------------------------------------------------------
+# The single-latent K = V form (nanowhale-100m page, cnnetsun.cn)
+# ----------------------------------------------------------------------------------------
+
+def kv_shared_reference(q_nope, q_pe, kv_nope, kv_pe, theta, q_pos, softmax_scale,
+                        causal: bool = True) -> Dict[str, np.ndarray]:
+    """Attention in which one cached vector per token is both key and value, in fp64.
+
+    The nanowhale-100m page ("single KV head, many query heads"; "applying RoPE"; "efficient
+    attention": scaled_dot_product_attention(q, kv_expanded, kv_expanded)): every head's
+    query attends over one shared head_dim vector per token, kv = [kv_nope ; kv_pe], whose
+    last d_r dims are rotated at the token's position, as are the query's last d_r dims at
+    the query position; the values are the same rotated vectors, so the output's last d_r
+    dims are a mix of vectors rotated to different positions. The page's "output inverse
+    rotation" then rotates those dims back by the query's own position (reading: the
+    position of the output row).
+
+    q_nope [q, H, d_n], q_pe [q, H, d_r] (unrotated), kv_nope [L, d_n], kv_pe [L, d_r]
+    (unrotated; token l at position l), theta [d_r/2], q_pos [q].
+    Returns o [q, H, d_n + d_r] (after the inverse rotation) and lse [q, H].
+    """
+    q_nope, q_pe = as_f64(q_nope), as_f64(q_pe)
+    kv_nope, kv_pe = as_f64(kv_nope), as_f64(kv_pe)
+    theta = np.asarray(theta, dtype=np.float64)
+    q_pos = np.asarray(q_pos, dtype=np.int64)
+    nq, H, _ = q_nope.shape
+    L = kv_nope.shape[0]
+    tok_pos = np.arange(L, dtype=np.int64)
+    kv = np.concatenate([kv_nope, rope_rotate(kv_pe, theta, tok_pos)], axis=-1)       # [L, Dh]
+    q_rot = rope_rotate(q_pe, theta, q_pos[:, None])                                   # [q, H, d_r]
+    Q = np.concatenate([q_nope, q_rot], axis=-1)                                       # [q, H, Dh]
+    s = softmax_scale * np.einsum("ihd,ld->ihl", Q, kv)
+    if causal:
+        s = np.where((tok_pos[None, :] <= q_pos[:, None])[:, None, :], s, -np.inf)
+    m = s.max(axis=-1, keepdims=True)
+    lse = m[..., 0] + np.log(np.exp(s - m).sum(axis=-1))
+    p = np.exp(s - lse[..., None])
+    o = np.einsum("ihl,ld->ihd", p, kv)                                                # V = K
+    dn = kv_nope.shape[1]
+    o[..., dn:] = rope_rotate(o[..., dn:], theta, -q_pos[:, None])                     # inverse
+    return {"o": o, "lse": lse}
+
+
+def mla_decode_absorbed(q_nope, q_pe, c_kv, k_r, w_uk, w_uv, bias, theta, q_pos,
+                        softmax_scale: float, causal: bool = True) -> Dict[str, np.ndarray]:
+    """The same attention in the absorbed order, in fp64, for ONE sequence: q_c =
+    einsum('hdc,bhqd->bhqc', W_UK, q_nope), scores q_c . c_kv + rotated q_pe . rotated k_r,
+    o_ = p c_kv (einsum 4), o = o_ W_UV (einsum 5) (DeepSeek-V2 page, "Matrix absorption").
+    Arguments and results as mla_decode_reference. Used as a second CPU baseline; it equals
+    the unabsorbed definition by associativity."""
+    q_nope, q_pe, c_kv, k_r = as_f64(q_nope), as_f64(q_pe), as_f64(c_kv), as_f64(k_r)
+    w_uk, w_uv = as_f64(w_uk), as_f64(w_uv)
+    theta = np.asarray(theta, dtype=np.float64)
+    q_pos = np.asarray(q_pos, dtype=np.int64)
+    nq, H, _ = q_nope.shape
+    L = c_kv.shape[0]
+    G = k_r.shape[1]
+    g_of = group_of_head(H, G)
+    tok_pos = np.arange(L, dtype=np.int64)
+    q_c, q_rot = absorb_reference(q_nope, q_pe, w_uk, theta, q_pos, G)
+    o_lat = np.zeros((nq, H, c_kv.shape[1]))
+    lse = np.zeros((nq, H))
+    for g in range(G):
+        k_rot = rope_rotate(k_r[:, g, :], theta[g], tok_pos)                           # [L, d_r]
+        hs = np.nonzero(g_of == g)[0]
+        s = softmax_scale * (np.einsum("ihc,lc->ihl", q_c[:, hs], c_kv) +
+                             np.einsum("ihe,le->ihl", q_rot[:, hs], k_rot))
+        if causal:
+            s = np.where((tok_pos[None, :] <= q_pos[:, None])[:, None, :], s, -np.inf)
+        m = s.max(axis=-1, keepdims=True)
+        lse_g = m[..., 0] + np.log(np.exp(s - m).sum(axis=-1))
+        o_lat[:, hs] = np.einsum("ihl,lc->ihc", np.exp(s - lse_g[..., None]), c_kv)    # (4)
+        lse[:, hs] = lse_g
+    o = out_up_reference(o_lat, w_uv, None if bias is None else as_f64(bias))          # (5)
+    return {"o": o, "o_latent": o_lat, "lse": lse}
+
+
+# ----------------------------------------------------------------------------------------
+# The KV down-projection that produces the cached latent (fused with the append on the GPU)
+# ----------------------------------------------------------------------------------------
+
+def down_kv_reference(hidden, w_dkv, kv_lora_rank: int, num_groups: int, rope_dim: int):
+    """The cached token's latent and unrotated rotary key from its hidden state, in fp64.
+
+    The MLAfication page (wzjinhao.cn) sends the hidden state X through down_kv to the
+    latent c_kv (the only part of K/V the cache keeps) and through k_r_proj to the low-
+    dimensional rotary key; the DeepSeek-V2 page does both with one matrix, eq. (41)
+    kv_a_proj_with_mqa, whose output is split into [kv_lora_rank, qk_rope_head_dim]. Here
+    w_dkv [r + G*d_r, hidden] stacks the down_kv rows and each group's k_r rows, and
+    [c_kv ; k_r] = w_dkv @ x for every token x [.., hidden].
+    Returns c_kv [.., r] and k_r [.., G, d_r] (fp64, before RoPE).
+    """
+    out = np.einsum("...k,dk->...d", as_f64(hidden), as_f64(w_dkv))
+    c_kv = out[..., :kv_lora_rank]
+    k_r = out[..., kv_lora_rank:].reshape(out.shape[:-1] + (num_groups, rope_dim))
+    return c_kv, k_r

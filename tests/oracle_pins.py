@@ -375,6 +375,99 @@ def pin_out_up_associativity(O):
     _close(O.out_up_reference(got["o_latent"], P["w_uv"], P["bias"]), got["o"], 1e-12, "einsum 5")
 
 
+# ----------------------------------------------------------------------------------------
+# pins on the single-latent K = V form and on the absorbed-order baseline
+# ----------------------------------------------------------------------------------------
+
+def _complex_rotate(x, theta, pos):
+    """Rotate interleaved pairs (x_2j, x_2j+1) as complex numbers times exp(i theta_j pos)."""
+    z = x[..., 0::2] + 1j * x[..., 1::2]
+    z = z * np.exp(1j * np.asarray(pos, dtype=np.float64)[..., None] * theta)
+    out = np.empty_like(x)
+    out[..., 0::2], out[..., 1::2] = z.real, z.imag
+    return out
+
+
+def pin_kv_shared_sdpa(O):
+    """K = V attention with the page's complex (interleaved-pair) rotary embedding, torch's
+    scaled_dot_product_attention with the same tensor as key and value, and the inverse
+    rotation of the output by multiplication with exp(-i theta pos_q). The oracle uses
+    half-split pairs (x_j, x_j+d/2); the two agree once the rotary dims are permuted."""
+    rng = np.random.default_rng(41)
+    for causal, (nq, H, dn, dr, L) in [(True, (3, 4, 6, 4, 23)), (False, (2, 3, 5, 6, 17)),
+                                       (True, (1, 2, 3, 2, 9))]:
+        qn, qp = rng.standard_normal((nq, H, dn)), rng.standard_normal((nq, H, dr))
+        kn, kp = rng.standard_normal((L, dn)), rng.standard_normal((L, dr))
+        theta = rng.uniform(0.05, 1.2, size=dr // 2)
+        q_pos = np.arange(L - nq, L)
+        scale = 0.61
+        got = O.kv_shared_reference(qn, qp, kn, kp, theta, q_pos, scale, causal=causal)
+        h = dr // 2
+        perm = np.empty(dr, dtype=np.int64)              # half-split index -> interleaved slot
+        perm[0::2], perm[1::2] = np.arange(h), np.arange(h) + h
+        q = np.concatenate([qn, _complex_rotate(qp[..., perm], theta, q_pos[:, None])], -1)
+        kv = np.concatenate([kn, _complex_rotate(kp[..., perm], theta, np.arange(L))], -1)
+        qt = torch.from_numpy(q).permute(1, 0, 2)[None]                    # [1, H, q, Dh]
+        kt = torch.from_numpy(kv)[None, None].expand(1, H, L, dn + dr)
+        mask = torch.from_numpy(np.arange(L)[None, :] <= q_pos[:, None]) if causal else None
+        o = torch.nn.functional.scaled_dot_product_attention(qt, kt, kt, attn_mask=mask,
+                                                             scale=scale)[0].permute(1, 0, 2).numpy()
+        o = o.copy()
+        o[..., dn:] = _complex_rotate(o[..., dn:], theta, -q_pos[:, None])
+        inv = np.argsort(perm)
+        o[..., dn:] = o[..., dn:][..., inv]
+        _close(got["o"], o, 1e-12, "kv-shared o vs sdpa")
+        s = torch.einsum("hid,ld->ihl", qt[0], torch.from_numpy(kv)) * scale
+        if causal:
+            s = s.masked_fill(~mask[:, None, :], float("-inf"))
+        _close(got["lse"], torch.logsumexp(s, dim=-1).numpy(), 1e-12, "kv-shared lse")
+
+
+def pin_kv_shared_single_token(O):
+    """One cached token at position 0 and a query at position 0: the output is that token's
+    vector itself (the rotation at position 0 is the identity), lse its scaled score."""
+    rng = np.random.default_rng(43)
+    qn, qp = rng.standard_normal((1, 3, 5)), rng.standard_normal((1, 3, 4))
+    kn, kp = rng.standard_normal((1, 5)), rng.standard_normal((1, 4))
+    got = O.kv_shared_reference(qn, qp, kn, kp, np.array([0.3, 0.9]), np.array([0]), 0.5)
+    want = np.concatenate([kn, kp], -1)[None].repeat(3, axis=1)
+    _close(got["o"], want, 1e-14, "single token o")
+    s = 0.5 * (np.einsum("ihd,d->ih", qn, kn[0]) + np.einsum("ihd,d->ih", qp, kp[0]))
+    _close(got["lse"], s, 1e-14, "single token lse")
+
+
+def pin_absorbed_baseline(O):
+    """The absorbed-order CPU baseline equals the unabsorbed definition (associativity of
+    einsums (1)-(3) against (4)-(5)) and the scalar brute force."""
+    for seed, kw in [(51, dict(nq=2, H=6, G=3, r=5, dn=4, dr=4, dv=3, L=11)),
+                     (52, dict(nq=1, H=4, G=1, r=8, dn=3, dr=2, dv=6, L=7, bias=False))]:
+        P = _problem(seed, **kw)
+        got = O.mla_decode_absorbed(**P)
+        ref = _brute_force(**P)
+        for k in ("o", "o_latent", "lse"):
+            _close(got[k], ref[k], 1e-11, f"absorbed baseline {k}")
+
+
+def pin_down_kv_bruteforce(O):
+    """The down-projection against literal loops over tokens, outputs and the hidden dim,
+    and the split of its output into the latent and each group's rotary key."""
+    rng = np.random.default_rng(61)
+    B, n, hid, r, G, dr = 2, 3, 7, 4, 2, 2
+    x = rng.standard_normal((B, n, hid))
+    w = rng.standard_normal((r + G * dr, hid))
+    c_kv, k_r = O.down_kv_reference(x, w, r, G, dr)
+    for b in range(B):
+        for t in range(n):
+            for d in range(r + G * dr):
+                acc = 0.0
+                for k in range(hid):
+                    acc += w[d][k] * x[b][t][k]
+                got = c_kv[b, t, d] if d < r else k_r[b, t, (d - r) // dr, (d - r) % dr]
+                assert abs(got - acc) <= 1e-12 * max(1.0, abs(acc)), (b, t, d)
+
+
 ALL_PINS = [pin_absorb_single_token, pin_out_up_associativity, pin_bruteforce, pin_associativity, pin_sdpa_identity_weights, pin_zero_query_uniform,
             pin_single_token, pin_rows_sum_to_one, pin_causal_prefix, pin_rope_complex,
-            pin_rope_norm_and_relative, pin_bf16_rounding, pin_rotate_fp32, pin_append_slots]
+            pin_rope_norm_and_relative, pin_bf16_rounding, pin_rotate_fp32, pin_append_slots,
+            pin_kv_shared_sdpa, pin_kv_shared_single_token, pin_absorbed_baseline,
+            pin_down_kv_bruteforce]

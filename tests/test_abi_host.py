@@ -174,3 +174,43 @@ def test_noalloc_validation_before_launch(mla_lib):
     d = _dims()
     assert mla.mla_decode_workspace_size(d, 4_000_000, 1, 64, 0) > 32 << 20
     assert _noalloc(d, batch=4_000_000, maxlen=64, maxp=1) == mla.MLA_ERR_WORKSPACE
+
+
+def test_kv_shared_validation(mla_lib):
+    L = mla.lib()
+    kv = _dims(CONFIGS["nanowhale_kv_shared"])
+    out = mla.MlaDims()
+    assert L.mla_kv_shared_decode_dims(ctypes.byref(kv), ctypes.byref(out)) == mla.MLA_OK
+    assert (out.kv_lora_rank, out.rope_dim, out.v_head_dim, out.num_kv_groups) == (512, 0, 512, 1)
+    assert mla.mla_row_width(out) == 512
+    # not a K = V layout: two key groups, d_n != r, d_v != D, no rotary dims
+    for bad in (dict(num_kv_groups=2), dict(qk_nope_dim=128), dict(v_head_dim=448),
+                dict(rope_dim=0, v_head_dim=448)):
+        d = _dims(CONFIGS["nanowhale_kv_shared"], **bad)
+        assert L.mla_kv_shared_decode_dims(ctypes.byref(d), ctypes.byref(out)) == \
+            mla.MLA_ERR_INVALID_ARG, bad
+        assert L.mla_kv_shared_query(ctypes.byref(d), FAKE, FAKE, FAKE, 2, 1, FAKE, None) == \
+            mla.MLA_ERR_INVALID_ARG, bad
+    assert L.mla_kv_shared_query(ctypes.byref(kv), None, FAKE, FAKE, 2, 1, FAKE, None) == \
+        mla.MLA_ERR_INVALID_ARG
+    assert L.mla_kv_shared_output(ctypes.byref(kv), FAKE, FAKE, FAKE, 2, 1, P(0x10008), None) == \
+        mla.MLA_ERR_INVALID_ARG                                   # misaligned output
+    assert L.mla_kv_shared_output(ctypes.byref(kv), FAKE, FAKE, FAKE, 2, 0, FAKE, None) == \
+        mla.MLA_ERR_INVALID_ARG                                   # q_len 0
+    assert L.mla_kv_shared_query(ctypes.byref(kv), FAKE, FAKE, FAKE, 0, 1, FAKE, None) == mla.MLA_OK
+
+
+def test_down_kv_append_validation(mla_lib):
+    L = mla.lib()
+    d = _dims()
+
+    def call(dd=d, hidden=FAKE, hid=5120, w=FAKE, batch=2, n=1, cache=FAKE, kv_out=None):
+        return L.mla_down_kv_append(ctypes.byref(dd), hidden, hid, w, FAKE, FAKE, FAKE, 4, FAKE,
+                                    batch, n, cache, 100, None, kv_out, None)
+    assert call(hid=100) == mla.MLA_ERR_INVALID_ARG              # not a multiple of 8
+    assert call(hidden=None) == mla.MLA_ERR_INVALID_ARG
+    assert call(w=P(0x10008)) == mla.MLA_ERR_INVALID_ARG          # misaligned weight
+    assert call(kv_out=P(0x10004)) == mla.MLA_ERR_INVALID_ARG     # misaligned kv_out
+    assert call(dd=_dims(num_kv_groups=4, num_heads=128, rope_dim=64)) == mla.MLA_ERR_UNSUPPORTED
+    assert call(batch=0) == mla.MLA_OK
+    assert call(n=0) == mla.MLA_OK

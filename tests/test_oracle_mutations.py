@@ -37,6 +37,19 @@ MUTATIONS = {
     "out_up_bias_dropped": ("        o = o + as_f64(bias)", "        o = o + 0.0"),
     "append_groups_swapped": ("out[pages, rows, r:] = f32_to_bf16_bits(y).reshape(n, G * dr)",
                               "out[pages, rows, r:] = f32_to_bf16_bits(y[:, ::-1]).reshape(n, G * dr)"),
+    "kv_shared_no_inverse_rotation": ("o[..., dn:] = rope_rotate(o[..., dn:], theta, -q_pos[:, None])",
+                                      "o[..., dn:] = o[..., dn:]"),
+    "kv_shared_inverse_sign": ("o[..., dn:] = rope_rotate(o[..., dn:], theta, -q_pos[:, None])",
+                               "o[..., dn:] = rope_rotate(o[..., dn:], theta, q_pos[:, None])"),
+    "kv_shared_value_unrotated": ('o = np.einsum("ihl,ld->ihd", p, kv)',
+                                  'o = np.einsum("ihl,ld->ihd", p, np.concatenate([kv_nope, kv_pe], -1))'),
+    "kv_shared_query_unrotated": ("Q = np.concatenate([q_nope, q_rot], axis=-1)",
+                                  "Q = np.concatenate([q_nope, q_pe], axis=-1)"),
+    "absorbed_dropped_rope_term": ('np.einsum("ihe,le->ihl", q_rot[:, hs], k_rot))',
+                                   '0.0 * np.einsum("ihe,le->ihl", q_rot[:, hs], k_rot))'),
+    "down_kv_transposed_weight": ('np.einsum("...k,dk->...d", as_f64(hidden), as_f64(w_dkv))',
+                                  'np.einsum("...k,dk->...d", as_f64(hidden), as_f64(w_dkv)[::-1])'),
+    "down_kv_split_off_by_one": ("k_r = out[..., kv_lora_rank:]", "k_r = out[..., kv_lora_rank - 1:-1]"),
 }
 
 
