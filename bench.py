@@ -55,17 +55,18 @@ def algorithmic_work(cfg, seq_lens):
 
     Bytes: every cached row (D bf16) of every sequence, read once for all heads and query
     rows. FLOPs: 2*H*(r + d_r) for the scores and 2*H*r for o_ per query row and visible
-    cached token (padding of the rotary slots and of the UMMA tiles not counted)."""
+    cached token (padding of the rotary slots and of the UMMA tiles not counted); for the
+    single-latent K = V form the value is the whole row, 2*H*D + 2*H*D."""
     D = cfg.row_width
     tokens = int(np.sum(seq_lens, dtype=np.int64))
     nbytes = tokens * D * 2
     q, H, r, dr = cfg.q_len, cfg.num_heads, cfg.kv_lora_rank, cfg.rope_dim
     vis = 0
     for L in seq_lens:
-        for i in range(q):
-            vis += int(L) - q + i + 1 if cfg.causal else int(L)
-    flops = vis * (2 * H * (r + dr) + 2 * H * r)
-    return nbytes, flops
+        L = int(L)
+        vis += q * L - (q * (q - 1)) // 2 if cfg.causal else q * L
+    per = 4 * H * D if cfg.name.startswith("nanowhale") else 2 * H * (r + dr) + 2 * H * r
+    return nbytes, vis * per
 
 
 # Child process of ClockSampler: polls NVML in a tight loop (no GIL shared with the timed
@@ -351,30 +352,48 @@ def roofline_of(cfg, seq_lens, t_ms, peaks):
     return roof
 
 
-def time_decode(prob, cfg, n, stream, flush=None):
-    """Per-launch times (ms) of `n` back-to-back mla_decode_attn calls, CUDA events on the
-    launching stream; an L2 flush between launches when `flush` is given."""
+def time_calls(fn, n, stream, flush=None):
+    """Per-call times (ms) of `n` back-to-back calls of fn(stream), CUDA events on the
+    launching stream; an L2 flush between calls when `flush` is given."""
     import torch
-
-    import head_latent_attention_attn_b200 as mla
     evs = []
     for _ in range(n):
         if flush is not None:
             flush.zero_()
         a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         a.record(stream)
-        mla.mla_decode_attn(prob.dims, prob.q_ext, prob.cache, prob.block_table, prob.seq_lens,
-                            prob.max_seq_len, prob.workspace, prob.o_latent, prob.lse,
-                            causal=cfg.causal, num_splits=prob.num_splits, stream=stream)
+        fn(stream)
         b.record(stream)
         evs.append((a, b))
     torch.cuda.synchronize()
     return [a.elapsed_time(b) for a, b in evs]
 
 
-# Workloads timed after the headline in the default run: every other decode shape.
+def time_decode(prob, cfg, n, stream, flush=None, kv_shared=False):
+    """Per-launch times (ms) of `n` back-to-back mla_decode_attn calls (for the K = V form,
+    the decode over whole rows that kv_shared_step set up)."""
+    import head_latent_attention_attn_b200 as mla
+    if kv_shared:
+        args = (prob.kv_dims, prob.q_ext_kv, prob.o_lat_kv, prob.lse_kv, prob.ws_kv)
+    else:
+        args = (prob.dims, prob.q_ext, prob.o_latent, prob.lse, prob.workspace)
+    dims, q_ext, o_lat, lse, ws = args
+
+    def call(stream):
+        mla.mla_decode_attn(dims, q_ext, prob.cache, prob.block_table, prob.seq_lens,
+                            prob.max_seq_len, ws, o_lat, lse, causal=cfg.causal,
+                            num_splits=prob.num_splits, stream=stream)
+    return time_calls(call, n, stream, flush)
+
+
+# Workloads timed after the headline in the default run: every other decode shape, the
+# single-latent K = V layer, the prefill chunks and the fused down-projection + append.
 PER_CONFIG = ("tiny", "qwen25_7b", "qwen3_30b_a3b", "hybrid_1m_q1", "hybrid_1m_q4",
-              "hybrid_256k_q1", "hybrid_256k_q4")
+              "hybrid_256k_q1", "hybrid_256k_q4", "nanowhale_kv_shared",
+              "prefill_deepseek_v2_q64", "prefill_deepseek_v2_q256", "prefill_deepseek_v2_q1024",
+              "prefill_hybrid_q64", "prefill_hybrid_q256", "prefill_hybrid_q1024")
+DOWN_KV = ("deepseek_v2", "qwen3_30b_a3b")   # mla_down_kv_append at these decode batches
+OUT_PROJ = ("deepseek_v2",)                  # mla_out_proj at this decode batch
 DECODE_BLOCK = 60   # decode launches timed back to back for the roofline figure
 
 
@@ -403,47 +422,46 @@ def run_gpu(args, cfg, rank, world, dist):
             dist.barrier()
         torch.cuda.synchronize()
 
-    def one_step(ev):
-        # ev = (step_start, dec_start, dec_end, step_end)
-        ev[0].record(stream)
+    def one_step():
+        # The four calls back to back: each kernel is launched so that it may start while
+        # the previous one drains (programmatic dependent launch), so no event is recorded
+        # between them (a stream event between two kernels would serialise them).
         mla.mla_cache_append(prob.dims, prob.c_new, prob.k_new, prob.cos_q, prob.sin_q,
                              prob.block_table, prob.start_pos, prob.cache,
                              dev_error=prob.workspace.view(torch.int32)[:1], stream=stream)
         mla.mla_absorb_q(prob.dims, prob.q_nope, prob.q_pe, prob.cos_q, prob.sin_q, prob.w_uk,
                          prob.q_ext, stream=stream)
-        ev[1].record(stream)
         mla.mla_decode_attn(prob.dims, prob.q_ext, prob.cache, prob.block_table, prob.seq_lens,
                             prob.max_seq_len, prob.workspace, prob.o_latent, prob.lse,
                             causal=cfg.causal, num_splits=args.splits, stream=stream)
-        ev[2].record(stream)
         mla.mla_out_up(prob.dims, prob.o_latent, prob.w_uv, prob.o, bias=prob.bias, stream=stream)
-        ev[3].record(stream)
 
-    mk = lambda: [torch.cuda.Event(enable_timing=True) for _ in range(4)]  # noqa: E731
     for _ in range(args.warmup):
         if flush is not None:
             flush.zero_()
-        one_step(mk())
+        one_step()
     time_decode(prob, cfg, 3, stream, flush)
     barrier()
-    evs = []
     with ClockSampler(_gpu_id(local)) as clk:
         barrier()
         clk.mark_start()
-        for _ in range(args.steps):
-            if flush is not None:
-                flush.zero_()
-            e = mk()
-            one_step(e)
-            evs.append(e)
+        if flush is None:
+            # inputs larger than L2: the K steps run back to back between two events
+            t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            t0.record(stream)
+            for _ in range(args.steps):
+                one_step()
+            t1.record(stream)
+            torch.cuda.synchronize()
+            step_ms = [t0.elapsed_time(t1) / args.steps]
+        else:
+            # small caches: an L2 flush between steps, each step between its own events
+            step_ms = time_calls(lambda st: one_step(), args.steps, stream, flush)
         # the decode alone, back to back: the roofline figure (median of DECODE_BLOCK launches)
         dec_block = time_decode(prob, cfg, DECODE_BLOCK, stream, flush)
         barrier()
         clk.mark_end()
-    step_ms = [e[0].elapsed_time(e[3]) for e in evs]
-    dec_ms = [e[1].elapsed_time(e[2]) for e in evs]
     t_step = statistics.mean(step_ms)
-    t_dec_step = statistics.mean(dec_ms)
     t_dec = statistics.median(dec_block)
     t_dec_mean = statistics.mean(dec_block)
     status = mla.mla_get_device_status(prob.workspace.view(torch.int32)[:1])
@@ -513,8 +531,7 @@ def run_gpu(args, cfg, rank, world, dist):
         raise RuntimeError("end-to-end outputs differ from the device-resident step")
 
     # ---- max over ranks -------------------------------------------------------------------
-    t_step, t_dec, t_dec_mean, t_dec_step, t_e2e = max_over_ranks(
-        [t_step, t_dec, t_dec_mean, t_dec_step, t_e2e], dist, dev)
+    t_step, t_dec, t_dec_mean, t_e2e = max_over_ranks([t_step, t_dec, t_dec_mean, t_e2e], dist, dev)
     peaks = _peaks()
     tokens = cfg.batch * cfg.q_len
     value = world * tokens / (t_step * 1e-3)
@@ -531,7 +548,9 @@ def run_gpu(args, cfg, rank, world, dist):
         "config": dict(_config_json(cfg), l2=("cache > L2, no flush" if flush is None
                                               else "L2 flushed between launches (504 MB write)")),
         "decode_us": 1e3 * t_dec, "decode_us_mean": 1e3 * t_dec_mean,
-        "decode_launches_timed": DECODE_BLOCK, "decode_us_in_step_mean": 1e3 * t_dec_step,
+        "decode_launches_timed": DECODE_BLOCK,
+        "step_timing": ("K steps back to back between two events" if flush is None
+                        else "each step between its own events, L2 flushed before each"),
         "decode_gbs": roof["achieved_gbs"], "decode_tflops": roof["achieved_tflops"],
         "roofline": roof,
         "e2e": {"value": world * tokens / (t_e2e * 1e-3), "unit": "tokens/s",
@@ -554,28 +573,33 @@ def run_gpu(args, cfg, rank, world, dist):
 
 
 def per_config_block(args, head_cfg, dev, stream, dist, peaks):
-    """mla_decode_attn on every other decode workload, in the same process: the median of
-    DECODE_BLOCK launches, its roofline and the clocks seen while it ran. Every rank runs
-    the same workloads (the timings are maxed over ranks)."""
+    """mla_decode_attn on every other workload, in the same process: the median of
+    DECODE_BLOCK launches, its roofline and the clocks seen while it ran; then the fused
+    down-projection + append. Every rank runs the same workloads (timings maxed over ranks)."""
     import torch
 
-    from mla_inputs import CONFIGS, make_workload
+    import head_latent_attention_attn_b200 as mla
+    from mla_inputs import CONFIGS, make_down_kv_inputs, make_o_proj_inputs, make_workload
     from mla_inputs.device import DeviceProblem
     out = {}
     for name in PER_CONFIG:
         if name == head_cfg.name:
             continue
         cfg = CONFIGS[name]
+        kv = name.startswith("nanowhale")
         wl = make_workload(cfg)
         prob = DeviceProblem(wl, device=str(dev))
-        prob.step()
+        if kv:
+            prob.kv_shared_step()
+        else:
+            prob.step()
         nbytes, _ = algorithmic_work(cfg, wl.seq_lens)
         flush = (torch.empty(4 * L2_BYTES // 4, dtype=torch.float32, device=dev)
                  if nbytes < 2 * L2_BYTES else None)
-        time_decode(prob, cfg, 3, stream, flush)
+        time_decode(prob, cfg, 3, stream, flush, kv)
         with ClockSampler(_gpu_id(dev.index or 0)) as clk:
             clk.mark_start()
-            ms = time_decode(prob, cfg, DECODE_BLOCK, stream, flush)
+            ms = time_decode(prob, cfg, DECODE_BLOCK, stream, flush, kv)
             clk.mark_end()
         t_med, t_mean = max_over_ranks([statistics.median(ms), statistics.mean(ms)], dist, dev)
         out[name] = {"decode_us": 1e3 * t_med, "decode_us_mean": 1e3 * t_mean,
@@ -585,6 +609,80 @@ def per_config_block(args, head_cfg, dev, stream, dist, peaks):
                      "l2": "cache > L2, no flush" if flush is None else "L2 flushed between launches",
                      "clocks": clk.summary()}
         del prob, flush, wl
+        torch.cuda.empty_cache()
+    # einsums (5) and (6) fused (mla_out_proj) at the DeepSeek-V2 decode batch
+    for name in OUT_PROJ:
+        cfg = CONFIGS[name]
+        rows = cfg.batch * cfg.q_len
+        dims = mla.make_dims(cfg.num_heads, cfg.num_kv_groups, cfg.kv_lora_rank, cfg.qk_nope_dim,
+                             cfg.rope_dim, cfg.v_head_dim, cfg.page_size, cfg.softmax_scale)
+        g = torch.Generator(device=dev)
+        g.manual_seed(cfg.seed)
+        o_lat = (torch.randn(rows, cfg.num_heads, cfg.kv_lora_rank, device=dev, generator=g) /
+                 math.sqrt(cfg.kv_lora_rank)).to(torch.bfloat16)
+        w_uv = make_workload(cfg.with_(context=64, lens_range=None, batch=1)).w_uv.to(dev)
+        w_o, _ = make_o_proj_inputs(cfg)
+        w_o = w_o.to(dev)
+        o = torch.empty(rows, cfg.num_heads, cfg.v_head_dim, dtype=torch.bfloat16, device=dev)
+        u = torch.empty(rows, cfg.hidden_size, dtype=torch.bfloat16, device=dev)
+        ws = torch.zeros(mla.mla_out_proj_workspace_size(dims, cfg.hidden_size, rows),
+                         dtype=torch.uint8, device=dev)
+        flush = torch.empty(4 * L2_BYTES // 4, dtype=torch.float32, device=dev)
+
+        def call(stream, dims=dims, o_lat=o_lat, w_uv=w_uv, w_o=w_o, ws=ws, o=o, u=u):
+            mla.mla_out_proj(dims, o_lat, w_uv, w_o, ws, o, u, stream=stream)
+        time_calls(call, 3, stream, flush)
+        with ClockSampler(_gpu_id(dev.index or 0)) as clk:
+            clk.mark_start()
+            ms = time_calls(call, DECODE_BLOCK, stream, flush)
+            clk.mark_end()
+        t_med, t_mean = max_over_ranks([statistics.median(ms), statistics.mean(ms)], dist, dev)
+        nbytes = (w_uv.numel() + w_o.numel() + o_lat.numel() + o.numel() + u.numel()) * 2
+        flops = 2 * rows * cfg.num_heads * cfg.v_head_dim * (cfg.kv_lora_rank + cfg.hidden_size)
+        gbs = nbytes / (t_med * 1e-3) / 1e9
+        out[f"out_proj[{name}]"] = {
+            "us": 1e3 * t_med, "us_mean": 1e3 * t_mean, "launches": DECODE_BLOCK, "rows": rows,
+            "hidden_size": cfg.hidden_size,
+            "roofline": {"bound": "hbm", "achieved": gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                         "frac": gbs / peaks["hbm_gbs"], "algorithmic_bytes_per_launch": nbytes,
+                         "algorithmic_flops_per_launch": flops, "peak_source": peaks["source"],
+                         "kernel": "oproj_kernel (einsum 5 then einsum 6, one cooperative launch)"},
+            "l2": "L2 flushed between launches", "clocks": clk.summary()}
+        del o_lat, w_uv, w_o, o, u, ws, flush
+        torch.cuda.empty_cache()
+    for name in DOWN_KV:
+        cfg = CONFIGS[name]
+        wl = make_workload(cfg.with_(context=128, lens_range=None))
+        prob = DeviceProblem(wl, device=str(dev))
+        hidden, w_dkv = make_down_kv_inputs(cfg, cfg.q_len)
+        hidden, w_dkv = hidden.to(dev), w_dkv.to(dev)
+        flush = torch.empty(4 * L2_BYTES // 4, dtype=torch.float32, device=dev)
+        ws = torch.zeros(mla.mla_down_kv_workspace_size(prob.dims, cfg.batch, cfg.q_len),
+                         dtype=torch.uint8, device=dev)
+
+        def call(stream, prob=prob, hidden=hidden, w_dkv=w_dkv, ws=ws):
+            mla.mla_down_kv_append(prob.dims, hidden, w_dkv, prob.cos_q, prob.sin_q,
+                                   prob.block_table, prob.start_pos, prob.cache, ws,
+                                   dev_error=prob.err, stream=stream)
+        time_calls(call, 3, stream, flush)
+        with ClockSampler(_gpu_id(dev.index or 0)) as clk:
+            clk.mark_start()
+            ms = time_calls(call, DECODE_BLOCK, stream, flush)
+            clk.mark_end()
+        t_med, t_mean = max_over_ranks([statistics.median(ms), statistics.mean(ms)], dist, dev)
+        rows = cfg.batch * cfg.q_len
+        nbytes = (w_dkv.numel() + hidden.numel() + rows * cfg.row_width) * 2
+        flops = 2 * rows * cfg.row_width * cfg.hidden_size
+        gbs = nbytes / (t_med * 1e-3) / 1e9
+        out[f"down_kv_append[{name}]"] = {
+            "us": 1e3 * t_med, "us_mean": 1e3 * t_mean, "launches": DECODE_BLOCK,
+            "rows": rows, "hidden_size": cfg.hidden_size,
+            "roofline": {"bound": "hbm", "achieved": gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                         "frac": gbs / peaks["hbm_gbs"], "algorithmic_bytes_per_launch": nbytes,
+                         "algorithmic_flops_per_launch": flops, "peak_source": peaks["source"],
+                         "kernel": "wgemm_kernel (fused cache-append epilogue)"},
+            "l2": "L2 flushed between launches", "clocks": clk.summary()}
+        del prob, flush, hidden, w_dkv, wl, ws
         torch.cuda.empty_cache()
     return out
 

@@ -36,7 +36,8 @@ C_SYMBOLS = ("mla_row_width", "mla_status_string", "mla_cache_append", "mla_abso
              "mla_decode_workspace_size", "mla_decode_attn", "mla_out_up",
              "mla_get_device_status", "mla_decode_attn_noalloc", "mla_selftest_wait_timeout",
              "mla_kv_shared_decode_dims", "mla_kv_shared_query", "mla_kv_shared_output",
-             "mla_down_kv_append")
+             "mla_down_kv_workspace_size", "mla_down_kv_append", "mla_out_proj_workspace_size",
+             "mla_out_proj")
 
 
 class MlaError(RuntimeError):
@@ -105,9 +106,16 @@ def lib() -> ctypes.CDLL:
     for fn in (L.mla_kv_shared_query, L.mla_kv_shared_output):
         fn.argtypes = [D, _P, _P, _P, _I32, _I32, _P, _P]
         fn.restype = _I32
+    L.mla_down_kv_workspace_size.argtypes = [D, _I32, _I32]
+    L.mla_down_kv_workspace_size.restype = ctypes.c_size_t
     L.mla_down_kv_append.argtypes = [D, _P, _I32, _P, _P, _P, _P, _I32, _P, _I32, _I32, _P,
-                                     _I64, _P, _P, _P]
+                                     _I64, _P, _P, _P, ctypes.c_size_t, _P]
     L.mla_down_kv_append.restype = _I32
+    L.mla_out_proj_workspace_size.argtypes = [D, _I32, _I32]
+    L.mla_out_proj_workspace_size.restype = ctypes.c_size_t
+    L.mla_out_proj.argtypes = [D, _P, _P, _I64, _P, _P, _P, _I32, _I32, _P, ctypes.c_size_t, _P,
+                               _P, _P]
+    L.mla_out_proj.restype = _I32
     _lib = L
     return L
 
@@ -174,11 +182,17 @@ def mla_cache_append(dims: MlaDims, c_kv, k_r, rope_cos, rope_sin, block_table, 
     _check(st, "mla_cache_append")
 
 
+def mla_down_kv_workspace_size(dims: MlaDims, batch: int, n_new: int) -> int:
+    return int(lib().mla_down_kv_workspace_size(ctypes.byref(dims), int(batch), int(n_new)))
+
+
 def mla_down_kv_append(dims: MlaDims, hidden, w_dkv, rope_cos, rope_sin, block_table,
-                       start_pos, cache, dev_error=None, kv_out=None, stream=None) -> None:
+                       start_pos, cache, workspace, dev_error=None, kv_out=None,
+                       stream=None) -> None:
     """[c_kv ; k_r] = w_dkv @ hidden (bf16) for hidden [B, n, hidden_dim], written into cache
     [P, ps, D] exactly as mla_cache_append would; kv_out [B, n, D] optionally receives the
-    projection before the rotation."""
+    projection before the rotation; workspace is a zeroed uint8 CUDA tensor of
+    mla_down_kv_workspace_size bytes (left zero by the call)."""
     B, n, hid = hidden.shape
     G, dr, D = dims.num_kv_groups, dims.rope_dim, dims.row_width
     _need(hidden, "hidden", torch.bfloat16)
@@ -197,11 +211,13 @@ def mla_down_kv_append(dims: MlaDims, hidden, w_dkv, rope_cos, rope_sin, block_t
         _need(dev_error, "dev_error", torch.int32)
     if kv_out is not None:
         _need(kv_out, "kv_out", torch.bfloat16, (B, n, D))
+    _need(workspace, "workspace", torch.uint8)
     st = lib().mla_down_kv_append(ctypes.byref(dims), _ptr(hidden), hid, _ptr(w_dkv),
                                   _ptr(rope_cos if dr > 0 else None),
                                   _ptr(rope_sin if dr > 0 else None), _ptr(block_table),
                                   block_table.shape[1], _ptr(start_pos), B, n, _ptr(cache),
-                                  cache.shape[0], _ptr(dev_error), _ptr(kv_out), _stream(stream))
+                                  cache.shape[0], _ptr(dev_error), _ptr(kv_out), _ptr(workspace),
+                                  workspace.numel(), _stream(stream))
     _check(st, "mla_down_kv_append")
 
 
@@ -340,6 +356,45 @@ def mla_kv_shared_output(dims: MlaDims, o_latent, rope_cos, rope_sin, o, stream=
                       rope_cos, rope_sin, o, stream)
 
 
+def mla_out_proj_workspace_size(dims: MlaDims, hidden: int, rows: int) -> int:
+    return int(lib().mla_out_proj_workspace_size(ctypes.byref(dims), int(hidden), int(rows)))
+
+
+def mla_out_proj(dims: MlaDims, o_latent, w_uv, w_o, workspace, o, u, bias_v=None, bias_o=None,
+                 w_uv_head_stride: Optional[int] = None, stream=None) -> None:
+    """o [rows, H, d_v] = W_UV o_latent (+ bias_v) and u [rows, hidden] = W_o o (+ bias_o) in
+    one kernel; w_o is [hidden, H * d_v]; workspace a zeroed uint8 CUDA tensor."""
+    H, r, dv = dims.num_heads, dims.kv_lora_rank, dims.v_head_dim
+    _need(o_latent, "o_latent", torch.bfloat16)
+    if o_latent.shape[-2:] != (H, r):
+        raise MlaError("o_latent must end in [H, r]", MLA_ERR_INVALID_ARG)
+    rows = o_latent.numel() // (H * r)
+    _need(w_o, "w_o", torch.bfloat16)
+    if w_o.dim() != 2 or w_o.shape[1] != H * dv:
+        raise MlaError("w_o must be [hidden, H * d_v]", MLA_ERR_INVALID_ARG)
+    hidden = w_o.shape[0]
+    _need(o, "o", torch.bfloat16)
+    if o.numel() != rows * H * dv:
+        raise MlaError("o must hold rows * H * d_v elements", MLA_ERR_INVALID_ARG)
+    _need(u, "u", torch.bfloat16)
+    if u.numel() != rows * hidden:
+        raise MlaError("u must hold rows * hidden elements", MLA_ERR_INVALID_ARG)
+    if w_uv_head_stride is None:
+        _need(w_uv, "w_uv", torch.bfloat16, (H, dv, r))
+        w_uv_head_stride = dv * r
+    else:
+        _need(w_uv, "w_uv", torch.bfloat16)
+    if bias_v is not None:
+        _need(bias_v, "bias_v", torch.bfloat16, (H, dv))
+    if bias_o is not None:
+        _need(bias_o, "bias_o", torch.bfloat16, (hidden,))
+    _need(workspace, "workspace", torch.uint8)
+    st = lib().mla_out_proj(ctypes.byref(dims), _ptr(o_latent), _ptr(w_uv), int(w_uv_head_stride),
+                            _ptr(bias_v), _ptr(w_o), _ptr(bias_o), hidden, rows, _ptr(workspace),
+                            workspace.numel(), _ptr(o), _ptr(u), _stream(stream))
+    _check(st, "mla_out_proj")
+
+
 def mla_get_device_status(dev_error, reset: bool = False, stream=None) -> int:
     """Synchronise and read a device error word (an int32 tensor, or a decode workspace)."""
     if dev_error.device.type != "cuda":
@@ -371,4 +426,6 @@ def mla_decode_step(dims: MlaDims, *, c_kv_new, k_r_new, cos_new, sin_new, start
 __all__ = ["MlaDims", "MlaError", "make_dims", "lib", "mla_row_width", "mla_cache_append",
            "mla_absorb_q", "mla_decode_workspace_size", "mla_decode_attn", "mla_out_up",
            "mla_decode_attn_noalloc", "mla_kv_shared_decode_dims", "mla_kv_shared_query",
-           "mla_kv_shared_output", "mla_down_kv_append", "mla_get_device_status", "mla_decode_step", "C_SYMBOLS", "STATUS_NAMES"]
+           "mla_kv_shared_output", "mla_down_kv_workspace_size", "mla_down_kv_append",
+           "mla_out_proj_workspace_size",
+           "mla_out_proj", "mla_get_device_status", "mla_decode_step", "C_SYMBOLS", "STATUS_NAMES"]

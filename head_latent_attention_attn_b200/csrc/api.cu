@@ -269,6 +269,7 @@ mla_status mla_absorb_q(const mla_dims* dims, const void* q_nope, const void* q_
   p.rows = int32_t(rows);
   p.heads = H;
   p.a_mn = 1;
+  p.splits = 1;
   p.q_pe = dims->rope_dim > 0 ? static_cast<const uint16_t*>(q_pe) : nullptr;
   p.rope_cos = rope_cos;
   p.rope_sin = rope_sin;
@@ -317,15 +318,29 @@ mla_status mla_out_up(const mla_dims* dims, const void* o_latent, const void* w_
   p.rows = rows;
   p.heads = H;
   p.a_mn = 0;
+  p.splits = 1;
   p.q_pe = nullptr;
   return launch_wgemm(p, nr, num_sms(), as_stream(stream)) == cudaSuccess ? MLA_OK : MLA_ERR_CUDA;
+}
+
+// Workspace of mla_down_kv_append: fp32 sums of the split K ([rows, D]) and one counter per
+// output tile (at most ceil(r/128) + 1 feature tiles per 16-row tile).
+static size_t down_kv_ws(const mla_dims* d, int64_t rows) {
+  const int64_t tiles = (int64_t(d->kv_lora_rank + 127) / 128 + 1) * ((rows + 15) / 16);
+  return (size_t(tiles) * 4 + 255) / 256 * 256 + size_t(rows) * size_t(row_width(d)) * 4;
+}
+
+size_t mla_down_kv_workspace_size(const mla_dims* dims, int32_t batch, int32_t n_new) {
+  if (check_dims(dims) != MLA_OK || batch < 0 || n_new < 0) return 0;
+  return down_kv_ws(dims, int64_t(batch) * n_new);
 }
 
 mla_status mla_down_kv_append(const mla_dims* dims, const void* hidden, int32_t hidden_dim,
                               const void* w_dkv, const float* rope_cos, const float* rope_sin,
                               const int32_t* block_table, int32_t max_pages_per_seq,
                               const int32_t* start_pos, int32_t batch, int32_t n_new, void* cache,
-                              int64_t num_pages, int32_t* dev_error, void* kv_out, void* stream) {
+                              int64_t num_pages, int32_t* dev_error, void* kv_out,
+                              void* workspace, size_t workspace_bytes, void* stream) {
   mla_status st = check_dims(dims);
   if (st != MLA_OK) return st;
   if (batch < 0 || n_new < 0 || hidden_dim <= 0 || hidden_dim % 8 != 0 ||
@@ -341,6 +356,8 @@ mla_status mla_down_kv_append(const mla_dims* dims, const void* hidden, int32_t 
   if (R > 128) return MLA_ERR_UNSUPPORTED;        // the rotary features share one tile
   const int64_t rows = int64_t(batch) * n_new;
   if (rows > int64_t(65535) * 128) return MLA_ERR_UNSUPPORTED;
+  if (!workspace || !aligned(workspace, 256) || workspace_bytes < down_kv_ws(dims, rows))
+    return MLA_ERR_WORKSPACE;
   const int D = row_width(dims);
   WGemmParams p{};
   {
@@ -381,7 +398,124 @@ mla_status mla_down_kv_append(const mla_dims* dims, const void* hidden, int32_t 
   p.page_size = dims->page_size;
   p.lat_r = r;
   p.lat_tiles = (r + 127) / 128;
+  // K (the model width) split so that the (feature tile, split, row tile) items fill the GPU
+  const int n_mt = p.lat_tiles + (R > 0 ? 1 : 0);
+  const int64_t n_nt = (rows + nr - 1) / nr;
+  const int nk = (hidden_dim + 63) / 64;
+  p.splits = int(std::max<int64_t>(1, std::min<int64_t>(nk, num_sms() / (n_mt * n_nt))));
+  const int64_t tiles = int64_t(n_mt) * n_nt;
+  p.tile_done = static_cast<int32_t*>(workspace);
+  p.acc = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) +
+                                   (size_t(tiles) * 4 + 255) / 256 * 256);
   return launch_wgemm(p, nr, num_sms(), as_stream(stream)) == cudaSuccess ? MLA_OK : MLA_ERR_CUDA;
+}
+
+}  // extern "C"
+
+namespace {
+
+// Workspace of mla_out_proj: counters, then the fp32 partials of stage B's K splits.
+struct OProjPlan {
+  int nr, n_nt, n_mt, splits, items, grid;
+  size_t head_off, tile_off, part_off, bytes;
+};
+
+mla_status plan_oproj(const mla_dims* d, int32_t hidden, int32_t rows, OProjPlan* P) {
+  mla_status st = check_dims(d);
+  if (st != MLA_OK) return st;
+  if (hidden <= 0 || hidden % 8 != 0 || rows < 0) return MLA_ERR_INVALID_ARG;
+  if (d->v_head_dim % 64 != 0) return MLA_ERR_UNSUPPORTED;   // K splits on whole 64-blocks
+  if (int64_t(rows) > int64_t(65535) * 128) return MLA_ERR_UNSUPPORTED;
+  const int H = d->num_heads;
+  P->nr = pick_nr(std::max(rows, 1));
+  P->n_nt = (std::max(rows, 1) + P->nr - 1) / P->nr;
+  P->n_mt = (hidden + 127) / 128;
+  const int sms = num_sms();
+  P->splits = std::max(1, std::min(H, sms / (P->n_mt * P->n_nt)));
+  P->items = H * ((d->v_head_dim + 127) / 128) * P->n_nt + P->n_mt * P->splits * P->n_nt;
+  P->grid = std::min(P->items, sms);
+  size_t off = 256;                              // cta_done + padding
+  P->head_off = off;
+  off = align256(off + size_t(H) * 4);
+  P->tile_off = off;
+  off = align256(off + size_t(P->n_mt) * P->n_nt * 4);
+  P->part_off = off;
+  off += size_t(P->splits) * size_t(std::max(rows, 1)) * size_t(hidden) * 4;
+  P->bytes = off;
+  return MLA_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+size_t mla_out_proj_workspace_size(const mla_dims* dims, int32_t hidden, int32_t rows) {
+  OProjPlan P;
+  return plan_oproj(dims, hidden, rows, &P) == MLA_OK ? P.bytes : 0;
+}
+
+mla_status mla_out_proj(const mla_dims* dims, const void* o_latent, const void* w_uv,
+                        int64_t w_uv_head_stride, const void* bias_v, const void* w_o,
+                        const void* bias_o, int32_t hidden, int32_t rows, void* workspace,
+                        size_t workspace_bytes, void* o, void* u, void* stream) {
+  OProjPlan P;
+  mla_status st = plan_oproj(dims, hidden, rows, &P);
+  if (st != MLA_OK) return st;
+  if (rows == 0) return MLA_OK;
+  const int H = dims->num_heads, r = dims->kv_lora_rank, dv = dims->v_head_dim;
+  if (!o_latent || !w_uv || !w_o || !o || !u) return MLA_ERR_INVALID_ARG;
+  if (w_uv_head_stride < int64_t(dv) * r || w_uv_head_stride % 8 != 0) return MLA_ERR_INVALID_ARG;
+  if (!aligned(o_latent, 16) || !aligned(w_uv, 16) || !aligned(w_o, 16) || !aligned(o, 16) ||
+      !aligned(u, 16))
+    return MLA_ERR_INVALID_ARG;
+  if (!workspace || !aligned(workspace, 256) || workspace_bytes < P.bytes) return MLA_ERR_WORKSPACE;
+  OProjParams p{};
+  {
+    const uint64_t d3[3] = {uint64_t(r), uint64_t(dv), uint64_t(H)};
+    const uint64_t s3[2] = {uint64_t(r) * 2, uint64_t(w_uv_head_stride) * 2};
+    const uint32_t box[3] = {64, 128, 1};
+    if (!encode_bf16_map(&p.tm_wuv, w_uv, 3, d3, s3, box, CU_TENSOR_MAP_SWIZZLE_128B))
+      return MLA_ERR_CUDA;
+  }
+  {
+    const uint64_t d3[3] = {uint64_t(r), uint64_t(H), uint64_t(rows)};
+    const uint64_t s3[2] = {uint64_t(r) * 2, uint64_t(H) * r * 2};
+    const uint32_t box[3] = {64, 1, uint32_t(P.nr)};
+    if (!encode_bf16_map(&p.tm_ol, o_latent, 3, d3, s3, box, CU_TENSOR_MAP_SWIZZLE_128B))
+      return MLA_ERR_CUDA;
+  }
+  const uint64_t K = uint64_t(H) * dv;
+  {
+    const uint64_t d2[2] = {K, uint64_t(hidden)};
+    const uint64_t s2[1] = {K * 2};
+    const uint32_t box[2] = {64, 128};
+    if (!encode_bf16_map(&p.tm_wo, w_o, 2, d2, s2, box, CU_TENSOR_MAP_SWIZZLE_128B))
+      return MLA_ERR_CUDA;
+  }
+  {
+    const uint64_t d2[2] = {K, uint64_t(rows)};
+    const uint64_t s2[1] = {K * 2};
+    const uint32_t box[2] = {64, uint32_t(P.nr)};
+    if (!encode_bf16_map(&p.tm_o, o, 2, d2, s2, box, CU_TENSOR_MAP_SWIZZLE_128B))
+      return MLA_ERR_CUDA;
+  }
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  p.o = static_cast<uint16_t*>(o);
+  p.u = static_cast<uint16_t*>(u);
+  p.bias_v = static_cast<const uint16_t*>(bias_v);
+  p.bias_o = static_cast<const uint16_t*>(bias_o);
+  p.part = reinterpret_cast<float*>(ws + P.part_off);
+  p.head_done = reinterpret_cast<int32_t*>(ws + P.head_off);
+  p.tile_done = reinterpret_cast<int32_t*>(ws + P.tile_off);
+  p.cta_done = reinterpret_cast<int32_t*>(ws + 4);
+  p.dev_error = reinterpret_cast<int32_t*>(ws);
+  p.H = H;
+  p.r = r;
+  p.dv = dv;
+  p.hidden = hidden;
+  p.rows = rows;
+  p.splits = P.splits;
+  return launch_oproj(p, P.nr, P.grid, as_stream(stream)) == cudaSuccess ? MLA_OK : MLA_ERR_CUDA;
 }
 
 size_t mla_decode_workspace_size(const mla_dims* dims, int32_t batch, int32_t q_len,

@@ -219,6 +219,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     tmem_relinquish();
   }
 
+  // set-up above may overlap the previous kernel; from here on global memory is touched
+  grid_dep_wait();
+  grid_dep_launch();
   // ---- schedule: this CTA's tile range [r0, r1) in its row block, first sequence -------
   // The row blocks of a sequence are worked on in lockstep by neighbouring CTAs, so the
   // second read of every page is served from L2.
@@ -610,6 +613,8 @@ __global__ void __launch_bounds__(kThreads, 1)
 __global__ void __launch_bounds__(128) mla_combine_kernel(const CombineParams p) {
   __shared__ float part[4][512];
   __shared__ float lse_s;
+  grid_dep_wait();
+  grid_dep_launch();
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int u = int(blockIdx.x / unsigned(p.ncol));
   const int n = int(blockIdx.x % unsigned(p.ncol));
@@ -695,6 +700,8 @@ __global__ void __launch_bounds__(128) mla_combine_kernel(const CombineParams p)
 // memory. Lanes own latents 4 * lane + 128 k + {0..3}: every load of a piece's bf16 row is
 // one 256-byte coalesced segment per warp.
 __global__ void __launch_bounds__(128) mla_combine_rows_kernel(const CombineParams p) {
+  grid_dep_wait();
+  grid_dep_launch();
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int64_t gw = int64_t(blockIdx.x) * 4 + warp;
   if (gw >= int64_t(p.units) * p.ncol) return;
@@ -787,12 +794,11 @@ cudaError_t launch_combine(const CombineParams& p, cudaStream_t stream) {
   if (rows <= 0 || rows > 0x7fffffffLL || p.r > 512 || p.r % 4 != 0) return cudaErrorInvalidValue;
   if (int64_t(p.vgrid) <= 4 * int64_t(p.units)) {
     // a few pieces per unit: one warp per row
-    mla_combine_rows_kernel<<<unsigned((rows + 3) / 4), 128, 0, stream>>>(p);
-  } else {
-    // many pieces per unit: the four warps of a block split one row's pieces
-    mla_combine_kernel<<<unsigned(rows), 128, 0, stream>>>(p);
+    return launch_pdl(mla_combine_rows_kernel, dim3(unsigned((rows + 3) / 4)), dim3(128), 0,
+                      stream, 1, p);
   }
-  return cudaGetLastError();
+  // many pieces per unit: the four warps of a block split one row's pieces
+  return launch_pdl(mla_combine_kernel, dim3(unsigned(rows)), dim3(128), 0, stream, 1, p);
 }
 
 template <int NCOL>
@@ -801,8 +807,7 @@ static cudaError_t launch_decode_n(const DecodeParams& p, dim3 grid, size_t smem
   cudaError_t e = cudaFuncSetAttribute(mla_decode_kernel<NCOL>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
   if (e != cudaSuccess) return e;
-  mla_decode_kernel<NCOL><<<grid, kThreads, smem, stream>>>(p);
-  return cudaGetLastError();
+  return launch_pdl(mla_decode_kernel<NCOL>, grid, dim3(kThreads), smem, stream, 1, p);
 }
 
 cudaError_t launch_decode(const DecodeParams& p, int ncol, dim3 grid, size_t smem,

@@ -311,6 +311,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     tmem_alloc(tmem_slot, kTmemCols);
     tmem_relinquish();
   }
+  // set-up above may overlap the previous kernel; from here on global memory is touched
+  grid_dep_wait();
+  grid_dep_launch();
   // Both CTAs of the cluster compute the same range (same pair index).
   find_tile_range<kThreads>(p, vc, vgrid, blockIdx.x == 0, warp_sum, sched);
   tc_fence_before();
@@ -895,21 +898,7 @@ cudaError_t launch_decode_pair(const DecodeParams& p, dim3 grid, size_t smem,
   cudaError_t e = cudaFuncSetAttribute(mla_decode_pair_kernel,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
   if (e != cudaSuccess) return e;
-  cudaLaunchConfig_t cfg = {};
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeClusterDimension;
-  attr[0].val.clusterDim.x = 2;
-  attr[0].val.clusterDim.y = 1;
-  attr[0].val.clusterDim.z = 1;
-  cfg.gridDim = grid;
-  cfg.blockDim = dim3(kThreads);
-  cfg.dynamicSmemBytes = smem;
-  cfg.stream = stream;
-  cfg.attrs = attr;
-  cfg.numAttrs = 1;
-  e = cudaLaunchKernelEx(&cfg, mla_decode_pair_kernel, p);
-  if (e != cudaSuccess) return e;
-  return cudaGetLastError();
+  return launch_pdl(mla_decode_pair_kernel, grid, dim3(kThreads), smem, stream, 2, p);
 }
 
 }  // namespace mla

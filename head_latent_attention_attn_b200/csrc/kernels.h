@@ -5,7 +5,39 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <utility>
+
 namespace mla {
+
+// Launch `kernel` with programmatic dependent launch (it may start while the previous kernel
+// on `stream` runs; see grid_dep_wait in ptx.cuh) and, when cluster_x > 1, clusters of
+// cluster_x CTAs.
+template <typename... KArgs, typename... Args>
+inline cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                              cudaStream_t stream, int cluster_x, Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cudaLaunchAttribute attr[2];
+  int n = 0;
+  attr[n].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[n].val.programmaticStreamSerializationAllowed = 1;
+  ++n;
+  if (cluster_x > 1) {
+    attr[n].id = cudaLaunchAttributeClusterDimension;
+    attr[n].val.clusterDim.x = unsigned(cluster_x);
+    attr[n].val.clusterDim.y = 1;
+    attr[n].val.clusterDim.z = 1;
+    ++n;
+  }
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cfg.attrs = attr;
+  cfg.numAttrs = unsigned(n);
+  cudaError_t e = cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
+  if (e != cudaSuccess) return e;
+  return cudaGetLastError();
+}
 
 // ---- mla_cache_append -------------------------------------------------------------------
 struct AppendParams {
@@ -61,10 +93,36 @@ struct WGemmParams {
   uint16_t* kv_out;          // [rows, D] bf16 GEMM output before the rotation, or null
   int64_t num_pages;
   int32_t max_pages, n_new, page_size, lat_r, lat_tiles;
+  // K split across CTAs (fused append only; 1 elsewhere): split s of an output tile sums
+  // the K blocks [s nk / splits, (s + 1) nk / splits) into acc with fp32 reductions, and the
+  // last split to finish (tile_done) reads the sums back, clears them and writes the rows.
+  int32_t splits;
+  float* acc;                // [rows, D] fp32, zero between calls
+  int32_t* tile_done;        // [tiles], zero between calls
 };
 // max_ctas: the persistent grid's size limit (one CTA per SM). With p.cache set the
 // output goes into the paged cache (see WGemmParams) instead of p.out.
 cudaError_t launch_wgemm(const WGemmParams& p, int nr, int max_ctas, cudaStream_t stream);
+
+// ---- mla_out_proj: einsum (5) then einsum (6) in one cooperative kernel (oproj.cu) -------
+struct OProjParams {
+  CUtensorMap tm_wuv;        // 3D {r, d_v, H} (head stride), box {64, 128, 1}
+  CUtensorMap tm_ol;         // 3D {r, H, rows}, box {64, 1, NR}: o_latent
+  CUtensorMap tm_wo;         // 2D {H*d_v, hidden}, box {64, 128}: W_o as [hidden][H*d_v]
+  CUtensorMap tm_o;          // 2D {H*d_v, rows}, box {64, NR}: stage A's output o
+  uint16_t* o;               // [rows, H, d_v] bf16 (stage A output, stage B input)
+  uint16_t* u;               // [rows, hidden] bf16
+  const uint16_t* bias_v;    // [H, d_v] or null
+  const uint16_t* bias_o;    // [hidden] or null
+  float* part;               // [splits, rows, hidden] fp32 partials of stage B
+  int32_t* head_done;        // [H] stage-A items done per head (cleared by the kernel)
+  int32_t* tile_done;        // [tiles] stage-B splits done per output tile (cleared)
+  int32_t* cta_done;         // [1] CTAs finished (cleared)
+  int32_t* dev_error;
+  int32_t H, r, dv, hidden, rows, splits;
+};
+size_t oproj_smem_bytes(int nr);
+cudaError_t launch_oproj(const OProjParams& p, int nr, int grid, cudaStream_t stream);
 
 // ---- mla_decode_attn -----------------------------------------------------------------------
 constexpr int kDecodeTok = 64;        // tokens per tile = one cache page

@@ -17,6 +17,8 @@
 namespace mla {
 
 __global__ void __launch_bounds__(256) kv_shared_rotate_kernel(KvSharedParams p) {
+  grid_dep_wait();
+  grid_dep_launch();
   const int64_t row = (int64_t(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
   const int lane = threadIdx.x & 31;
   if (row >= p.rows) return;
@@ -46,8 +48,8 @@ cudaError_t launch_kv_shared_rotate(const KvSharedParams& p, cudaStream_t stream
   if (p.rows == 0) return cudaSuccess;
   const int threads = 256;
   const int64_t blocks = (p.rows * 32 + threads - 1) / threads;
-  kv_shared_rotate_kernel<<<dim3(unsigned(blocks)), threads, 0, stream>>>(p);
-  return cudaGetLastError();
+  return launch_pdl(kv_shared_rotate_kernel, dim3(unsigned(blocks)), dim3(threads), 0, stream, 1,
+                    p);
 }
 
 }  // namespace mla

@@ -156,6 +156,27 @@ MLA_DEVICE void tma_prefetch_l2_2d(const CUtensorMap* map, int32_t x, int32_t y)
                : "memory");
 }
 
+// Bring a tile of a 3D tensor map into L2.
+MLA_DEVICE void tma_prefetch_l2_3d(const CUtensorMap* map, int32_t x, int32_t y, int32_t z) {
+  asm volatile("cp.async.bulk.prefetch.tensor.3d.L2.global.tile [%0, {%1, %2, %3}];" ::"l"(
+                   reinterpret_cast<uint64_t>(map)),
+               "r"(x), "r"(y), "r"(z)
+               : "memory");
+}
+
+// ---------------------------------------------------------------------------------------
+// Programmatic dependent launch. Every kernel here is launched so that it may start while
+// the kernel before it on the stream is still running. Each thread calls grid_dep_wait()
+// before its first access to global memory that another kernel may write (inputs, outputs,
+// workspace), which returns once the preceding grid has completed and its memory is
+// visible; before that only set-up (barriers, TMEM, tensor-map and L2 prefetches) runs.
+// grid_dep_launch() lets the next kernel on the stream be scheduled once every CTA of this
+// grid has issued it (or exited), so no CTA of the next grid can hold an SM that a CTA of
+// this grid still needs. Both are no-ops when there is no such neighbour.
+// ---------------------------------------------------------------------------------------
+MLA_DEVICE void grid_dep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+MLA_DEVICE void grid_dep_launch() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
 MLA_DEVICE void prefetch_tensormap(const CUtensorMap* map) {
   asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
 }

@@ -46,17 +46,26 @@ MLA_DEVICE uint8_t* align1024(uint8_t* p) {
 // Work item `it` -> (head, first output feature, first activation row). For the fused
 // append the last feature tile is the rotary one and starts at feature r (all of a
 // group's rotation pairs then sit in one tile); the others are 128-aligned latent tiles.
+// With K split in `splits` parts, items are (head, feature tile, split, row tile) and an
+// item covers the K blocks [kb0, kb1).
 struct WgItem {
-  int h, m0, n0, mt;
-  MLA_DEVICE WgItem(int it, int n_mt, int n_nt, int nr, int rope_tile_m0) {
+  int h, m0, n0, mt, s, kb0, kb1, tile;
+  MLA_DEVICE WgItem(int it, int n_mt, int n_nt, int nr, int rope_tile_m0, int splits, int nk) {
     const int nt = it % n_nt;
-    const int hm = it / n_nt;
+    const int rest = it / n_nt;
+    s = rest % splits;
+    const int hm = rest / splits;
     h = hm / n_mt;
     mt = hm % n_mt;
     m0 = (rope_tile_m0 >= 0 && mt == n_mt - 1) ? rope_tile_m0 : mt * 128;
     n0 = nt * nr;
+    kb0 = s * nk / splits;
+    kb1 = (s + 1) * nk / splits;
+    tile = mt * n_nt + nt;
   }
 };
+
+MLA_DEVICE bool warp_leader(int sp, int lane) { return sp == 2 && lane == 0; }
 
 // Physical cache row of activation row `row` (token t of sequence b) for the fused append,
 // or -1 when its position or page is out of range (the caller sets the error word).
@@ -190,32 +199,79 @@ MLA_DEVICE void write_rope_slots(const WGemmParams& p, int tid, int nthreads) {
 // values, exactly as mla_cache_append) and rounded to bf16 with ties to even.
 // All four warps pass both named barriers whatever their accumulator wait returned (`ok`);
 // a failed wait leaves the CTA's abort flag set, and then no warp writes the tile.
+// With the K split in several CTAs (p.splits > 1) each split first adds its fp32 sums into
+// p.acc; the last split of the tile to finish reads the totals back (clearing them for the
+// next call) and writes the rows. `last` is a shared-memory flag of the CTA.
 template <int NR>
 MLA_DEVICE void append_epilogue(const WGemmParams& p, const WgItem& w, int buf, uint32_t tmem,
                                 int sp, int lane, uint16_t* stage, uint64_t* acc_empty, bool ok,
-                                volatile int* abort_flag) {
+                                volatile int* abort_flag, volatile int* last) {
   const int m_loc = sp * 32 + lane;
   const int nrows = min(NR, p.rows - w.n0);
+  const int D = p.lat_r + p.groups * p.rope_dim;
+  const int f = w.m0 + m_loc;                     // feature of this thread's TMEM lane
+  // the latent tiles own features [m0, r), the rotary tile [r, D)
+  const bool own = w.m0 < p.lat_r ? f < p.lat_r : f < D;
+  const bool split = p.splits > 1;
   if (ok) {
 #pragma unroll 1
     for (int c0 = 0; c0 < NR; c0 += 16) {
       float v[16];
       tmem_ld16(tmem + (uint32_t(sp * 32) << 16) + uint32_t(buf * NR + c0), v);
       tmem_wait_ld();
+      if (split) {
+        if (own) {
 #pragma unroll
-      for (int j = 0; j < 16; ++j) stage[(c0 + j) * 128 + m_loc] = f32_to_bf16_rne(v[j]);
+          for (int j = 0; j < 16; ++j)
+            if (c0 + j < nrows) atomicAdd(p.acc + int64_t(w.n0 + c0 + j) * D + f, v[j]);
+        }
+      } else {
+#pragma unroll
+        for (int j = 0; j < 16; ++j) stage[(c0 + j) * 128 + m_loc] = f32_to_bf16_rne(v[j]);
+      }
     }
+    if (split) __threadfence();
   }
   tc_fence_before();
   __syncwarp();
   if (lane == 0) mbar_arrive(acc_empty);
-  named_bar_sync(1, kWgEpiThreads);               // the staging tile is complete
+  named_bar_sync(1, kWgEpiThreads);
+  if (split) {
+    if (warp_leader(sp, lane) && *abort_flag == 0) {
+      const int old = atomicAdd(p.tile_done + w.tile, 1);
+      *last = (old == p.splits - 1) ? 1 : 0;
+    }
+    named_bar_sync(1, kWgEpiThreads);
+    if (*last != 0 && *abort_flag == 0) {
+      // read the totals back (4 features per thread and step, several rows' loads in
+      // flight), clear them for the next call and round them into the staging tile
+      __threadfence();
+      const int f_end = w.m0 < p.lat_r ? min(w.m0 + 128, p.lat_r) : D;   // multiple of 4
+#pragma unroll 4
+      for (int idx = m_loc; idx < nrows * 32; idx += kWgEpiThreads) {
+        const int n = idx >> 5, c = 4 * (idx & 31);
+        float4 v = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+        if (w.m0 + c < f_end) {
+          float4* a = reinterpret_cast<float4*>(p.acc + int64_t(w.n0 + n) * D + w.m0 + c);
+          v = __ldcg(a);
+          __stcg(a, make_float4(0.0f, 0.0f, 0.0f, 0.0f));
+        }
+        *reinterpret_cast<uint2*>(stage + n * 128 + c) =
+            make_uint2(cvt_bf16x2(v.x, v.y), cvt_bf16x2(v.z, v.w));
+      }
+      if (warp_leader(sp, lane)) p.tile_done[w.tile] = 0;
+    }
+    named_bar_sync(1, kWgEpiThreads);             // the staging tile is complete
+    const bool write = *last != 0;
+    named_bar_sync(1, kWgEpiThreads);             // every thread has read `last`
+    if (warp_leader(sp, lane)) *last = 0;
+    if (!write) return;
+  }
   if (*abort_flag != 0) {
     named_bar_sync(1, kWgEpiThreads);
     return;
   }
   const int tid = m_loc;                          // 0..127
-  const int D = p.lat_r + p.groups * p.rope_dim;
   if (w.m0 < p.lat_r) {
     // latent tile: features [m0, min(m0 + 128, r)) of every token, 8 per 16-byte chunk
     const int chunks = (min(128, p.lat_r - w.m0)) / 8;
@@ -273,6 +329,7 @@ __global__ void __launch_bounds__(kWgThreads, 1) wgemm_kernel(const __grid_const
   uint64_t* acc_empty = acc_full + 2;                                 // [2] accumulator drained
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(acc_empty + 2);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  volatile int* last_flag = abort_flag + 1;
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -280,8 +337,9 @@ __global__ void __launch_bounds__(kWgThreads, 1) wgemm_kernel(const __grid_const
   const int rope_m0 = (append && p.groups * p.rope_dim > 0) ? p.lat_r : -1;
   const int n_mt = append ? p.lat_tiles + (rope_m0 >= 0 ? 1 : 0) : (p.M + 127) / 128;
   const int n_nt = (p.rows + NR - 1) / NR;
-  const int items = n_mt * p.heads * n_nt;
   const int nk = (p.K + 63) / 64;
+  const int splits = p.splits > 1 ? p.splits : 1;
+  const int items = n_mt * p.heads * splits * n_nt;
   constexpr uint32_t kCols = 2 * NR < 32 ? 32 : 2 * NR;   // two accumulators of NR columns
   const WaitCtx wc{abort_flag, p.dev_error};
 
@@ -295,6 +353,7 @@ __global__ void __launch_bounds__(kWgThreads, 1) wgemm_kernel(const __grid_const
       mbar_init(&acc_empty[i], 4);                    // the four epilogue warps
     }
     *abort_flag = 0;
+    *last_flag = 0;
     fence_mbar_init();
   }
   if (warp == 1) {
@@ -311,12 +370,30 @@ __global__ void __launch_bounds__(kWgThreads, 1) wgemm_kernel(const __grid_const
     if (elect_one()) {
       prefetch_tensormap(&p.tm_w);
       prefetch_tensormap(&p.tm_x);
+      // The weights are no kernel's output here: warm L2 with this CTA's weight tiles while
+      // the previous kernel may still run (an L2 prefetch is coherent with any writer).
+      for (int it = blockIdx.x; it < items; it += gridDim.x) {
+        const WgItem w(it, n_mt, n_nt, NR, rope_m0, splits, nk);
+        for (int kb = w.kb0; kb < w.kb1; ++kb) {
+          if (p.a_mn) {
+            tma_prefetch_l2_3d(&p.tm_w, w.m0, kb * 64, w.h);
+            tma_prefetch_l2_3d(&p.tm_w, w.m0 + 64, kb * 64, w.h);
+          } else {
+            tma_prefetch_l2_3d(&p.tm_w, kb * 64, w.m0, w.h);
+          }
+        }
+      }
+    }
+    __syncwarp();
+    grid_dep_wait();
+    grid_dep_launch();
+    if (elect_one()) {
       SlotRing ring(S);
       int g = 0;   // stages issued
       bool ok = true;
       for (int it = blockIdx.x; ok && it < items; it += gridDim.x) {
-        const WgItem w(it, n_mt, n_nt, NR, rope_m0);
-        for (int kb = 0; kb < nk; ++kb, ++g, ring.next()) {
+        const WgItem w(it, n_mt, n_nt, NR, rope_m0, splits, nk);
+        for (int kb = w.kb0; kb < w.kb1; ++kb, ++g, ring.next()) {
           if (g >= S && !mbar_wait(&empty[ring.slot], (ring.round - 1) & 1, wc)) {
             ok = false;
             break;
@@ -340,18 +417,21 @@ __global__ void __launch_bounds__(kWgThreads, 1) wgemm_kernel(const __grid_const
     __syncwarp();
   } else if (warp == 1) {
     // ============================ UMMA issuer, two accumulators ==========================
+    grid_dep_wait();
+    grid_dep_launch();
     if (elect_one()) {
       const uint32_t idesc = make_idesc_bf16(128, NR, p.a_mn, 0);
       SlotRing ring(S);
       bool ok = true;
       int li = 0;   // items of this CTA so far
       for (int it = blockIdx.x; ok && it < items; it += gridDim.x, ++li) {
+        const WgItem w(it, n_mt, n_nt, NR, rope_m0, splits, nk);
         const int buf = li & 1;
         // the epilogue has drained this accumulator (item li - 2)
         if (li >= 2 && !mbar_wait(&acc_empty[buf], ((li >> 1) - 1) & 1, wc)) break;
         tc_fence_after();
         const uint32_t d = tmem + uint32_t(buf * NR);
-        for (int kb = 0; kb < nk; ++kb, ring.next()) {
+        for (int kb = w.kb0; kb < w.kb1; ++kb, ring.next()) {
           if (!mbar_wait(&full[ring.slot], ring.round & 1, wc)) {
             ok = false;
             break;
@@ -365,7 +445,7 @@ __global__ void __launch_bounds__(kWgThreads, 1) wgemm_kernel(const __grid_const
             const uint64_t ad = p.a_mn ? make_sdesc(a + kk * 2048, 8192, 1024, kSw128)
                                        : make_sdesc(a + kk * 32, 16, 1024, kSw128);
             const uint64_t bd = make_sdesc(b + kk * 32, 16, 1024, kSw128);
-            umma_bf16(d, ad, bd, idesc, (kb | kk) != 0);
+            umma_bf16(d, ad, bd, idesc, (kb != w.kb0 || kk != 0) ? 1u : 0u);
           }
           umma_commit(&empty[ring.slot]);
         }
@@ -375,20 +455,22 @@ __global__ void __launch_bounds__(kWgThreads, 1) wgemm_kernel(const __grid_const
     __syncwarp();
   } else {
     // ============== epilogue warps 2-5: warp w reaches TMEM lanes 32 (w % 4) .. ==========
+    grid_dep_wait();
+    grid_dep_launch();
     const int sp = warp & 3;
     if (p.q_pe != nullptr && p.rope_dim > 0)
       write_rope_slots(p, int(blockIdx.x) * kWgEpiThreads + int(threadIdx.x) - 64,
                        int(gridDim.x) * kWgEpiThreads);
     int li = 0;
     for (int it = blockIdx.x; it < items; it += gridDim.x, ++li) {
-      const WgItem w(it, n_mt, n_nt, NR, rope_m0);
+      const WgItem w(it, n_mt, n_nt, NR, rope_m0, splits, nk);
       const int buf = li & 1;
       const bool ok = __all_sync(0xffffffffu, mbar_wait(&acc_full[buf], (li >> 1) & 1, wc));
       tc_fence_after();
       if (append) {
         append_epilogue<NR>(p, w, buf, tmem, sp, lane,
                             reinterpret_cast<uint16_t*>(base + Lay::kBars + 256), &acc_empty[buf],
-                            ok, abort_flag);
+                            ok, abort_flag, last_flag);
         continue;
       }
       if (ok) {
@@ -435,10 +517,9 @@ static cudaError_t launch_wgemm_nr(const WGemmParams& p, int max_ctas, cudaStrea
   if (e != cudaSuccess) return e;
   const int64_t n_mt = append ? p.lat_tiles + (p.groups * p.rope_dim > 0 ? 1 : 0)
                               : (p.M + 127) / 128;
-  const int64_t items = n_mt * p.heads * ((p.rows + NR - 1) / NR);
+  const int64_t items = n_mt * p.heads * (p.splits > 1 ? p.splits : 1) * ((p.rows + NR - 1) / NR);
   const int grid = int(items < max_ctas ? items : max_ctas);
-  wgemm_kernel<NR><<<grid, kWgThreads, smem, stream>>>(p);
-  return cudaGetLastError();
+  return launch_pdl(wgemm_kernel<NR>, dim3(grid), dim3(kWgThreads), size_t(smem), stream, 1, p);
 }
 
 cudaError_t launch_wgemm(const WGemmParams& p, int nr, int max_ctas, cudaStream_t stream) {

@@ -117,17 +117,24 @@ mla_status mla_cache_append(const mla_dims* dims, const void* c_kv, const void* 
  *   rope_cos/sin, block_table, start_pos, cache, num_pages, dev_error: as mla_cache_append
  *   kv_out      bf16 [B, n_new, D] or NULL    if given, also receives the GEMM's bf16
  *                                             output [c_kv ; k_r] before the rotation
+ *   workspace   >= mla_down_kv_workspace_size(dims, B, n_new) bytes, 256-byte aligned,
+ *               zeroed once after allocation; each call leaves it zero again (it holds the
+ *               fp32 sums of the model width split across CTAs and their counters), so it
+ *               serves later calls on the same stream, not concurrent ones
  *
  * For each token: [c_kv ; k_r] = bf16_rne(fp32 sum over hidden of w_dkv * x), then exactly
- * what mla_cache_append writes for that c_kv and k_r (the same cache bytes). Requires
+ * what mla_cache_append writes for that c_kv and k_r (the same cache bytes). The sum over
+ * the model width is split across CTAs and added with fp32 atomics, so its last bit may
+ * differ from call to call. Requires
  * G*d_r <= 128 (MLA_ERR_UNSUPPORTED otherwise). Bounds faults as mla_cache_append.
  */
+size_t mla_down_kv_workspace_size(const mla_dims* dims, int32_t batch, int32_t n_new);
 mla_status mla_down_kv_append(const mla_dims* dims, const void* hidden, int32_t hidden_dim,
                               const void* w_dkv, const float* rope_cos, const float* rope_sin,
                               const int32_t* block_table, int32_t max_pages_per_seq,
                               const int32_t* start_pos, int32_t batch, int32_t n_new,
                               void* cache, int64_t num_pages, int32_t* dev_error, void* kv_out,
-                              void* stream);
+                              void* workspace, size_t workspace_bytes, void* stream);
 
 /*
  * mla_absorb_q - fold W_UK into the query and rotate its RoPE part.
@@ -149,6 +156,34 @@ mla_status mla_absorb_q(const mla_dims* dims, const void* q_nope, const void* q_
                         const float* rope_cos, const float* rope_sin, const void* w_uk,
                         int64_t w_uk_head_stride, int32_t batch, int32_t q_len, void* q_ext,
                         void* stream);
+
+/*
+ * mla_out_proj - einsums (5) and (6) of the DeepSeek-V2 page's "Matrix absorption" section
+ * in one kernel: the value up-projection o = einsum('bhqc,hdc->bhqd', o_, W_UV) (+ up_v bias)
+ * followed by the output projection u = einsum('hdD,bhqd->bqD', W_o, o) (+ bias), the
+ * latter being the page's o_proj of size [num_heads * v_head_dim, hidden_size].
+ *
+ *   o_latent  bf16 [rows, H, r]             rows = B*q (mla_decode_attn's o_latent)
+ *   w_uv, w_uv_head_stride, bias_v          as mla_out_up (bias_v [H, d_v] or NULL)
+ *   w_o       bf16 [hidden, H*d_v]          row k holds W_o[h, d, k] at column h*d_v + d
+ *                                           (a torch.nn.Linear(H*d_v, hidden) weight)
+ *   bias_o    bf16 [hidden] or NULL
+ *   workspace >= mla_out_proj_workspace_size(dims, hidden, rows) bytes, 256-byte aligned,
+ *             zeroed once after allocation; the call leaves its counters zero again, so
+ *             the workspace serves later calls on the same stream (not concurrent ones).
+ *             Its first int32 is a device error word (MLA_DEVERR_TIMEOUT if a wait ran out).
+ *   o         bf16 [rows, H, d_v] output (the up-projected values, also the input of (6))
+ *   u         bf16 [rows, hidden] output (fp32 accumulate; stage (6) adds its K splits in
+ *             a fixed order, so the result is deterministic)
+ * Requires d_v % 64 == 0 and hidden % 8 == 0 (MLA_ERR_UNSUPPORTED / MLA_ERR_INVALID_ARG).
+ * The kernel is a cooperative launch (all its CTAs resident at once, one per SM); it fails
+ * with MLA_ERR_CUDA if the device cannot hold them.
+ */
+size_t mla_out_proj_workspace_size(const mla_dims* dims, int32_t hidden, int32_t rows);
+mla_status mla_out_proj(const mla_dims* dims, const void* o_latent, const void* w_uv,
+                        int64_t w_uv_head_stride, const void* bias_v, const void* w_o,
+                        const void* bias_o, int32_t hidden, int32_t rows, void* workspace,
+                        size_t workspace_bytes, void* o, void* u, void* stream);
 
 /*
  * Bytes of workspace mla_decode_attn needs for this problem (0 on invalid input).

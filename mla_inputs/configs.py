@@ -15,6 +15,8 @@ Shapes come from the pages' models:
   KV groups, rank 512, 8 RoPE dims per KV group, ragged context lengths.
 * hybrid_*: the MLA layers of the zebra hybrid model (trdm.cn page):
   16 heads, kv_lora_rank 256, context extended to 1,048,576 tokens.
+* prefill_*: one sequence's prefill chunk of q = 64, 256 or 1024 tokens attending
+  causally over the cache (DeepSeek-V2 shape over 4,096 tokens; hybrid shape over 16,384).
 * nanowhale_kv_shared: the single-latent K = V layer of nanowhale-100m (cnnetsun.cn
   page): 8 heads, one 512-d key/value vector per token with RoPE on its last 64 dims.
 
@@ -118,9 +120,23 @@ NANOWHALE_KV_SHARED = _cfg(name="nanowhale_kv_shared", index=5, batch=128, q_len
                            rope_dim=64, v_head_dim=512, context=2048,
                            softmax_scale=1.0 / math.sqrt(512.0), hidden_size=320)
 
+# Prefill chunks: q new tokens attend causally over the latent cache they were appended to
+# (the DeepSeek-V2 page's attention, with the query block of the hybrid workload's q = 4
+# widened to a prefill chunk). One sequence, the DeepSeek-V2 and hybrid layer shapes.
+PREFILL = {}
+for _q in (64, 256, 1024):
+    PREFILL[f"prefill_deepseek_v2_q{_q}"] = _cfg(
+        name=f"prefill_deepseek_v2_q{_q}", index=6, batch=1, q_len=_q, num_heads=128,
+        num_kv_groups=1, kv_lora_rank=512, qk_nope_dim=128, rope_dim=64, v_head_dim=128,
+        context=4096, softmax_scale=1.0 / math.sqrt(192.0), hidden_size=5120)
+    PREFILL[f"prefill_hybrid_q{_q}"] = _cfg(
+        name=f"prefill_hybrid_q{_q}", index=7, batch=1, q_len=_q, num_heads=16,
+        num_kv_groups=1, kv_lora_rank=256, qk_nope_dim=128, rope_dim=64, v_head_dim=128,
+        context=16384, softmax_scale=1.0 / math.sqrt(192.0), hidden_size=2048)
+
 CONFIGS = {c.name: c for c in (TINY, QWEN25_7B, DEEPSEEK_V2, QWEN3_30B_A3B, HYBRID_1M_Q1,
                                HYBRID_1M_Q4, HYBRID_256K_Q1, HYBRID_256K_Q4,
-                               NANOWHALE_KV_SHARED)}
+                               NANOWHALE_KV_SHARED, *PREFILL.values())}
 
 
 def shrink(cfg: MLAConfig, batch: Optional[int] = None, context: Optional[int] = None,

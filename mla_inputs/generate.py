@@ -157,3 +157,15 @@ def make_down_kv_inputs(cfg: MLAConfig, n_new: int) -> Tuple[torch.Tensor, torch
     hidden = torch.randn(cfg.batch, n_new, cfg.hidden_size, generator=gen).to(torch.bfloat16)
     w_dkv = _randn(gen, (cfg.row_width, cfg.hidden_size), cfg.hidden_size)
     return hidden, w_dkv
+
+
+def make_o_proj_inputs(cfg: MLAConfig, with_bias: bool = False):
+    """The output projection for ``cfg``: w_o [hidden, H * d_v] ~ N(0, 1) / sqrt(H * d_v) (row k
+    holds W_o[h, d, k] at column h * d_v + d) and, if asked, bias [hidden] ~ N(0, 1) / sqrt(hidden),
+    bf16, from their own seeded generator."""
+    gen = torch.Generator("cpu")
+    gen.manual_seed(cfg.seed * 37 + 23)
+    K = cfg.num_heads * cfg.v_head_dim
+    w_o = _randn(gen, (cfg.hidden_size, K), K)
+    bias = _randn(gen, (cfg.hidden_size,), cfg.hidden_size) if with_bias else None
+    return w_o, bias

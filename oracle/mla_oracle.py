@@ -18,6 +18,8 @@ What it computes, and where the pages define it
   own, for checking the two projection steps separately.
 * ``mla_decode_absorbed``: the same attention in the absorbed order (a second CPU
   baseline; equal to the unabsorbed definition by associativity).
+* ``o_proj_reference``: einsum (6), the output projection of the heads' values to the
+  model width (W_o of shape [H, d_v, hidden]).
 * ``down_kv_reference``: the hidden -> [c_kv ; k_r] projection whose output the cache
   stores (down_kv / k_r_proj of the MLAfication page, kv_a_proj_with_mqa of the
   DeepSeek-V2 page).
@@ -325,3 +327,13 @@ def down_kv_reference(hidden, w_dkv, kv_lora_rank: int, num_groups: int, rope_di
     c_kv = out[..., :kv_lora_rank]
     k_r = out[..., kv_lora_rank:].reshape(out.shape[:-1] + (num_groups, rope_dim))
     return c_kv, k_r
+
+
+def o_proj_reference(o, w_o, bias=None):
+    """The output projection, einsum (6) of the "Matrix absorption" section:
+    u = einsum('hdD,bhqd->bqD', W_o, o), i.e. u[.., D] = sum over heads h and value dims d of
+    W_o[h, d, D] o[.., h, d] (+ bias[D]). o [..., H, d_v], w_o [H, d_v, hidden] -> [..., hidden]."""
+    u = np.einsum("...hd,hdk->...k", as_f64(o), as_f64(w_o))
+    if bias is not None:
+        u = u + as_f64(bias)
+    return u

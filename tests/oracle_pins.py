@@ -466,8 +466,33 @@ def pin_down_kv_bruteforce(O):
                 assert abs(got - acc) <= 1e-12 * max(1.0, abs(acc)), (b, t, d)
 
 
+def pin_o_proj_original_order(O):
+    """Einsum (6) after (4)-(5) equals einsum (3) of the original order, computed from the
+    up-projected values and the attention weights with literal loops: u[i, D] = sum over h, d
+    of W_o[h, d, D] * sum_l p[i, h, l] * V_h[l, d]."""
+    P = _problem(71, nq=2, H=3, G=1, r=4, dn=2, dr=2, dv=3, L=5, bias=False)
+    rng = np.random.default_rng(72)
+    hid = 4
+    w_o = rng.standard_normal((3, 3, hid))
+    b_o = rng.standard_normal(hid)
+    got = O.mla_decode_reference(want_p=True, **P)
+    u = O.o_proj_reference(O.out_up_reference(got["o_latent"], P["w_uv"]), w_o, b_o)
+    p = got["p"]
+    for i in range(2):
+        for D in range(hid):
+            acc = b_o[D]
+            for h in range(3):
+                for d in range(3):
+                    v = 0.0
+                    for l in range(5):
+                        vl = sum(P["w_uv"][h][d][c] * P["c_kv"][l][c] for c in range(4))
+                        v += p[i][h][l] * vl
+                    acc += w_o[h][d][D] * v
+            assert abs(u[i, D] - acc) <= 1e-11 * max(1.0, abs(acc)), (i, D)
+
+
 ALL_PINS = [pin_absorb_single_token, pin_out_up_associativity, pin_bruteforce, pin_associativity, pin_sdpa_identity_weights, pin_zero_query_uniform,
             pin_single_token, pin_rows_sum_to_one, pin_causal_prefix, pin_rope_complex,
             pin_rope_norm_and_relative, pin_bf16_rounding, pin_rotate_fp32, pin_append_slots,
             pin_kv_shared_sdpa, pin_kv_shared_single_token, pin_absorbed_baseline,
-            pin_down_kv_bruteforce]
+            pin_down_kv_bruteforce, pin_o_proj_original_order]

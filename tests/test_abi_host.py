@@ -204,9 +204,13 @@ def test_down_kv_append_validation(mla_lib):
     L = mla.lib()
     d = _dims()
 
-    def call(dd=d, hidden=FAKE, hid=5120, w=FAKE, batch=2, n=1, cache=FAKE, kv_out=None):
+    def call(dd=d, hidden=FAKE, hid=5120, w=FAKE, batch=2, n=1, cache=FAKE, kv_out=None,
+             ws=P(0x10000), wsb=1 << 20):
         return L.mla_down_kv_append(ctypes.byref(dd), hidden, hid, w, FAKE, FAKE, FAKE, 4, FAKE,
-                                    batch, n, cache, 100, None, kv_out, None)
+                                    batch, n, cache, 100, None, kv_out, ws, wsb, None)
+    assert call(ws=None) == mla.MLA_ERR_WORKSPACE
+    assert call(wsb=16) == mla.MLA_ERR_WORKSPACE
+    assert mla.mla_down_kv_workspace_size(d, 64, 1) >= 64 * 576 * 4
     assert call(hid=100) == mla.MLA_ERR_INVALID_ARG              # not a multiple of 8
     assert call(hidden=None) == mla.MLA_ERR_INVALID_ARG
     assert call(w=P(0x10008)) == mla.MLA_ERR_INVALID_ARG          # misaligned weight
@@ -214,3 +218,21 @@ def test_down_kv_append_validation(mla_lib):
     assert call(dd=_dims(num_kv_groups=4, num_heads=128, rope_dim=64)) == mla.MLA_ERR_UNSUPPORTED
     assert call(batch=0) == mla.MLA_OK
     assert call(n=0) == mla.MLA_OK
+
+
+def test_out_proj_validation(mla_lib):
+    L = mla.lib()
+    d = _dims()
+    assert mla.mla_out_proj_workspace_size(d, 5120, 64) > 0
+    assert mla.mla_out_proj_workspace_size(d, 5121, 64) == 0             # hidden % 8
+    assert mla.mla_out_proj_workspace_size(_dims(v_head_dim=96), 5120, 64) == 0   # d_v % 64
+
+    def call(dd=d, ol=FAKE, wo=FAKE, hidden=5120, rows=4, ws=P(0x10000), wsb=1 << 30, u=FAKE):
+        return L.mla_out_proj(ctypes.byref(dd), ol, FAKE, 128 * 512, None, wo, None, hidden, rows,
+                              ws, wsb, FAKE, u, None)
+    assert call(ol=None) == mla.MLA_ERR_INVALID_ARG
+    assert call(u=P(0x10002)) == mla.MLA_ERR_INVALID_ARG
+    assert call(ws=None) == mla.MLA_ERR_WORKSPACE
+    assert call(wsb=64) == mla.MLA_ERR_WORKSPACE
+    assert call(dd=_dims(v_head_dim=96)) == mla.MLA_ERR_UNSUPPORTED
+    assert call(rows=0) == mla.MLA_OK

@@ -50,6 +50,8 @@ MUTATIONS = {
     "down_kv_transposed_weight": ('np.einsum("...k,dk->...d", as_f64(hidden), as_f64(w_dkv))',
                                   'np.einsum("...k,dk->...d", as_f64(hidden), as_f64(w_dkv)[::-1])'),
     "down_kv_split_off_by_one": ("k_r = out[..., kv_lora_rank:]", "k_r = out[..., kv_lora_rank - 1:-1]"),
+    "o_proj_transposed_head_dims": ('np.einsum("...hd,hdk->...k", as_f64(o), as_f64(w_o))',
+                                    'np.einsum("...hd,hdk->...k", as_f64(o)[..., ::-1], as_f64(w_o))'),
 }
 
 
