@@ -402,7 +402,8 @@ mla_status mla_down_kv_append(const mla_dims* dims, const void* hidden, int32_t 
   const int n_mt = p.lat_tiles + (R > 0 ? 1 : 0);
   const int64_t n_nt = (rows + nr - 1) / nr;
   const int nk = (hidden_dim + 63) / 64;
-  p.splits = int(std::max<int64_t>(1, std::min<int64_t>(nk, num_sms() / (n_mt * n_nt))));
+  // (at least 8 K blocks of 64 per split: fewer, longer items than one per SM)
+  p.splits = int(std::max<int64_t>(1, std::min<int64_t>(nk / 8, num_sms() / (n_mt * n_nt))));
   const int64_t tiles = int64_t(n_mt) * n_nt;
   p.tile_done = static_cast<int32_t*>(workspace);
   p.acc = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) +

@@ -7,8 +7,8 @@
 // activation rows on N (like wgemm.cu). Stage B reads stage A's output, so the kernel is
 // persistent and co-resident (a cooperative launch): every CTA takes its stage-A items
 // first; a stage-B item waits, in its TMA producer only, for per-head completion counters
-// that the stage-A epilogues release, and streams its W_o tiles as soon as those heads are
-// done. Stage B's K is cut into S splits so that its items fill the GPU in about one wave
+// that the stage-A epilogues release (polled with one round of relaxed loads, then one
+// acquire fence), and streams its W_o tiles as soon as those heads are done. Stage B's K is cut into S splits so that its items fill the GPU in about one wave
 // (W_o is the bulk of the bytes: 168 MB at the DeepSeek-V2 shape, o only 2 MB and L2
 // resident); each split stores an fp32 partial, and the last split of a tile to finish (a
 // counter per tile) adds the S partials in a fixed order and writes u in bf16, so the
@@ -43,11 +43,12 @@ MLA_DEVICE uint8_t* op_align1024(uint8_t* p) {
   return reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(p) + 1023) & ~uintptr_t(1023));
 }
 
-MLA_DEVICE int ld_acquire(const int32_t* p) {
+MLA_DEVICE int ld_relaxed(const int32_t* p) {
   int v;
-  asm volatile("ld.acquire.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+  asm volatile("ld.relaxed.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
   return v;
 }
+MLA_DEVICE void fence_acq_rel_gpu() { asm volatile("fence.acq_rel.gpu;" ::: "memory"); }
 MLA_DEVICE void fence_proxy_async_global() {
   asm volatile("fence.proxy.async.global;" ::: "memory");
 }
@@ -164,20 +165,25 @@ __global__ void __launch_bounds__(kOpThreads, 1) oproj_kernel(const __grid_const
           }
           tma_load_2d(a, &p.tm_wo, w.k0 + kb * 64, w.m0, &full[ring.slot]);
           if (need) {
-            // o of this split's heads is written by stage-A epilogues of any CTA
+            // o of this split's heads is written by stage-A epilogues of any CTA. Each pass
+            // reads every head's counter with independent relaxed loads (one L2 round trip
+            // for all of them, not one per head); once all are complete, one acquire fence
+            // orders the o loads below after the epilogues' release.
             const int h0 = w.s * p.H / p.splits, h1 = (w.s + 1) * p.H / p.splits;
             const uint64_t t0 = globaltimer_ns();
-            for (int h = h0; h < h1 && ok; ++h) {
-              while (ld_acquire(p.head_done + h) < headA_target) {
-                __nanosleep(256);                   // keep the counters' L2 lines quiet
-                if (*abort_flag || globaltimer_ns() - t0 > kWaitLimitNs) {
-                  *abort_flag = 1;
-                  if (p.dev_error) atomicOr(p.dev_error, MLA_DEVERR_TIMEOUT);
-                  ok = false;
-                  break;
-                }
+            while (true) {
+              bool all = true;
+              for (int h = h0; h < h1; ++h) all &= ld_relaxed(p.head_done + h) >= headA_target;
+              if (all) break;
+              __nanosleep(128);
+              if (*abort_flag || globaltimer_ns() - t0 > kWaitLimitNs) {
+                *abort_flag = 1;
+                if (p.dev_error) atomicOr(p.dev_error, MLA_DEVERR_TIMEOUT);
+                ok = false;
+                break;
               }
             }
+            fence_acq_rel_gpu();
             fence_proxy_async_global();
             need = false;
           }

@@ -272,6 +272,14 @@ MLA_DEVICE void append_epilogue(const WGemmParams& p, const WgItem& w, int buf, 
     return;
   }
   const int tid = m_loc;                          // 0..127
+  // the cache row of every token of the tile, looked up once (two dependent loads each)
+  int64_t* slot_s = reinterpret_cast<int64_t*>(stage + NR * 128);
+  if (tid < nrows) {
+    const int64_t slot = append_slot(p, w.n0 + tid);
+    if (slot < 0 && p.dev_error) atomicOr(p.dev_error, MLA_DEVERR_BOUNDS);
+    slot_s[tid] = slot;
+  }
+  named_bar_sync(1, kWgEpiThreads);
   if (w.m0 < p.lat_r) {
     // latent tile: features [m0, min(m0 + 128, r)) of every token, 8 per 16-byte chunk
     const int chunks = (min(128, p.lat_r - w.m0)) / 8;
@@ -280,12 +288,8 @@ MLA_DEVICE void append_epilogue(const WGemmParams& p, const WgItem& w, int buf, 
       const int row = w.n0 + n;
       const uint4 v = *reinterpret_cast<const uint4*>(stage + n * 128 + c * 8);
       if (p.kv_out) *reinterpret_cast<uint4*>(p.kv_out + int64_t(row) * D + w.m0 + c * 8) = v;
-      const int64_t slot = append_slot(p, row);
-      if (slot < 0) {
-        if (c == 0 && p.dev_error) atomicOr(p.dev_error, MLA_DEVERR_BOUNDS);
-        continue;
-      }
-      *reinterpret_cast<uint4*>(p.cache + slot * D + w.m0 + c * 8) = v;
+      const int64_t slot = slot_s[n];
+      if (slot >= 0) *reinterpret_cast<uint4*>(p.cache + slot * D + w.m0 + c * 8) = v;
     }
   } else {
     // rotary tile: features [r, D), pair j of group g = (x_j, x_{j + d_r/2})
@@ -301,11 +305,8 @@ MLA_DEVICE void append_epilogue(const WGemmParams& p, const WgItem& w, int buf, 
         p.kv_out[int64_t(row) * D + p.lat_r + f] = b0;
         p.kv_out[int64_t(row) * D + p.lat_r + f + half] = b1;
       }
-      const int64_t slot = append_slot(p, row);
-      if (slot < 0) {
-        if (pi == 0 && p.dev_error) atomicOr(p.dev_error, MLA_DEVERR_BOUNDS);
-        continue;
-      }
+      const int64_t slot = slot_s[n];
+      if (slot < 0) continue;
       const float x0 = bf16_bits_to_f32(b0), x1 = bf16_bits_to_f32(b1);
       const int64_t ci = (int64_t(row) * p.groups + g) * half + j;
       const float cj = p.rope_cos[ci], sj = p.rope_sin[ci];
@@ -510,8 +511,9 @@ __global__ void __launch_bounds__(kWgThreads, 1) wgemm_kernel(const __grid_const
 template <int NR>
 static cudaError_t launch_wgemm_nr(const WGemmParams& p, int max_ctas, cudaStream_t stream) {
   const bool append = p.cache != nullptr;
-  // the fused append stages one [NR][128] bf16 tile after the barriers
-  const int smem = WgLayout<NR>::kTotal + (append ? NR * 128 * 2 : 0);
+  // the fused append stages one [NR][128] bf16 tile and NR cache-row indices after the
+  // barriers
+  const int smem = WgLayout<NR>::kTotal + (append ? NR * 128 * 2 + NR * 8 : 0);
   cudaError_t e = cudaFuncSetAttribute(wgemm_kernel<NR>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
