@@ -269,6 +269,7 @@ mla_status mla_absorb_q(const mla_dims* dims, const void* q_nope, const void* q_
   p.rows = int32_t(rows);
   p.heads = H;
   p.a_mn = 1;
+  p.vec_out = (D % 8 == 0 && r % 8 == 0) ? 1 : 0;   // q_ext is 16-byte aligned (checked above)
   p.splits = 1;
   p.q_pe = dims->rope_dim > 0 ? static_cast<const uint16_t*>(q_pe) : nullptr;
   p.rope_cos = rope_cos;
@@ -318,6 +319,7 @@ mla_status mla_out_up(const mla_dims* dims, const void* o_latent, const void* w_
   p.rows = rows;
   p.heads = H;
   p.a_mn = 0;
+  p.vec_out = dv % 8 == 0 ? 1 : 0;                  // o is 16-byte aligned (checked above)
   p.splits = 1;
   p.q_pe = nullptr;
   return launch_wgemm(p, nr, num_sms(), as_stream(stream)) == cudaSuccess ? MLA_OK : MLA_ERR_CUDA;

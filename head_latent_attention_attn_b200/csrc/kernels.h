@@ -78,6 +78,7 @@ struct WGemmParams {
   int32_t* dev_error;
   int32_t M, K, rows, heads;
   int32_t a_mn;              // 1: weight stored [K][M] (W_UK), 0: stored [M][K] (W_UV)
+  int32_t vec_out;           // 1: out, both strides and M are multiples of 8 elements
   // rotary part of q_ext (mla_absorb_q only; q_pe == nullptr otherwise)
   const uint16_t* q_pe;      // [rows, H, d_r]
   const float* rope_cos;     // [rows, G, d_r/2]

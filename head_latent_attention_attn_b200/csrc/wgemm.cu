@@ -318,6 +318,62 @@ MLA_DEVICE void append_epilogue(const WGemmParams& p, const WgItem& w, int buf, 
   named_bar_sync(1, kWgEpiThreads);               // the staging tile may be reused
 }
 
+// Epilogue of absorb / out_up for one item, run by the four epilogue warps: the
+// accumulator (output feature m0 + lane of each TMEM lane, one column per activation row)
+// plus the bias is rounded to bf16 into a [NR rows][128 features] staging tile, the
+// accumulator is handed back, and the tile is written out row by row, so that consecutive
+// threads write consecutive 16-byte pieces of an output row (the rows of one item are
+// out_row_stride apart). All four warps pass both named barriers whatever their
+// accumulator wait returned (`ok`); a failed wait leaves the CTA's abort flag set, and
+// then no warp writes the tile.
+template <int NR>
+MLA_DEVICE void plain_epilogue(const WGemmParams& p, const WgItem& w, int buf, uint32_t tmem,
+                               int sp, int lane, uint16_t* stage, uint64_t* acc_empty, bool ok,
+                               volatile int* abort_flag) {
+  const int m_loc = sp * 32 + lane;
+  const int m = w.m0 + m_loc;                  // output feature of this thread's TMEM lane
+  const int nrows = min(NR, p.rows - w.n0);
+  if (ok) {
+    const float bias = (p.bias != nullptr && m < p.M)
+                           ? bf16_bits_to_f32(p.bias[int64_t(w.h) * p.M + m]) : 0.0f;
+    // Not unrolled: the code runs once per item with a cold instruction cache (the decode
+    // kernel runs between these launches).
+#pragma unroll 1
+    for (int c0 = 0; c0 < NR; c0 += 16) {
+      float v[16];
+      tmem_ld16(tmem + (uint32_t(sp * 32) << 16) + uint32_t(buf * NR + c0), v);
+      tmem_wait_ld();
+#pragma unroll
+      for (int j = 0; j < 16; ++j) stage[(c0 + j) * 128 + m_loc] = f32_to_bf16_rne(v[j] + bias);
+    }
+  }
+  tc_fence_before();
+  __syncwarp();
+  if (lane == 0) mbar_arrive(acc_empty);
+  named_bar_sync(1, kWgEpiThreads);            // the staging tile is complete
+  if (*abort_flag == 0) {
+    const int mt = min(128, p.M - w.m0);       // features of this tile
+    uint16_t* out = p.out + int64_t(w.n0) * p.out_row_stride + int64_t(w.h) * p.out_head_stride +
+                    w.m0;
+    if (p.vec_out != 0) {
+      // host-checked: M, both strides and the base are multiples of 8 elements
+      const int cpr = mt >> 3;                 // 16-byte pieces per row
+#pragma unroll 4
+      for (int idx = m_loc; idx < nrows * cpr; idx += kWgEpiThreads) {
+        const int n = idx / cpr, c = idx - (idx / cpr) * cpr;
+        *reinterpret_cast<uint4*>(out + int64_t(n) * p.out_row_stride + c * 8) =
+            *reinterpret_cast<const uint4*>(stage + n * 128 + c * 8);
+      }
+    } else {
+      for (int idx = m_loc; idx < nrows * mt; idx += kWgEpiThreads) {
+        const int n = idx / mt, c = idx - (idx / mt) * mt;
+        out[int64_t(n) * p.out_row_stride + c] = stage[n * 128 + c];
+      }
+    }
+  }
+  named_bar_sync(1, kWgEpiThreads);            // the staging tile may be reused
+}
+
 template <int NR>
 __global__ void __launch_bounds__(kWgThreads, 1) wgemm_kernel(const __grid_constant__ WGemmParams p) {
   using Lay = WgLayout<NR>;
@@ -474,33 +530,9 @@ __global__ void __launch_bounds__(kWgThreads, 1) wgemm_kernel(const __grid_const
                             ok, abort_flag, last_flag);
         continue;
       }
-      if (ok) {
-        const int m = w.m0 + sp * 32 + lane;   // output feature of this thread's TMEM lane
-        const float bias = (p.bias != nullptr && m < p.M)
-                               ? bf16_bits_to_f32(p.bias[int64_t(w.h) * p.M + m]) : 0.0f;
-        uint16_t* out = p.out + int64_t(w.h) * p.out_head_stride + m +
-                        int64_t(w.n0) * p.out_row_stride;
-        const int nrows = min(NR, p.rows - w.n0);
-        // Not unrolled: the code runs once per item with a cold instruction cache (the decode
-        // kernel runs between these launches), and a fully unrolled drain of 128 rows cost
-        // more in instruction fetch than it saved.
-#pragma unroll 1
-        for (int c0 = 0; c0 < NR; c0 += 16) {
-          float v[16];
-          tmem_ld16(tmem + (uint32_t(sp * 32) << 16) + uint32_t(buf * NR + c0), v);
-          tmem_wait_ld();
-          if (m < p.M) {
-#pragma unroll
-            for (int j = 0; j < 16; ++j) {
-              if (c0 + j < nrows) *out = f32_to_bf16_rne(v[j] + bias);
-              out += p.out_row_stride;
-            }
-          }
-        }
-      }
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&acc_empty[buf]);
+      plain_epilogue<NR>(p, w, buf, tmem, sp, lane,
+                         reinterpret_cast<uint16_t*>(base + Lay::kBars + 256), &acc_empty[buf],
+                         ok, abort_flag);
     }
   }
   tc_fence_before();
@@ -511,9 +543,9 @@ __global__ void __launch_bounds__(kWgThreads, 1) wgemm_kernel(const __grid_const
 template <int NR>
 static cudaError_t launch_wgemm_nr(const WGemmParams& p, int max_ctas, cudaStream_t stream) {
   const bool append = p.cache != nullptr;
-  // the fused append stages one [NR][128] bf16 tile and NR cache-row indices after the
-  // barriers
-  const int smem = WgLayout<NR>::kTotal + (append ? NR * 128 * 2 + NR * 8 : 0);
+  // the epilogue stages one [NR][128] bf16 tile after the barriers (the fused append also
+  // NR cache-row indices)
+  const int smem = WgLayout<NR>::kTotal + NR * 128 * 2 + (append ? NR * 8 : 0);
   cudaError_t e = cudaFuncSetAttribute(wgemm_kernel<NR>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
