@@ -423,18 +423,12 @@ def run_gpu(args, cfg, rank, world, dist):
         torch.cuda.synchronize()
 
     def one_step():
-        # The four calls back to back: each kernel is launched so that it may start while
-        # the previous one drains (programmatic dependent launch), so no event is recorded
-        # between them (a stream event between two kernels would serialise them).
-        mla.mla_cache_append(prob.dims, prob.c_new, prob.k_new, prob.cos_q, prob.sin_q,
-                             prob.block_table, prob.start_pos, prob.cache,
-                             dev_error=prob.workspace.view(torch.int32)[:1], stream=stream)
-        mla.mla_absorb_q(prob.dims, prob.q_nope, prob.q_pe, prob.cos_q, prob.sin_q, prob.w_uk,
-                         prob.q_ext, stream=stream)
-        mla.mla_decode_attn(prob.dims, prob.q_ext, prob.cache, prob.block_table, prob.seq_lens,
-                            prob.max_seq_len, prob.workspace, prob.o_latent, prob.lse,
-                            causal=cfg.causal, num_splits=args.splits, stream=stream)
-        mla.mla_out_up(prob.dims, prob.o_latent, prob.w_uv, prob.o, bias=prob.bias, stream=stream)
+        # One library call: the append folded into the absorption kernel, the decode (and
+        # the merge of cut sequences), the up-projection. Each kernel is launched so that it
+        # may start while the previous one drains (programmatic dependent launch), so no
+        # event is recorded between them (a stream event between two kernels would
+        # serialise them).
+        prob.step(stream)
 
     for _ in range(args.warmup):
         if flush is not None:
@@ -536,10 +530,10 @@ def run_gpu(args, cfg, rank, world, dist):
     tokens = cfg.batch * cfg.q_len
     value = world * tokens / (t_step * 1e-3)
     roof = roofline_of(cfg, wl.seq_lens, t_dec, peaks)
-    # append, absorb, decode, out_up (+ the split combine when the plan has > 1 split;
-    # a one-split plan needs only the 256-byte error-word workspace)
+    # absorb with the append folded in, decode, out_up (+ the split combine when the plan has
+    # > 1 split; a one-split plan needs only the 256-byte error-word workspace)
     merge = 1 if plan_splits_ws > 256 else 0
-    launches = (4 + merge) * args.steps + (1 + merge) * DECODE_BLOCK
+    launches = (3 + merge) * args.steps + (1 + merge) * DECODE_BLOCK
     line = {
         "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": t_step,

@@ -37,7 +37,7 @@ C_SYMBOLS = ("mla_row_width", "mla_status_string", "mla_cache_append", "mla_abso
              "mla_get_device_status", "mla_decode_attn_noalloc", "mla_selftest_wait_timeout",
              "mla_kv_shared_decode_dims", "mla_kv_shared_query", "mla_kv_shared_output",
              "mla_down_kv_workspace_size", "mla_down_kv_append", "mla_out_proj_workspace_size",
-             "mla_out_proj")
+             "mla_out_proj", "mla_decode_step")
 
 
 class MlaError(RuntimeError):
@@ -116,6 +116,10 @@ def lib() -> ctypes.CDLL:
     L.mla_out_proj.argtypes = [D, _P, _P, _I64, _P, _P, _P, _I32, _I32, _P, ctypes.c_size_t, _P,
                                _P, _P]
     L.mla_out_proj.restype = _I32
+    L.mla_decode_step.argtypes = [D, _P, _P, _P, _P, _P, _I32, _P, _P, _P, _P, _P, _I64, _P, _I64,
+                                  _P, _P, _I64, _P, _I32, _P, _I32, _I32, _I32, _I32, _I32, _P,
+                                  _P, ctypes.c_size_t, _P, _P, _P, _P]
+    L.mla_decode_step.restype = _I32
     _lib = L
     return L
 
@@ -413,14 +417,59 @@ def mla_selftest_wait_timeout(dev_error, stream=None) -> None:
 def mla_decode_step(dims: MlaDims, *, c_kv_new, k_r_new, cos_new, sin_new, start_pos,
                     q_nope, q_pe, cos_q, sin_q, w_uk, w_uv, bias, cache, block_table, seq_lens,
                     max_seq_len: int, q_ext, workspace, o_latent, lse, o, causal: bool = True,
-                    num_splits: int = 0, stream=None) -> None:
-    """One decode step through the four library calls, on one stream, all buffers given."""
-    mla_cache_append(dims, c_kv_new, k_r_new, cos_new, sin_new, block_table, start_pos, cache,
-                     dev_error=workspace.view(torch.int32)[:1], stream=stream)
-    mla_absorb_q(dims, q_nope, q_pe, cos_q, sin_q, w_uk, q_ext, stream=stream)
-    mla_decode_attn(dims, q_ext, cache, block_table, seq_lens, max_seq_len, workspace, o_latent,
-                    lse, causal=causal, num_splits=num_splits, stream=stream)
-    mla_out_up(dims, o_latent, w_uv, o, bias=bias, stream=stream)
+                    num_splits: int = 0, w_uk_head_stride: Optional[int] = None,
+                    w_uv_head_stride: Optional[int] = None, stream=None) -> None:
+    """One decode step in one library call (append, absorb, attention, up-projection): the
+    outputs of mla_cache_append, mla_absorb_q, mla_decode_attn and mla_out_up on the same
+    arguments. c_kv_new [B, n, r] / k_r_new [B, n, G, d_r] are the appended tokens."""
+    B, q = q_nope.shape[0], q_nope.shape[1]
+    n = c_kv_new.shape[1]
+    H, G, dr, r, dv, D = (dims.num_heads, dims.num_kv_groups, dims.rope_dim, dims.kv_lora_rank,
+                          dims.v_head_dim, dims.row_width)
+    _need(c_kv_new, "c_kv_new", torch.bfloat16, (B, n, r))
+    _need(q_nope, "q_nope", torch.bfloat16, (B, q, H, dims.qk_nope_dim))
+    if dr > 0:
+        _need(k_r_new, "k_r_new", torch.bfloat16, (B, n, G, dr))
+        _need(cos_new, "cos_new", torch.float32, (B, n, G, dr // 2))
+        _need(sin_new, "sin_new", torch.float32, (B, n, G, dr // 2))
+        _need(q_pe, "q_pe", torch.bfloat16, (B, q, H, dr))
+        _need(cos_q, "cos_q", torch.float32, (B, q, G, dr // 2))
+        _need(sin_q, "sin_q", torch.float32, (B, q, G, dr // 2))
+    _need(start_pos, "start_pos", torch.int32, (B,))
+    if w_uk_head_stride is None:
+        _need(w_uk, "w_uk", torch.bfloat16, (H, dims.qk_nope_dim, r))
+        w_uk_head_stride = dims.qk_nope_dim * r
+    else:
+        _need(w_uk, "w_uk", torch.bfloat16)
+    if w_uv_head_stride is None:
+        _need(w_uv, "w_uv", torch.bfloat16, (H, dv, r))
+        w_uv_head_stride = dv * r
+    else:
+        _need(w_uv, "w_uv", torch.bfloat16)
+    if bias is not None:
+        _need(bias, "bias", torch.bfloat16, (H, dv))
+    _need(cache, "cache", torch.bfloat16)
+    if cache.dim() != 3 or cache.shape[1] != dims.page_size or cache.shape[2] != D:
+        raise MlaError(f"cache shape {tuple(cache.shape)} does not match dims", MLA_ERR_INVALID_ARG)
+    _need(block_table, "block_table", torch.int32)
+    if block_table.dim() != 2 or block_table.shape[0] != B:
+        raise MlaError("block_table must be [B, max_pages]", MLA_ERR_INVALID_ARG)
+    _need(seq_lens, "seq_lens", torch.int32, (B,))
+    _need(q_ext, "q_ext", torch.bfloat16, (B, q, H, D))
+    _need(workspace, "workspace", torch.uint8)
+    _need(o_latent, "o_latent", torch.bfloat16, (B, q, H, r))
+    _need(lse, "lse", torch.float32, (B, q, H))
+    _need(o, "o", torch.bfloat16, (B, q, H, dv))
+    st = lib().mla_decode_step(
+        ctypes.byref(dims), _ptr(c_kv_new), _ptr(k_r_new if dr > 0 else None),
+        _ptr(cos_new if dr > 0 else None), _ptr(sin_new if dr > 0 else None), _ptr(start_pos), n,
+        _ptr(q_nope), _ptr(q_pe if dr > 0 else None), _ptr(cos_q if dr > 0 else None),
+        _ptr(sin_q if dr > 0 else None), _ptr(w_uk), int(w_uk_head_stride), _ptr(w_uv),
+        int(w_uv_head_stride), _ptr(bias), _ptr(cache), cache.shape[0], _ptr(block_table),
+        block_table.shape[1], _ptr(seq_lens), B, q, int(max_seq_len), 1 if causal else 0,
+        int(num_splits), _ptr(q_ext), _ptr(workspace), workspace.numel(), _ptr(o_latent),
+        _ptr(lse), _ptr(o), _stream(stream))
+    _check(st, "mla_decode_step")
 
 
 __all__ = ["MlaDims", "MlaError", "make_dims", "lib", "mla_row_width", "mla_cache_append",

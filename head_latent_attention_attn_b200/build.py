@@ -19,7 +19,7 @@ OBJ = os.path.join(ROOT, "_build", "mla")
 LIB = os.path.join(PKG, "libmla.so")
 SOURCES = ["host_common.cu", "api.cu", "append.cu", "wgemm.cu", "decode.cu", "decode_pair.cu",
            "noalloc.cu", "kv_shared.cu", "oproj.cu"]
-HEADERS = ["ptx.cuh", "kernels.h", "host_common.h", "decode_sched.cuh"]
+HEADERS = ["ptx.cuh", "kernels.h", "host_common.h", "decode_sched.cuh", "append.cuh"]
 
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 FLAGS = ["-O3", "-lineinfo", "-std=c++17", "-Xcompiler", "-fPIC", "-Xcompiler", "-O2",

@@ -90,6 +90,7 @@ struct DecodePlan {
   size_t range_off, unit_start_off, part_lse_off, part_o_off;
 };
 
+
 size_t align256(size_t x) { return (x + 255) / 256 * 256; }
 
 mla_status plan_decode(const mla_dims* d, int32_t batch, int32_t q_len, int32_t max_seq_len,
@@ -189,21 +190,28 @@ const char* mla_status_string(mla_status s) {
   return "MLA_ERR_UNKNOWN";
 }
 
-mla_status mla_cache_append(const mla_dims* dims, const void* c_kv, const void* k_r,
-                            const float* rope_cos, const float* rope_sin,
-                            const int32_t* block_table, int32_t max_pages_per_seq,
-                            const int32_t* start_pos, int32_t batch, int32_t n_new, void* cache,
-                            int64_t num_pages, int32_t* dev_error, void* stream) {
+}  // extern "C"
+
+namespace {
+
+// Validation and parameters of mla_cache_append; *empty is set when there is nothing to do.
+mla_status build_append(const mla_dims* dims, const void* c_kv, const void* k_r,
+                        const float* rope_cos, const float* rope_sin, const int32_t* block_table,
+                        int32_t max_pages_per_seq, const int32_t* start_pos, int32_t batch,
+                        int32_t n_new, void* cache, int64_t num_pages, int32_t* dev_error,
+                        AppendParams* out, bool* empty) {
   mla_status st = check_dims(dims);
   if (st != MLA_OK) return st;
   if (batch < 0 || n_new < 0 || max_pages_per_seq <= 0 || num_pages <= 0 ||
       num_pages > INT32_MAX)
     return MLA_ERR_INVALID_ARG;
-  if (batch == 0 || n_new == 0) return MLA_OK;
+  *empty = batch == 0 || n_new == 0;
+  if (*empty) return MLA_OK;
   if (!c_kv || !block_table || !start_pos || !cache) return MLA_ERR_INVALID_ARG;
   if (dims->rope_dim > 0 && (!k_r || !rope_cos || !rope_sin)) return MLA_ERR_INVALID_ARG;
   if (!aligned(c_kv, 16) || !aligned(cache, 16)) return MLA_ERR_INVALID_ARG;
-  AppendParams p{};
+  AppendParams& p = *out;
+  p = AppendParams{};
   p.c_kv = static_cast<const uint16_t*>(c_kv);
   p.k_r = static_cast<const uint16_t*>(k_r);
   p.rope_cos = rope_cos;
@@ -220,21 +228,35 @@ mla_status mla_cache_append(const mla_dims* dims, const void* c_kv, const void* 
   p.groups = dims->num_kv_groups;
   p.rope_dim = dims->rope_dim;
   p.page_size = dims->page_size;
-  return launch_cache_append(p, as_stream(stream)) == cudaSuccess ? MLA_OK : MLA_ERR_CUDA;
+  return MLA_OK;
+}
+
+// The output tiles of absorb / out_up go out by TMA store when the strides allow it: box
+// {128 features, 1 head, nr rows} over {M, H, rows}; columns past M and rows past `rows`
+// are clipped by the TMA. Returns 0 (element copies) when the map cannot be made.
+int encode_out_map(WGemmParams& p, void* out, int nr) {
+  if (p.M % 8 != 0 || p.out_head_stride % 8 != 0 || p.out_row_stride % 8 != 0) return 0;
+  const uint64_t d3[3] = {uint64_t(p.M), uint64_t(p.heads), uint64_t(p.rows)};
+  const uint64_t s3[2] = {uint64_t(p.out_head_stride) * 2, uint64_t(p.out_row_stride) * 2};
+  const uint32_t box[3] = {128, 1, uint32_t(nr)};
+  return encode_bf16_map(&p.tm_out, out, 3, d3, s3, box, CU_TENSOR_MAP_SWIZZLE_NONE) ? 1 : 0;
 }
 
 static int pick_nr(int64_t rows) {
   return rows <= 16 ? 16 : rows <= 32 ? 32 : rows <= 64 ? 64 : 128;
 }
 
-mla_status mla_absorb_q(const mla_dims* dims, const void* q_nope, const void* q_pe,
+// Validation and parameters of mla_absorb_q (tensor maps encoded); *nr is the row tile and
+// *empty is set when there is nothing to do.
+mla_status build_absorb(const mla_dims* dims, const void* q_nope, const void* q_pe,
                         const float* rope_cos, const float* rope_sin, const void* w_uk,
                         int64_t w_uk_head_stride, int32_t batch, int32_t q_len, void* q_ext,
-                        void* stream) {
+                        WGemmParams* out, int* nr_out, bool* empty, bool encode = true) {
   mla_status st = check_dims(dims);
   if (st != MLA_OK) return st;
   if (batch < 0 || q_len <= 0) return MLA_ERR_INVALID_ARG;
-  if (batch == 0) return MLA_OK;
+  *empty = batch == 0;
+  if (*empty) return MLA_OK;
   const int H = dims->num_heads, r = dims->kv_lora_rank, dn = dims->qk_nope_dim;
   if (!q_nope || !w_uk || !q_ext) return MLA_ERR_INVALID_ARG;
   if (dims->rope_dim > 0 && (!q_pe || !rope_cos || !rope_sin)) return MLA_ERR_INVALID_ARG;
@@ -242,8 +264,10 @@ mla_status mla_absorb_q(const mla_dims* dims, const void* q_nope, const void* q_
   if (!aligned(q_nope, 16) || !aligned(w_uk, 16) || !aligned(q_ext, 16)) return MLA_ERR_INVALID_ARG;
   const int64_t rows = int64_t(batch) * q_len;
   if (rows > int64_t(65535) * 128) return MLA_ERR_UNSUPPORTED;
+  if (!encode) return MLA_OK;   // validation only
   const int D = row_width(dims);
-  WGemmParams p{};
+  WGemmParams& p = *out;
+  p = WGemmParams{};
   {
     const uint64_t dims3[3] = {uint64_t(r), uint64_t(dn), uint64_t(H)};
     const uint64_t str[2] = {uint64_t(r) * 2, uint64_t(w_uk_head_stride) * 2};
@@ -269,7 +293,6 @@ mla_status mla_absorb_q(const mla_dims* dims, const void* q_nope, const void* q_
   p.rows = int32_t(rows);
   p.heads = H;
   p.a_mn = 1;
-  p.vec_out = (D % 8 == 0 && r % 8 == 0) ? 1 : 0;   // q_ext is 16-byte aligned (checked above)
   p.splits = 1;
   p.q_pe = dims->rope_dim > 0 ? static_cast<const uint16_t*>(q_pe) : nullptr;
   p.rope_cos = rope_cos;
@@ -278,22 +301,28 @@ mla_status mla_absorb_q(const mla_dims* dims, const void* q_nope, const void* q_
   p.rope_dim = dims->rope_dim;
   p.rope_vec = (dims->rope_dim % 8 == 0 && aligned(q_pe, 8) && aligned(rope_cos, 16) &&
                 aligned(rope_sin, 16)) ? 1 : 0;
-  return launch_wgemm(p, nr, num_sms(), as_stream(stream)) == cudaSuccess ? MLA_OK : MLA_ERR_CUDA;
+  p.tma_out = encode_out_map(p, p.out, nr);
+  *nr_out = nr;
+  return MLA_OK;
 }
 
-mla_status mla_out_up(const mla_dims* dims, const void* o_latent, const void* w_uv,
-                      int64_t w_uv_head_stride, const void* bias, int32_t rows, void* o,
-                      void* stream) {
+// Validation and parameters of mla_out_up (tensor maps encoded).
+mla_status build_out_up(const mla_dims* dims, const void* o_latent, const void* w_uv,
+                        int64_t w_uv_head_stride, const void* bias, int32_t rows, void* o,
+                        WGemmParams* out, int* nr_out, bool* empty, bool encode = true) {
   mla_status st = check_dims(dims);
   if (st != MLA_OK) return st;
   if (rows < 0) return MLA_ERR_INVALID_ARG;
-  if (rows == 0) return MLA_OK;
+  *empty = rows == 0;
+  if (*empty) return MLA_OK;
   const int H = dims->num_heads, r = dims->kv_lora_rank, dv = dims->v_head_dim;
   if (!o_latent || !w_uv || !o) return MLA_ERR_INVALID_ARG;
   if (w_uv_head_stride < int64_t(dv) * r || w_uv_head_stride % 8 != 0) return MLA_ERR_INVALID_ARG;
   if (!aligned(o_latent, 16) || !aligned(w_uv, 16) || !aligned(o, 16)) return MLA_ERR_INVALID_ARG;
   if (int64_t(rows) > int64_t(65535) * 128) return MLA_ERR_UNSUPPORTED;
-  WGemmParams p{};
+  if (!encode) return MLA_OK;   // validation only
+  WGemmParams& p = *out;
+  p = WGemmParams{};
   {
     const uint64_t dims3[3] = {uint64_t(r), uint64_t(dv), uint64_t(H)};
     const uint64_t str[2] = {uint64_t(r) * 2, uint64_t(w_uv_head_stride) * 2};
@@ -319,9 +348,53 @@ mla_status mla_out_up(const mla_dims* dims, const void* o_latent, const void* w_
   p.rows = rows;
   p.heads = H;
   p.a_mn = 0;
-  p.vec_out = dv % 8 == 0 ? 1 : 0;                  // o is 16-byte aligned (checked above)
   p.splits = 1;
   p.q_pe = nullptr;
+  p.tma_out = encode_out_map(p, p.out, nr);
+  *nr_out = nr;
+  return MLA_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+mla_status mla_cache_append(const mla_dims* dims, const void* c_kv, const void* k_r,
+                            const float* rope_cos, const float* rope_sin,
+                            const int32_t* block_table, int32_t max_pages_per_seq,
+                            const int32_t* start_pos, int32_t batch, int32_t n_new, void* cache,
+                            int64_t num_pages, int32_t* dev_error, void* stream) {
+  AppendParams p;
+  bool empty = false;
+  const mla_status st = build_append(dims, c_kv, k_r, rope_cos, rope_sin, block_table,
+                                     max_pages_per_seq, start_pos, batch, n_new, cache,
+                                     num_pages, dev_error, &p, &empty);
+  if (st != MLA_OK || empty) return st;
+  return launch_cache_append(p, as_stream(stream)) == cudaSuccess ? MLA_OK : MLA_ERR_CUDA;
+}
+
+mla_status mla_absorb_q(const mla_dims* dims, const void* q_nope, const void* q_pe,
+                        const float* rope_cos, const float* rope_sin, const void* w_uk,
+                        int64_t w_uk_head_stride, int32_t batch, int32_t q_len, void* q_ext,
+                        void* stream) {
+  WGemmParams p;
+  int nr = 0;
+  bool empty = false;
+  const mla_status st = build_absorb(dims, q_nope, q_pe, rope_cos, rope_sin, w_uk,
+                                     w_uk_head_stride, batch, q_len, q_ext, &p, &nr, &empty);
+  if (st != MLA_OK || empty) return st;
+  return launch_wgemm(p, nr, num_sms(), as_stream(stream)) == cudaSuccess ? MLA_OK : MLA_ERR_CUDA;
+}
+
+mla_status mla_out_up(const mla_dims* dims, const void* o_latent, const void* w_uv,
+                      int64_t w_uv_head_stride, const void* bias, int32_t rows, void* o,
+                      void* stream) {
+  WGemmParams p;
+  int nr = 0;
+  bool empty = false;
+  const mla_status st = build_out_up(dims, o_latent, w_uv, w_uv_head_stride, bias, rows, o, &p,
+                                     &nr, &empty);
+  if (st != MLA_OK || empty) return st;
   return launch_wgemm(p, nr, num_sms(), as_stream(stream)) == cudaSuccess ? MLA_OK : MLA_ERR_CUDA;
 }
 
@@ -528,27 +601,36 @@ size_t mla_decode_workspace_size(const mla_dims* dims, int32_t batch, int32_t q_
   return P.ws_bytes;
 }
 
-mla_status mla_decode_attn(const mla_dims* dims, const void* q_ext, const void* cache,
-                           int64_t num_pages, const int32_t* block_table,
-                           int32_t max_pages_per_seq, const int32_t* seq_lens, int32_t batch,
-                           int32_t q_len, int32_t max_seq_len, int32_t causal,
-                           int32_t num_splits, void* workspace, size_t workspace_bytes,
-                           void* o_latent, float* lse, void* stream) {
-  DecodePlan P;
+}  // extern "C"
+
+namespace {
+
+// Validation, plan and parameters of mla_decode_attn (tensor maps encoded); *empty is set
+// when there is nothing to do.
+mla_status build_decode(const mla_dims* dims, const void* q_ext, const void* cache,
+                        int64_t num_pages, const int32_t* block_table, int32_t max_pages_per_seq,
+                        const int32_t* seq_lens, int32_t batch, int32_t q_len,
+                        int32_t max_seq_len, int32_t causal, int32_t num_splits, void* workspace,
+                        size_t workspace_bytes, void* o_latent, float* lse, DecodePlan* Pout,
+                        DecodeParams* pout, bool* empty, bool encode = true) {
+  DecodePlan& P = *Pout;
   mla_status st = plan_decode(dims, batch, q_len, max_seq_len, num_splits, &P);
   if (st != MLA_OK) return st;
   if (num_pages <= 0 || num_pages * kDecodeTok > (int64_t(1) << 31) || max_pages_per_seq <= 0 ||
       (causal != 0 && causal != 1))
     return MLA_ERR_INVALID_ARG;
-  if (batch == 0) return MLA_OK;
+  *empty = batch == 0;
+  if (*empty) return MLA_OK;
   if (!q_ext || !cache || !block_table || !seq_lens || !o_latent || !lse)
     return MLA_ERR_INVALID_ARG;
   if (!aligned(q_ext, 16) || !aligned(cache, 16)) return MLA_ERR_INVALID_ARG;
   if (!workspace || !aligned(workspace, 256)) return MLA_ERR_WORKSPACE;
   if (workspace_bytes < P.ws_bytes) return MLA_ERR_WORKSPACE;
+  if (!encode) return MLA_OK;   // validation only
   const int D = row_width(dims);
   const int64_t qH = int64_t(q_len) * dims->num_heads;
-  DecodeParams p{};
+  DecodeParams& p = *pout;
+  p = DecodeParams{};
   {
     const uint64_t d2[2] = {uint64_t(D), uint64_t(num_pages) * kDecodeTok};
     const uint64_t s2[1] = {uint64_t(D) * 2};
@@ -603,7 +685,11 @@ mla_status mla_decode_attn(const mla_dims* dims, const void* q_ext, const void* 
   p.tmem_cols = P.tmem_cols;
   p.npt = P.npt;
   p.scale_log2 = dims->softmax_scale * 1.4426950408889634f;
-  cudaStream_t s = as_stream(stream);
+  return MLA_OK;
+}
+
+// The decode kernel of a built plan and, when units may be cut between CTAs, the merge.
+mla_status launch_decode_plan(const DecodePlan& P, const DecodeParams& p, cudaStream_t s) {
   const cudaError_t le = P.pair ? launch_decode_pair(p, dim3(P.grid), P.smem, s)
                                 : launch_decode(p, P.ncol, dim3(P.grid), P.smem, s);
   if (le != cudaSuccess) return MLA_ERR_CUDA;
@@ -614,12 +700,12 @@ mla_status mla_decode_attn(const mla_dims* dims, const void* q_ext, const void* 
     c.part_lse = p.part_lse;
     c.unit_start = p.unit_start;
     c.range_len = p.range_len;
-    c.seq_lens = seq_lens;
+    c.seq_lens = p.seq_lens;
     c.o_latent = p.o_latent;
-    c.lse = lse;
-    c.q_len = q_len;
-    c.max_seq_len = max_seq_len;
-    c.max_pages = max_pages_per_seq;
+    c.lse = p.lse;
+    c.q_len = p.q_len;
+    c.max_seq_len = p.max_seq_len;
+    c.max_pages = p.max_pages;
     c.qH = p.qH;
     c.r = p.r;
     c.ncol = P.ncol;
@@ -629,6 +715,75 @@ mla_status mla_decode_attn(const mla_dims* dims, const void* q_ext, const void* 
     if (launch_combine(c, s) != cudaSuccess) return MLA_ERR_CUDA;
   }
   return MLA_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+mla_status mla_decode_attn(const mla_dims* dims, const void* q_ext, const void* cache,
+                           int64_t num_pages, const int32_t* block_table,
+                           int32_t max_pages_per_seq, const int32_t* seq_lens, int32_t batch,
+                           int32_t q_len, int32_t max_seq_len, int32_t causal,
+                           int32_t num_splits, void* workspace, size_t workspace_bytes,
+                           void* o_latent, float* lse, void* stream) {
+  DecodePlan P;
+  DecodeParams p;
+  bool empty = false;
+  const mla_status st = build_decode(dims, q_ext, cache, num_pages, block_table,
+                                     max_pages_per_seq, seq_lens, batch, q_len, max_seq_len,
+                                     causal, num_splits, workspace, workspace_bytes, o_latent,
+                                     lse, &P, &p, &empty);
+  if (st != MLA_OK || empty) return st;
+  return launch_decode_plan(P, p, as_stream(stream));
+}
+
+mla_status mla_decode_step(const mla_dims* dims, const void* c_kv_new, const void* k_r_new,
+                           const float* rope_cos_new, const float* rope_sin_new,
+                           const int32_t* start_pos, int32_t n_new, const void* q_nope,
+                           const void* q_pe, const float* rope_cos_q, const float* rope_sin_q,
+                           const void* w_uk, int64_t w_uk_head_stride, const void* w_uv,
+                           int64_t w_uv_head_stride, const void* bias_v, void* cache,
+                           int64_t num_pages, const int32_t* block_table,
+                           int32_t max_pages_per_seq, const int32_t* seq_lens, int32_t batch,
+                           int32_t q_len, int32_t max_seq_len, int32_t causal,
+                           int32_t num_splits, void* q_ext, void* workspace,
+                           size_t workspace_bytes, void* o_latent, float* lse, void* o,
+                           void* stream) {
+  // every part is validated (no tensor map encoded, nothing launched) before any is built
+  AppendParams ap;
+  bool ap_empty = false;
+  mla_status st = build_append(dims, c_kv_new, k_r_new, rope_cos_new, rope_sin_new, block_table,
+                               max_pages_per_seq, start_pos, batch, n_new, cache, num_pages,
+                               static_cast<int32_t*>(workspace), &ap, &ap_empty);
+  if (st != MLA_OK) return st;
+  const int64_t rows = int64_t(batch) * q_len;
+  if (rows > INT32_MAX) return MLA_ERR_UNSUPPORTED;
+  WGemmParams ab, ou;
+  DecodePlan P;
+  DecodeParams dp;
+  int nr_ab = 0, nr_ou = 0;
+  bool ab_empty = false, de_empty = false, ou_empty = false;
+  for (int pass = 0; pass < 2; ++pass) {
+    const bool enc = pass == 1;
+    st = build_absorb(dims, q_nope, q_pe, rope_cos_q, rope_sin_q, w_uk, w_uk_head_stride, batch,
+                      q_len, q_ext, &ab, &nr_ab, &ab_empty, enc);
+    if (st != MLA_OK) return st;
+    st = build_decode(dims, q_ext, cache, num_pages, block_table, max_pages_per_seq, seq_lens,
+                      batch, q_len, max_seq_len, causal, num_splits, workspace, workspace_bytes,
+                      o_latent, lse, &P, &dp, &de_empty, enc);
+    if (st != MLA_OK) return st;
+    st = build_out_up(dims, o_latent, w_uv, w_uv_head_stride, bias_v, int32_t(rows), o, &ou,
+                      &nr_ou, &ou_empty, enc);
+    if (st != MLA_OK) return st;
+    if (ab_empty) return MLA_OK;   // batch == 0: nothing to do anywhere
+  }
+  cudaStream_t s = as_stream(stream);
+  if (!ap_empty) ab.app = ap;     // the absorption's epilogue warps write the new rows
+  if (launch_wgemm(ab, nr_ab, num_sms(), s) != cudaSuccess) return MLA_ERR_CUDA;
+  st = launch_decode_plan(P, dp, s);
+  if (st != MLA_OK) return st;
+  return launch_wgemm(ou, nr_ou, num_sms(), s) == cudaSuccess ? MLA_OK : MLA_ERR_CUDA;
 }
 
 }  // extern "C"

@@ -1,9 +1,6 @@
 // append.cu - mla_cache_append kernel: scatter new tokens' latent and rotated key into
-// the paged cache. One warp per token: the latent row moves as 16-byte vectors, the
-// rotary pairs are rotated in fp32 (separately rounded multiply / subtract / add) and
-// rounded to bf16 with ties to even.
-#include "kernels.h"
-#include "ptx.cuh"
+// the paged cache, one warp per token (append.cuh).
+#include "append.cuh"
 
 namespace mla {
 
@@ -12,47 +9,8 @@ __global__ void __launch_bounds__(256) cache_append_kernel(AppendParams p) {
   grid_dep_launch();
   const int64_t gw = (int64_t(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
   const int lane = threadIdx.x & 31;
-  const int64_t ntok = int64_t(p.batch) * p.n_new;
-  if (gw >= ntok) return;
-  const int b = int(gw / p.n_new);
-  const int t = int(gw % p.n_new);
-  const int64_t pos = int64_t(p.start_pos[b]) + t;
-  const int64_t lp = pos >= 0 ? pos / p.page_size : -1;
-  if (pos < 0 || lp >= p.max_pages) {
-    if (lane == 0 && p.dev_error) atomicOr(p.dev_error, MLA_DEVERR_BOUNDS);
-    return;
-  }
-  const int32_t page = p.block_table[int64_t(b) * p.max_pages + lp];
-  if (page < 0 || page >= p.num_pages) {
-    if (lane == 0 && p.dev_error) atomicOr(p.dev_error, MLA_DEVERR_BOUNDS);
-    return;
-  }
-  const int D = p.r + p.groups * p.rope_dim;
-  uint16_t* dst = p.cache + (int64_t(page) * p.page_size + pos % p.page_size) * D;
-
-  // latent: exact copy, 8 bf16 per 16-byte vector (r % 8 == 0, rows 16-byte aligned)
-  const uint4* src4 = reinterpret_cast<const uint4*>(p.c_kv + gw * p.r);
-  uint4* dst4 = reinterpret_cast<uint4*>(dst);
-  for (int i = lane; i < p.r / 8; i += 32) dst4[i] = src4[i];
-
-  // rotary key of every group
-  const int half = p.rope_dim / 2;
-  const int npairs = p.groups * half;
-  const uint16_t* kr = p.k_r + gw * int64_t(p.groups) * p.rope_dim;
-  const float* cs = p.rope_cos + gw * npairs;
-  const float* sn = p.rope_sin + gw * npairs;
-  for (int idx = lane; idx < npairs; idx += 32) {
-    const int g = idx / half;
-    const int j = idx - g * half;
-    const float x0 = bf16_bits_to_f32(kr[g * p.rope_dim + j]);
-    const float x1 = bf16_bits_to_f32(kr[g * p.rope_dim + j + half]);
-    const float c = cs[idx];
-    const float s = sn[idx];
-    const float y0 = __fsub_rn(__fmul_rn(x0, c), __fmul_rn(x1, s));
-    const float y1 = __fadd_rn(__fmul_rn(x1, c), __fmul_rn(x0, s));
-    dst[p.r + g * p.rope_dim + j] = f32_to_bf16_rne(y0);
-    dst[p.r + g * p.rope_dim + j + half] = f32_to_bf16_rne(y1);
-  }
+  if (gw >= int64_t(p.batch) * p.n_new) return;
+  append_token(p, gw, lane);
 }
 
 cudaError_t launch_cache_append(const AppendParams& p, cudaStream_t stream) {

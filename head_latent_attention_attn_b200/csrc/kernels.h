@@ -73,12 +73,13 @@ struct WGemmParams {
   CUtensorMap tm_w;          // 3D weight map, box 128 x 64 (see launcher)
   CUtensorMap tm_x;          // 3D activations {K, H, rows}, box {64, 1, NR}
   uint16_t* out;             // element (n, h, m) at n*out_row_stride + h*out_head_stride + m
+  CUtensorMap tm_out;        // 3D {M, H, rows} over out, box {min(128, M), 1, NR}
   int64_t out_row_stride, out_head_stride;
   const uint16_t* bias;      // [H, M] or null
   int32_t* dev_error;
   int32_t M, K, rows, heads;
   int32_t a_mn;              // 1: weight stored [K][M] (W_UK), 0: stored [M][K] (W_UV)
-  int32_t vec_out;           // 1: out, both strides and M are multiples of 8 elements
+  int32_t tma_out;           // 1: tm_out stores the output tiles (else element copies)
   // rotary part of q_ext (mla_absorb_q only; q_pe == nullptr otherwise)
   const uint16_t* q_pe;      // [rows, H, d_r]
   const float* rope_cos;     // [rows, G, d_r/2]
@@ -100,6 +101,9 @@ struct WGemmParams {
   int32_t splits;
   float* acc;                // [rows, D] fp32, zero between calls
   int32_t* tile_done;        // [tiles], zero between calls
+  // cache append folded into the absorption (the one-call decode step; batch == 0 when
+  // unused): the epilogue warps write the new tokens' cache rows before their first item
+  AppendParams app;
 };
 // max_ctas: the persistent grid's size limit (one CTA per SM). With p.cache set the
 // output goes into the paged cache (see WGemmParams) instead of p.out.

@@ -148,6 +148,28 @@ MLA_DEVICE void tma_load_3d(void* dst, const CUtensorMap* map, int32_t x, int32_
       : "memory");
 }
 
+// TMA tiled store of a box from shared memory to global memory, tracked in this thread's
+// bulk groups. The box's generic-proxy writes must be fenced (fence_proxy_async_smem) and
+// complete (a barrier) before the store is issued.
+MLA_DEVICE void tma_store_3d(const CUtensorMap* map, const void* src, int32_t x, int32_t y,
+                             int32_t z) {
+  asm volatile("cp.async.bulk.tensor.3d.global.shared::cta.bulk_group [%0, {%2, %3, %4}], [%1];"
+               ::"l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(src)), "r"(x), "r"(y),
+               "r"(z)
+               : "memory");
+}
+MLA_DEVICE void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
+// Wait until at most N of this thread's committed bulk groups still read shared memory.
+template <int N>
+MLA_DEVICE void bulk_wait_read() {
+  asm volatile("cp.async.bulk.wait_group.read %0;" ::"n"(N) : "memory");
+}
+// Wait until at most N of this thread's committed bulk groups are still in flight.
+template <int N>
+MLA_DEVICE void bulk_wait() {
+  asm volatile("cp.async.bulk.wait_group %0;" ::"n"(N) : "memory");
+}
+
 // Bring a tile of a 2D tensor map into L2 (no shared-memory destination, no completion).
 MLA_DEVICE void tma_prefetch_l2_2d(const CUtensorMap* map, int32_t x, int32_t y) {
   asm volatile("cp.async.bulk.prefetch.tensor.2d.L2.global.tile [%0, {%1, %2}];" ::"l"(

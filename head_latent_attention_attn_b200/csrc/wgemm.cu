@@ -18,6 +18,7 @@
 // one of two TMEM accumulators, and warps 2-5 (one per TMEM sub-partition) drain the
 // other accumulator, so an item's epilogue overlaps the next item's loads and UMMAs. For
 // the absorb step the epilogue warps first write q_ext's rotary slots.
+#include "append.cuh"
 #include "decode_sched.cuh"
 #include "kernels.h"
 #include "ptx.cuh"
@@ -29,14 +30,19 @@ constexpr int kWgThreads = 192;        // warp 0 TMA, warp 1 UMMA, warps 2-5 epi
 constexpr int kWgEpiThreads = 128;
 constexpr int kWgABytes = 128 * 128;   // 128 x 64 bf16 weight tile (two 64x64 boxes for W_UK)
 
+// Shared memory: the TMA stages, 256 bytes of barriers, two epilogue staging tiles of
+// [NR rows][128 features] bf16, NR cache-row indices (fused append), 1 KB alignment slack.
 template <int NR>
 struct WgLayout {
   static constexpr int kB = NR * 128;                 // NR rows x 64 bf16
   static constexpr int kStage = kWgABytes + kB;
-  static constexpr int kFit = (192 * 1024) / kStage;
+  static constexpr int kEpi = NR * 128 * 2;           // one staging tile
+  static constexpr int kFit = (227 * 1024 - 256 - 2 * kEpi - NR * 8 - 1024) / kStage;
   static constexpr int kStages = kFit < 8 ? kFit : 8;
   static constexpr int kBars = kStage * kStages;      // barriers after the stages
-  static constexpr int kTotal = kBars + 256 + 1024;   // barriers + alignment slack
+  static constexpr int kEpiOff = kBars + 256;
+  static constexpr int kSlotOff = kEpiOff + 2 * kEpi;
+  static constexpr int kTotal = kSlotOff + NR * 8 + 1024;
 };
 
 MLA_DEVICE uint8_t* align1024(uint8_t* p) {
@@ -204,8 +210,9 @@ MLA_DEVICE void write_rope_slots(const WGemmParams& p, int tid, int nthreads) {
 // next call) and writes the rows. `last` is a shared-memory flag of the CTA.
 template <int NR>
 MLA_DEVICE void append_epilogue(const WGemmParams& p, const WgItem& w, int buf, uint32_t tmem,
-                                int sp, int lane, uint16_t* stage, uint64_t* acc_empty, bool ok,
-                                volatile int* abort_flag, volatile int* last) {
+                                int sp, int lane, uint16_t* stage, int64_t* slot_s,
+                                uint64_t* acc_empty, bool ok, volatile int* abort_flag,
+                                volatile int* last) {
   const int m_loc = sp * 32 + lane;
   const int nrows = min(NR, p.rows - w.n0);
   const int D = p.lat_r + p.groups * p.rope_dim;
@@ -273,7 +280,6 @@ MLA_DEVICE void append_epilogue(const WGemmParams& p, const WgItem& w, int buf, 
   }
   const int tid = m_loc;                          // 0..127
   // the cache row of every token of the tile, looked up once (two dependent loads each)
-  int64_t* slot_s = reinterpret_cast<int64_t*>(stage + NR * 128);
   if (tid < nrows) {
     const int64_t slot = append_slot(p, w.n0 + tid);
     if (slot < 0 && p.dev_error) atomicOr(p.dev_error, MLA_DEVERR_BOUNDS);
@@ -320,19 +326,21 @@ MLA_DEVICE void append_epilogue(const WGemmParams& p, const WgItem& w, int buf, 
 
 // Epilogue of absorb / out_up for one item, run by the four epilogue warps: the
 // accumulator (output feature m0 + lane of each TMEM lane, one column per activation row)
-// plus the bias is rounded to bf16 into a [NR rows][128 features] staging tile, the
-// accumulator is handed back, and the tile is written out row by row, so that consecutive
-// threads write consecutive 16-byte pieces of an output row (the rows of one item are
-// out_row_stride apart). All four warps pass both named barriers whatever their
+// plus the bias is rounded to bf16 into a [NR rows][128 features] staging tile (two
+// tiles, used by alternate items), the accumulator is handed back, and one thread stores
+// the tile with the TMA (rows out_row_stride apart, columns past M and rows past `rows`
+// clipped). Before a tile is written again the store that read it two items earlier has
+// finished reading it (bulk_wait_read<1> after each store, then the closing barrier).
+// Without the tensor map (strides that are no multiple of 16 bytes) the threads copy the
+// tile element by element. All four warps pass both named barriers whatever their
 // accumulator wait returned (`ok`); a failed wait leaves the CTA's abort flag set, and
-// then no warp writes the tile.
+// then the tile is not written.
 template <int NR>
 MLA_DEVICE void plain_epilogue(const WGemmParams& p, const WgItem& w, int buf, uint32_t tmem,
                                int sp, int lane, uint16_t* stage, uint64_t* acc_empty, bool ok,
                                volatile int* abort_flag) {
   const int m_loc = sp * 32 + lane;
   const int m = w.m0 + m_loc;                  // output feature of this thread's TMEM lane
-  const int nrows = min(NR, p.rows - w.n0);
   if (ok) {
     const float bias = (p.bias != nullptr && m < p.M)
                            ? bf16_bits_to_f32(p.bias[int64_t(w.h) * p.M + m]) : 0.0f;
@@ -344,31 +352,34 @@ MLA_DEVICE void plain_epilogue(const WGemmParams& p, const WgItem& w, int buf, u
       tmem_ld16(tmem + (uint32_t(sp * 32) << 16) + uint32_t(buf * NR + c0), v);
       tmem_wait_ld();
 #pragma unroll
-      for (int j = 0; j < 16; ++j) stage[(c0 + j) * 128 + m_loc] = f32_to_bf16_rne(v[j] + bias);
+      for (int j = 0; j < 16; ++j) stage[(c0 + j) * 128 + m_loc] = cvt_bf16(v[j] + bias);
     }
   }
   tc_fence_before();
   __syncwarp();
   if (lane == 0) mbar_arrive(acc_empty);
+  if (p.tma_out != 0) {
+    fence_proxy_async_smem();                  // the tile's writes, seen by the TMA
+    named_bar_sync(1, kWgEpiThreads);          // the staging tile is complete
+    if (m_loc == 0) {
+      if (*abort_flag == 0) {
+        tma_store_3d(&p.tm_out, stage, w.m0, w.h, w.n0);
+        bulk_commit();
+      }
+      bulk_wait_read<1>();                     // the other tile's store has read it
+    }
+    named_bar_sync(1, kWgEpiThreads);
+    return;
+  }
   named_bar_sync(1, kWgEpiThreads);            // the staging tile is complete
   if (*abort_flag == 0) {
+    const int nrows = min(NR, p.rows - w.n0);
     const int mt = min(128, p.M - w.m0);       // features of this tile
     uint16_t* out = p.out + int64_t(w.n0) * p.out_row_stride + int64_t(w.h) * p.out_head_stride +
                     w.m0;
-    if (p.vec_out != 0) {
-      // host-checked: M, both strides and the base are multiples of 8 elements
-      const int cpr = mt >> 3;                 // 16-byte pieces per row
-#pragma unroll 4
-      for (int idx = m_loc; idx < nrows * cpr; idx += kWgEpiThreads) {
-        const int n = idx / cpr, c = idx - (idx / cpr) * cpr;
-        *reinterpret_cast<uint4*>(out + int64_t(n) * p.out_row_stride + c * 8) =
-            *reinterpret_cast<const uint4*>(stage + n * 128 + c * 8);
-      }
-    } else {
-      for (int idx = m_loc; idx < nrows * mt; idx += kWgEpiThreads) {
-        const int n = idx / mt, c = idx - (idx / mt) * mt;
-        out[int64_t(n) * p.out_row_stride + c] = stage[n * 128 + c];
-      }
+    for (int idx = m_loc; idx < nrows * mt; idx += kWgEpiThreads) {
+      const int n = idx / mt, c = idx - (idx / mt) * mt;
+      out[int64_t(n) * p.out_row_stride + c] = stage[n * 128 + c];
     }
   }
   named_bar_sync(1, kWgEpiThreads);            // the staging tile may be reused
@@ -427,6 +438,7 @@ __global__ void __launch_bounds__(kWgThreads, 1) wgemm_kernel(const __grid_const
     if (elect_one()) {
       prefetch_tensormap(&p.tm_w);
       prefetch_tensormap(&p.tm_x);
+      if (p.tma_out) prefetch_tensormap(&p.tm_out);
       // The weights are no kernel's output here: warm L2 with this CTA's weight tiles while
       // the previous kernel may still run (an L2 prefetch is coherent with any writer).
       for (int it = blockIdx.x; it < items; it += gridDim.x) {
@@ -515,6 +527,12 @@ __global__ void __launch_bounds__(kWgThreads, 1) wgemm_kernel(const __grid_const
     grid_dep_wait();
     grid_dep_launch();
     const int sp = warp & 3;
+    {
+      // new tokens' cache rows (one warp per token) while the first accumulator fills
+      const int64_t ntok = int64_t(p.app.batch) * p.app.n_new;
+      for (int64_t gw = int64_t(blockIdx.x) * 4 + (warp - 2); gw < ntok; gw += int64_t(gridDim.x) * 4)
+        append_token(p.app, gw, lane);
+    }
     if (p.q_pe != nullptr && p.rope_dim > 0)
       write_rope_slots(p, int(blockIdx.x) * kWgEpiThreads + int(threadIdx.x) - 64,
                        int(gridDim.x) * kWgEpiThreads);
@@ -526,14 +544,17 @@ __global__ void __launch_bounds__(kWgThreads, 1) wgemm_kernel(const __grid_const
       tc_fence_after();
       if (append) {
         append_epilogue<NR>(p, w, buf, tmem, sp, lane,
-                            reinterpret_cast<uint16_t*>(base + Lay::kBars + 256), &acc_empty[buf],
+                            reinterpret_cast<uint16_t*>(base + Lay::kEpiOff),
+                            reinterpret_cast<int64_t*>(base + Lay::kSlotOff), &acc_empty[buf],
                             ok, abort_flag, last_flag);
         continue;
       }
       plain_epilogue<NR>(p, w, buf, tmem, sp, lane,
-                         reinterpret_cast<uint16_t*>(base + Lay::kBars + 256), &acc_empty[buf],
-                         ok, abort_flag);
+                         reinterpret_cast<uint16_t*>(base + Lay::kEpiOff + (li & 1) * Lay::kEpi),
+                         &acc_empty[buf], ok, abort_flag);
     }
+    // the last tiles' stores have written global memory before the CTA leaves
+    if (p.tma_out != 0 && sp == 0 && lane == 0) bulk_wait<0>();
   }
   tc_fence_before();
   __syncthreads();
@@ -543,9 +564,7 @@ __global__ void __launch_bounds__(kWgThreads, 1) wgemm_kernel(const __grid_const
 template <int NR>
 static cudaError_t launch_wgemm_nr(const WGemmParams& p, int max_ctas, cudaStream_t stream) {
   const bool append = p.cache != nullptr;
-  // the epilogue stages one [NR][128] bf16 tile after the barriers (the fused append also
-  // NR cache-row indices)
-  const int smem = WgLayout<NR>::kTotal + NR * 128 * 2 + (append ? NR * 8 : 0);
+  const int smem = WgLayout<NR>::kTotal;
   cudaError_t e = cudaFuncSetAttribute(wgemm_kernel<NR>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;

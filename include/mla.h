@@ -11,6 +11,7 @@
  *   mla_decode_attn   scores = q_pe.k_pe + q_c.c_kv, scaled, softmaxed;
  *                     o_ = einsum('bhql,blc->bhqc', attn, c_kv)   (einsum 4) and lse
  *   mla_out_up        o = einsum('bhqc,hdc->bhqd', o_, W_UV) (+ bias)  (einsum 5)
+ *   mla_decode_step   the four above in one call (the append folded into the absorption)
  *
  * Conventions shared by every call
  *   - Every data pointer is DEVICE memory owned by the caller; the library allocates
@@ -227,6 +228,43 @@ mla_status mla_decode_attn(const mla_dims* dims, const void* q_ext, const void* 
                            int32_t q_len, int32_t max_seq_len, int32_t causal,
                            int32_t num_splits, void* workspace, size_t workspace_bytes,
                            void* o_latent, float* lse, void* stream);
+
+/*
+ * mla_decode_step - one whole decode step in one call: mla_cache_append, mla_absorb_q,
+ * mla_decode_attn and mla_out_up on the same arguments, in that order (the absorbed
+ * order of the DeepSeek-V2 page's "Matrix absorption" section, einsums (4) and (5)).
+ * Every output is the one the four calls would produce, bit for bit. The append is
+ * folded into the absorption kernel (its rows are written while the first weight tiles
+ * arrive), so the step launches three kernels (four when the decode plan cuts sequences
+ * between CTAs and runs its merge).
+ *
+ *   c_kv_new, k_r_new, rope_cos_new, rope_sin_new, start_pos, n_new
+ *                              as mla_cache_append's c_kv, k_r, rope_cos, rope_sin,
+ *                              start_pos, n_new (n_new = 0: nothing appended)
+ *   q_nope, q_pe, rope_cos_q, rope_sin_q, w_uk, w_uk_head_stride
+ *                              as mla_absorb_q
+ *   w_uv, w_uv_head_stride, bias_v
+ *                              as mla_out_up
+ *   cache ... num_splits, workspace, workspace_bytes, o_latent, lse
+ *                              as mla_decode_attn
+ *   q_ext                      bf16 [B, q, H, D] scratch for the absorbed query (written)
+ *   o                          bf16 [B, q, H, d_v] output
+ * The append reports bounds faults into the workspace's device error word (its first
+ * int32), like the decode. Every argument is validated before anything is launched;
+ * the statuses are those of the four calls.
+ */
+mla_status mla_decode_step(const mla_dims* dims, const void* c_kv_new, const void* k_r_new,
+                           const float* rope_cos_new, const float* rope_sin_new,
+                           const int32_t* start_pos, int32_t n_new, const void* q_nope,
+                           const void* q_pe, const float* rope_cos_q, const float* rope_sin_q,
+                           const void* w_uk, int64_t w_uk_head_stride, const void* w_uv,
+                           int64_t w_uv_head_stride, const void* bias_v, void* cache,
+                           int64_t num_pages, const int32_t* block_table,
+                           int32_t max_pages_per_seq, const int32_t* seq_lens, int32_t batch,
+                           int32_t q_len, int32_t max_seq_len, int32_t causal,
+                           int32_t num_splits, void* q_ext, void* workspace,
+                           size_t workspace_bytes, void* o_latent, float* lse, void* o,
+                           void* stream);
 
 /*
  * mla_out_up - apply the value up-projection to the attention output (einsum 5 of the

@@ -100,6 +100,39 @@ def test_decode_validation(mla_lib):
     assert _decode(_dims(), batch=0) == mla.MLA_OK
 
 
+def _step(d, **kw):
+    a = dict(c_kv=FAKE, k_r=FAKE, cosn=FAKE, sinn=FAKE, start=FAKE, n=1, qn=FAKE, qpe=FAKE,
+             cosq=FAKE, sinq=FAKE, wuk=FAKE, wuks=128 * 512, wuv=FAKE, wuvs=128 * 512, bias=None,
+             cache=FAKE, npages=100, table=FAKE, maxp=4, lens=FAKE, batch=2, qlen=1, maxlen=256,
+             causal=1, splits=1, qext=FAKE, ws=P(0x10000), wsb=1 << 20, ol=FAKE, lse=FAKE, o=FAKE)
+    a.update(kw)
+    return mla.lib().mla_decode_step(
+        ctypes.byref(d), a["c_kv"], a["k_r"], a["cosn"], a["sinn"], a["start"], a["n"], a["qn"],
+        a["qpe"], a["cosq"], a["sinq"], a["wuk"], a["wuks"], a["wuv"], a["wuvs"], a["bias"],
+        a["cache"], a["npages"], a["table"], a["maxp"], a["lens"], a["batch"], a["qlen"],
+        a["maxlen"], a["causal"], a["splits"], a["qext"], a["ws"], a["wsb"], a["ol"], a["lse"],
+        a["o"], None)
+
+
+def test_decode_step_validation(mla_lib):
+    """The one-call step returns the status of the first of its four parts whose arguments
+    fail, before anything is launched (FAKE pointers are never dereferenced)."""
+    assert _step(_dims(num_kv_groups=3)) == mla.MLA_ERR_INVALID_ARG
+    assert _step(_dims(), c_kv=None) == mla.MLA_ERR_INVALID_ARG               # append
+    assert _step(_dims(), npages=0) == mla.MLA_ERR_INVALID_ARG
+    assert _step(_dims(), qn=None) == mla.MLA_ERR_INVALID_ARG                 # absorb
+    assert _step(_dims(), wuks=128 * 512 - 8) == mla.MLA_ERR_INVALID_ARG
+    assert _step(_dims(), qext=P(0x10008)) == mla.MLA_ERR_INVALID_ARG
+    assert _step(_dims(page_size=32)) == mla.MLA_ERR_UNSUPPORTED              # decode plan
+    assert _step(_dims(), causal=2) == mla.MLA_ERR_INVALID_ARG                # decode
+    assert _step(_dims(), lens=None) == mla.MLA_ERR_INVALID_ARG
+    assert _step(_dims(), ws=None) == mla.MLA_ERR_WORKSPACE
+    assert _step(_dims(), splits=4, wsb=4096) == mla.MLA_ERR_WORKSPACE
+    assert _step(_dims(), wuv=None) == mla.MLA_ERR_INVALID_ARG                # out_up
+    assert _step(_dims(), o=P(0x10008)) == mla.MLA_ERR_INVALID_ARG
+    assert _step(_dims(), batch=0) == mla.MLA_OK                              # nothing to do
+
+
 def test_workspace_size(mla_lib):
     a256 = lambda x: (x + 255) // 256 * 256  # noqa: E731
     # 128 heads, q = 1: one block of 128 query rows per sequence on a cluster of two CTAs

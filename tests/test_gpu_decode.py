@@ -128,3 +128,55 @@ def test_length_beyond_plan_is_flagged():
     assert mla.mla_get_device_status(prob.workspace.view(torch.int32)[:1], reset=True) == \
         mla.MLA_ERR_DEVICE_BOUNDS
     check_sequence(prob, 1, "bad length, seq 1")
+
+
+@pytest.mark.parametrize("name", ["deepseek_v2", "qwen3_30b_a3b", "qwen25_7b_q4", "deepseek_v2_bias"])
+def test_one_call_step_equals_four_calls(name):
+    """mla_decode_step (the append folded into the absorption) writes the same cache rows and
+    the same q_ext, o_latent, lse and o, bit for bit, as the four separate calls."""
+    wl = make_workload(SMALL[name], spare_pages=3)
+    a = GpuProblem(wl)
+    b = GpuProblem(wl)
+    a.step()                                   # one call
+    mla.mla_cache_append(b.dims, b.c_new, b.k_new, b.cos_q, b.sin_q, b.block_table, b.start_pos,
+                         b.cache, dev_error=b.workspace.view(torch.int32)[:1])
+    mla.mla_absorb_q(b.dims, b.q_nope, b.q_pe, b.cos_q, b.sin_q, b.w_uk, b.q_ext)
+    mla.mla_decode_attn(b.dims, b.q_ext, b.cache, b.block_table, b.seq_lens, b.max_seq_len,
+                        b.workspace, b.o_latent, b.lse, causal=wl.cfg.causal)
+    mla.mla_out_up(b.dims, b.o_latent, b.w_uv, b.o, bias=b.bias)
+    torch.cuda.synchronize()
+    assert a.device_status() == mla.MLA_OK and b.device_status() == mla.MLA_OK
+    for t in ("q_ext", "o_latent", "lse", "o"):
+        assert torch.equal(getattr(a, t), getattr(b, t)), t
+    # cache rows: compare as bits (unused rows hold NaN in both)
+    assert torch.equal(a.cache.view(torch.int16), b.cache.view(torch.int16))
+
+
+@pytest.mark.parametrize("name,lens", [
+    ("deepseek_v2", [1700, 64, 64, 65, 130, 64, 64, 64]),      # one unit cut into many pieces
+    ("qwen3_30b_a3b", [900, 70, 64, 700, 64, 66, 64, 64]),
+])
+def test_skewed_cut_units(name, lens):
+    """Two ranges per unit on average with skewed lengths: units cut into 2..many pieces
+    (merged by the merge kernel), against the oracle and against a one-range-per-unit plan
+    (no cuts); a second call on the same workspace gives the same bits."""
+    cfg = shrink(CONFIGS[name], batch=len(lens), context=max(lens), name="skewed")
+    wl = make_workload(cfg, seq_lens=np.array(lens, dtype=np.int32))
+    prob = GpuProblem(wl, num_splits=2)
+    prob.step()
+    torch.cuda.synchronize()
+    assert prob.device_status() == mla.MLA_OK
+    for b in range(len(lens)):
+        check_sequence(prob, b, f"{name} skewed")
+    o2 = prob.o_latent.float().clone()
+    l2 = prob.lse.clone()
+    prob.decode_only(num_splits=2)          # same workspace again
+    torch.cuda.synchronize()
+    assert torch.equal(prob.o_latent.float(), o2) and torch.equal(prob.lse, l2)
+    ws1 = mla.mla_decode_workspace_size(prob.dims, cfg.batch, cfg.q_len, prob.max_seq_len, 1)
+    prob.workspace = torch.zeros(ws1, dtype=torch.uint8, device="cuda")
+    prob.decode_only(num_splits=1)
+    torch.cuda.synchronize()
+    err = (prob.o_latent.float() - o2).abs().max().item() / o2.abs().max().item()
+    assert err <= 2 ** -7, err
+    assert (prob.lse - l2).abs().max().item() <= 1e-5
