@@ -18,8 +18,10 @@
 // between CTAs leaves one normalised partial per piece (o in bf16, lse in fp32), merged
 // afterwards by mla_combine_kernel with the log-sum-exp identity.
 //
-// Roles (192 threads): warp 0 TMA producer, warp 1 UMMA issuer and TMEM owner, warps 2-5
-// softmax and epilogue. In the M=64 accumulator layout rows 16*sp..16*sp+15 sit in lanes
+// Roles (224 threads): warp 0 TMA producer, warp 1 S^T issuer and TMEM owner, warps 2-5
+// softmax and epilogue, warp 6 PV issuer. (Issued by one lane of a softmax warp, the 16
+// PV products of a page took ~2.5x their issue cost; a warp of their own issues them at
+// the rate the tensor core accepts them.) In the M=64 accumulator layout rows 16*sp..16*sp+15 sit in lanes
 // 32*sp..32*sp+15 of TMEM sub-partition sp; the 16x32bx2 load gives each of those 16
 // tokens to two threads, one per half of the NCOL columns.
 //
@@ -53,7 +55,7 @@ __device__ unsigned long long g_mla_trace[10 * kTraceTiles + 1];
 
 namespace {
 
-constexpr int kThreads = 192;
+constexpr int kThreads = 224;
 constexpr int kBlkBytes = kDecodeTok * 128;   // one 64 x 64 bf16 block, 8 KB
 constexpr float kLazyThreshold = 8.0f;        // log2 units
 // Initial reference max: finite, so a masked score (-inf) minus it is exactly -inf (weight
@@ -70,7 +72,7 @@ struct DecodeLayout {
 
 __host__ __device__ inline uint32_t round_up(uint32_t x, uint32_t a) { return (x + a - 1) / a * a; }
 
-__host__ __device__ constexpr int num_bars(int nslot) { return 2 * nslot + 8; }
+__host__ __device__ constexpr int num_bars(int nslot) { return 2 * nslot + 10; }
 
 __host__ __device__ inline DecodeLayout decode_layout(int ncol, int nblk, int slot_blocks,
                                                       int nslot, int npt) {
@@ -188,6 +190,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t* s_full = q_empty + 1;                      // [2]
   uint64_t* s_free = s_full + 2;                       // [2]
   uint64_t* pv_done = s_free + 2;                      // [2]
+  uint64_t* p_full = pv_done + 2;                      // [npt] P^T written (4 softmax warps)
 
   constexpr uint32_t kPtBytes = ((kDecodeTok * NCOL * 2) + 1023) / 1024 * 1024;
   constexpr uint32_t kQBlk = NCOL * 128;
@@ -210,6 +213,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&s_full[i], 1);
       mbar_init(&s_free[i], 4);
       mbar_init(&pv_done[i], 1);
+      mbar_init(&p_full[i], 4);
     }
     *abort_flag = 0;
     fence_mbar_init();
@@ -326,8 +330,54 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
     }
     __syncwarp();
-  } else if (has_work) {
-    // ============================ softmax, PV issue, epilogue ============================
+  } else if (warp == 6) {
+    // =============================== UMMA issuer for PV ==================================
+    // O^T += C^T P^T for page j once the four softmax warps have written P^T(j) and zeroed
+    // the page's rows past the context; the first page of a piece overwrites O^T (the
+    // softmax warps read the previous piece's O^T before they arrive on P^T's barrier).
+    if (has_work && elect_one()) {
+      const uint32_t idesc_o = make_idesc_bf16(128, NCOL, 1, 1);
+      const uint64_t pa0 = make_sdesc(smem_u32(slots), kBlkBytes, 1024, kSw128);
+      const uint64_t pb0 = make_sdesc(smem_u32(pt), kPtBytes, 8 * NCOL * 2, pt_swizzle(NCOL));
+      UnitWalk w{sched[0], sched[1]};
+      int jj = 0;
+      SlotRing ring(p.nslot), pring(p.npt);
+      bool ok = true;
+      for (; ok && w.s < r1; w.s += w.tiles, ++w.b) {
+        w.load(p, cg);
+        const int tb = max(w.s, r0), te = min(w.s + w.tiles, r1);
+        for (int t = tb; t < te; ++t, ++jj, ring.next(), pring.next()) {
+          if (!mbar_wait(&p_full[pring.slot], pring.round & 1, wc)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          MLA_TRACE_AT(7, jj);
+          const bool first = (t == tb);
+          // K-step outer, latent chunk inner: consecutive MMAs feed different accumulators;
+          // descriptors stepped (16 tokens = 2 KB of C^T, 16 rows of P^T; 128 latent = 2
+          // blocks)
+          const uint64_t ad0 = pa0 + ((ring.slot * slot_bytes) >> 4);
+          uint64_t bd = pb0 + ((pring.slot * kPtBytes) >> 4);
+#pragma unroll
+          for (int kk = 0; kk < 4; ++kk) {
+            uint64_t ad = ad0 + uint64_t(kk * (2048 >> 4));
+            const uint32_t acc = (!first || kk > 0) ? 1u : 0u;
+            for (int c = 0; c < p.nch; ++c) {
+              umma_bf16(tmem + (2 + c) * NCOL, ad, bd, idesc_o, acc);
+              ad += uint64_t((2 * kBlkBytes) >> 4);
+            }
+            bd += uint64_t((16 * NCOL * 2) >> 4);
+          }
+          umma_commit(&pv_done[jj & 1]);
+          umma_commit(&empty[ring.slot]);
+          MLA_TRACE_AT(3, jj);
+        }
+      }
+    }
+    __syncwarp();
+  } else if (has_work) {   // warps 2-5
+    // ================================ softmax, epilogue ==================================
     const int sp = warp & 3;                  // TMEM sub-partition this warp may access
     const int wi = warp - 2;                  // index among the 4 softmax warps
     const int tid = threadIdx.x - 64;         // 0..127
@@ -337,10 +387,6 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int c0 = hf * HALF;                 // first column of this thread
     const bool col_owner = (lane & 15) == 0;  // publishes its half-warp's column values
     const float c_log2 = p.scale_log2;
-    // PV operands: C^T of the tile (MN-major) and P^T (MN-major), advanced by offsets
-    const uint32_t idesc_o = make_idesc_bf16(128, NCOL, 1, 1);
-    const uint64_t pa0 = make_sdesc(smem_u32(slots), kBlkBytes, 1024, kSw128);
-    const uint64_t pb0 = make_sdesc(smem_u32(pt), kPtBytes, 8 * NCOL * 2, pt_swizzle(NCOL));
 
     UnitWalk w{sched[0], sched[1]};
     int jj = 0;
@@ -496,37 +542,11 @@ __global__ void __launch_bounds__(kThreads, 1)
             for (int ch = 0; ch < 8; ++ch) rowp[ch] = make_uint4(0, 0, 0, 0);
           }
         }
+        // P^T(j) and the zeroed rows are complete: hand the page to the PV issuer
         fence_proxy_async_smem();
         tc_fence_before();
-        named_bar_sync(1, 128);
-        if (threadIdx.x == 64) {
-          // O^T += C^T P^T for this tile; the first tile of a piece overwrites O^T (the
-          // previous piece's epilogue reads finished before the barrier above)
-          MLA_TRACE_AT(7, jj);
-          tc_fence_after();
-          const bool first = (t == tb);
-          const uint32_t soff = slot * slot_bytes;
-          const uint32_t poff = pbuf * kPtBytes;
-          // K-step outer, latent chunk inner: consecutive MMAs feed different accumulators;
-          // descriptors stepped (16 tokens = 2 KB of C^T, 16 rows of P^T; 128 latent = 2 blocks)
-          {
-            const uint64_t ad0 = pa0 + (soff >> 4);
-            uint64_t bd = pb0 + (poff >> 4);
-#pragma unroll
-            for (int kk = 0; kk < 4; ++kk) {
-              uint64_t ad = ad0 + uint64_t(kk * (2048 >> 4));
-              const uint32_t acc = (!first || kk > 0) ? 1u : 0u;
-              for (int c = 0; c < p.nch; ++c) {
-                umma_bf16(tmem + (2 + c) * NCOL, ad, bd, idesc_o, acc);
-                ad += uint64_t((2 * kBlkBytes) >> 4);
-              }
-              bd += uint64_t((16 * NCOL * 2) >> 4);
-            }
-          }
-          umma_commit(&pv_done[jj & 1]);
-          umma_commit(&empty[slot]);
-          MLA_TRACE_AT(3, jj);
-        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&p_full[pbuf]);
       }
 
       // ---------------------------- epilogue of this piece --------------------------------
