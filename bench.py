@@ -243,12 +243,18 @@ def decode_kernel_name(cfg):
 
 
 def _source_hash(cfg):
-    """Hash of the sources of the decode kernel that runs this shape."""
-    files = ("decode_pair.cu" if uses_pair_kernel(cfg) else "decode.cu",
-             "decode_sched.cuh", "ptx.cuh", "kernels.h")
+    """Hash of the sources of the decode kernel that runs this shape: its .cu file, the
+    schedule and PTX helpers, and its parameter struct (the rest of kernels.h belongs to the
+    other kernels)."""
+    csrc = os.path.join(ROOT, "head_latent_attention_attn_b200", "csrc")
+    files = ("decode_pair.cu" if uses_pair_kernel(cfg) else "decode.cu", "decode_sched.cuh",
+             "ptx.cuh")
     h = hashlib.sha256()
     for f in files:
-        h.update(open(os.path.join(ROOT, "head_latent_attention_attn_b200", "csrc", f), "rb").read())
+        h.update(open(os.path.join(csrc, f), "rb").read())
+    hdr = open(os.path.join(csrc, "kernels.h")).read()
+    i = hdr.index("struct DecodeParams {")
+    h.update(hdr[i:hdr.index("};", i)].encode())
     return h.hexdigest()[:16]
 
 
@@ -576,8 +582,10 @@ def per_config_block(args, head_cfg, dev, stream, dist, peaks):
     from mla_inputs import CONFIGS, make_down_kv_inputs, make_o_proj_inputs, make_workload
     from mla_inputs.device import DeviceProblem
     out = {}
+    only = {x.strip() for x in args.per_config.split(",") if x.strip()}
+    want = (lambda key: not only or key in only)
     for name in PER_CONFIG:
-        if name == head_cfg.name:
+        if name == head_cfg.name or not want(name):
             continue
         cfg = CONFIGS[name]
         kv = name.startswith("nanowhale")
@@ -605,7 +613,7 @@ def per_config_block(args, head_cfg, dev, stream, dist, peaks):
         del prob, flush, wl
         torch.cuda.empty_cache()
     # einsums (5) and (6) fused (mla_out_proj) at the DeepSeek-V2 decode batch
-    for name in OUT_PROJ:
+    for name in (OUT_PROJ if want("out_proj") else ()):
         cfg = CONFIGS[name]
         rows = cfg.batch * cfg.q_len
         dims = mla.make_dims(cfg.num_heads, cfg.num_kv_groups, cfg.kv_lora_rank, cfg.qk_nope_dim,
@@ -644,19 +652,17 @@ def per_config_block(args, head_cfg, dev, stream, dist, peaks):
             "l2": "L2 flushed between launches", "clocks": clk.summary()}
         del o_lat, w_uv, w_o, o, u, ws, flush
         torch.cuda.empty_cache()
-    for name in DOWN_KV:
+    for name in (DOWN_KV if want("down_kv") else ()):
         cfg = CONFIGS[name]
         wl = make_workload(cfg.with_(context=128, lens_range=None))
         prob = DeviceProblem(wl, device=str(dev))
         hidden, w_dkv = make_down_kv_inputs(cfg, cfg.q_len)
         hidden, w_dkv = hidden.to(dev), w_dkv.to(dev)
         flush = torch.empty(4 * L2_BYTES // 4, dtype=torch.float32, device=dev)
-        ws = torch.zeros(mla.mla_down_kv_workspace_size(prob.dims, cfg.batch, cfg.q_len),
-                         dtype=torch.uint8, device=dev)
 
-        def call(stream, prob=prob, hidden=hidden, w_dkv=w_dkv, ws=ws):
+        def call(stream, prob=prob, hidden=hidden, w_dkv=w_dkv):
             mla.mla_down_kv_append(prob.dims, hidden, w_dkv, prob.cos_q, prob.sin_q,
-                                   prob.block_table, prob.start_pos, prob.cache, ws,
+                                   prob.block_table, prob.start_pos, prob.cache,
                                    dev_error=prob.err, stream=stream)
         time_calls(call, 3, stream, flush)
         with ClockSampler(_gpu_id(dev.index or 0)) as clk:
@@ -674,9 +680,9 @@ def per_config_block(args, head_cfg, dev, stream, dist, peaks):
             "roofline": {"bound": "hbm", "achieved": gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
                          "frac": gbs / peaks["hbm_gbs"], "algorithmic_bytes_per_launch": nbytes,
                          "algorithmic_flops_per_launch": flops, "peak_source": peaks["source"],
-                         "kernel": "wgemm_kernel (fused cache-append epilogue)"},
+                         "kernel": "down_kv_kernel (split-K on clusters, cache-append epilogue)"},
             "l2": "L2 flushed between launches", "clocks": clk.summary()}
-        del prob, flush, hidden, w_dkv, wl, ws
+        del prob, flush, hidden, w_dkv, wl
         torch.cuda.empty_cache()
     return out
 
@@ -702,6 +708,9 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-per-config", action="store_true",
                     help="time only the headline workload")
+    ap.add_argument("--per-config", default="",
+                    help="comma-separated subset of the per-config entries to time (workload "
+                         "names, 'out_proj', 'down_kv'); default all")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
 

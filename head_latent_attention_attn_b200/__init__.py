@@ -36,7 +36,7 @@ C_SYMBOLS = ("mla_row_width", "mla_status_string", "mla_cache_append", "mla_abso
              "mla_decode_workspace_size", "mla_decode_attn", "mla_out_up",
              "mla_get_device_status", "mla_decode_attn_noalloc", "mla_selftest_wait_timeout",
              "mla_kv_shared_decode_dims", "mla_kv_shared_query", "mla_kv_shared_output",
-             "mla_down_kv_workspace_size", "mla_down_kv_append", "mla_out_proj_workspace_size",
+             "mla_down_kv_append", "mla_out_proj_workspace_size",
              "mla_out_proj", "mla_decode_step")
 
 
@@ -106,10 +106,8 @@ def lib() -> ctypes.CDLL:
     for fn in (L.mla_kv_shared_query, L.mla_kv_shared_output):
         fn.argtypes = [D, _P, _P, _P, _I32, _I32, _P, _P]
         fn.restype = _I32
-    L.mla_down_kv_workspace_size.argtypes = [D, _I32, _I32]
-    L.mla_down_kv_workspace_size.restype = ctypes.c_size_t
     L.mla_down_kv_append.argtypes = [D, _P, _I32, _P, _P, _P, _P, _I32, _P, _I32, _I32, _P,
-                                     _I64, _P, _P, _P, ctypes.c_size_t, _P]
+                                     _I64, _P, _P, _P]
     L.mla_down_kv_append.restype = _I32
     L.mla_out_proj_workspace_size.argtypes = [D, _I32, _I32]
     L.mla_out_proj_workspace_size.restype = ctypes.c_size_t
@@ -186,17 +184,11 @@ def mla_cache_append(dims: MlaDims, c_kv, k_r, rope_cos, rope_sin, block_table, 
     _check(st, "mla_cache_append")
 
 
-def mla_down_kv_workspace_size(dims: MlaDims, batch: int, n_new: int) -> int:
-    return int(lib().mla_down_kv_workspace_size(ctypes.byref(dims), int(batch), int(n_new)))
-
-
 def mla_down_kv_append(dims: MlaDims, hidden, w_dkv, rope_cos, rope_sin, block_table,
-                       start_pos, cache, workspace, dev_error=None, kv_out=None,
-                       stream=None) -> None:
+                       start_pos, cache, dev_error=None, kv_out=None, stream=None) -> None:
     """[c_kv ; k_r] = w_dkv @ hidden (bf16) for hidden [B, n, hidden_dim], written into cache
     [P, ps, D] exactly as mla_cache_append would; kv_out [B, n, D] optionally receives the
-    projection before the rotation; workspace is a zeroed uint8 CUDA tensor of
-    mla_down_kv_workspace_size bytes (left zero by the call)."""
+    projection before the rotation."""
     B, n, hid = hidden.shape
     G, dr, D = dims.num_kv_groups, dims.rope_dim, dims.row_width
     _need(hidden, "hidden", torch.bfloat16)
@@ -215,13 +207,12 @@ def mla_down_kv_append(dims: MlaDims, hidden, w_dkv, rope_cos, rope_sin, block_t
         _need(dev_error, "dev_error", torch.int32)
     if kv_out is not None:
         _need(kv_out, "kv_out", torch.bfloat16, (B, n, D))
-    _need(workspace, "workspace", torch.uint8)
     st = lib().mla_down_kv_append(ctypes.byref(dims), _ptr(hidden), hid, _ptr(w_dkv),
                                   _ptr(rope_cos if dr > 0 else None),
                                   _ptr(rope_sin if dr > 0 else None), _ptr(block_table),
                                   block_table.shape[1], _ptr(start_pos), B, n, _ptr(cache),
-                                  cache.shape[0], _ptr(dev_error), _ptr(kv_out), _ptr(workspace),
-                                  workspace.numel(), _stream(stream))
+                                  cache.shape[0], _ptr(dev_error), _ptr(kv_out),
+                                  _stream(stream))
     _check(st, "mla_down_kv_append")
 
 
@@ -475,6 +466,6 @@ def mla_decode_step(dims: MlaDims, *, c_kv_new, k_r_new, cos_new, sin_new, start
 __all__ = ["MlaDims", "MlaError", "make_dims", "lib", "mla_row_width", "mla_cache_append",
            "mla_absorb_q", "mla_decode_workspace_size", "mla_decode_attn", "mla_out_up",
            "mla_decode_attn_noalloc", "mla_kv_shared_decode_dims", "mla_kv_shared_query",
-           "mla_kv_shared_output", "mla_down_kv_workspace_size", "mla_down_kv_append",
+           "mla_kv_shared_output", "mla_down_kv_append",
            "mla_out_proj_workspace_size",
            "mla_out_proj", "mla_get_device_status", "mla_decode_step", "C_SYMBOLS", "STATUS_NAMES"]

@@ -18,7 +18,7 @@ CSRC = os.path.join(PKG, "csrc")
 OBJ = os.path.join(ROOT, "_build", "mla")
 LIB = os.path.join(PKG, "libmla.so")
 SOURCES = ["host_common.cu", "api.cu", "append.cu", "wgemm.cu", "decode.cu", "decode_pair.cu",
-           "noalloc.cu", "kv_shared.cu", "oproj.cu"]
+           "noalloc.cu", "kv_shared.cu", "oproj.cu", "down_kv.cu", "combine.cu"]
 HEADERS = ["ptx.cuh", "kernels.h", "host_common.h", "decode_sched.cuh", "append.cuh"]
 
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]

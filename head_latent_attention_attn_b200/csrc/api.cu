@@ -293,7 +293,6 @@ mla_status build_absorb(const mla_dims* dims, const void* q_nope, const void* q_
   p.rows = int32_t(rows);
   p.heads = H;
   p.a_mn = 1;
-  p.splits = 1;
   p.q_pe = dims->rope_dim > 0 ? static_cast<const uint16_t*>(q_pe) : nullptr;
   p.rope_cos = rope_cos;
   p.rope_sin = rope_sin;
@@ -348,7 +347,6 @@ mla_status build_out_up(const mla_dims* dims, const void* o_latent, const void* 
   p.rows = rows;
   p.heads = H;
   p.a_mn = 0;
-  p.splits = 1;
   p.q_pe = nullptr;
   p.tma_out = encode_out_map(p, p.out, nr);
   *nr_out = nr;
@@ -398,24 +396,11 @@ mla_status mla_out_up(const mla_dims* dims, const void* o_latent, const void* w_
   return launch_wgemm(p, nr, num_sms(), as_stream(stream)) == cudaSuccess ? MLA_OK : MLA_ERR_CUDA;
 }
 
-// Workspace of mla_down_kv_append: fp32 sums of the split K ([rows, D]) and one counter per
-// output tile (at most ceil(r/128) + 1 feature tiles per 16-row tile).
-static size_t down_kv_ws(const mla_dims* d, int64_t rows) {
-  const int64_t tiles = (int64_t(d->kv_lora_rank + 127) / 128 + 1) * ((rows + 15) / 16);
-  return (size_t(tiles) * 4 + 255) / 256 * 256 + size_t(rows) * size_t(row_width(d)) * 4;
-}
-
-size_t mla_down_kv_workspace_size(const mla_dims* dims, int32_t batch, int32_t n_new) {
-  if (check_dims(dims) != MLA_OK || batch < 0 || n_new < 0) return 0;
-  return down_kv_ws(dims, int64_t(batch) * n_new);
-}
-
 mla_status mla_down_kv_append(const mla_dims* dims, const void* hidden, int32_t hidden_dim,
                               const void* w_dkv, const float* rope_cos, const float* rope_sin,
                               const int32_t* block_table, int32_t max_pages_per_seq,
                               const int32_t* start_pos, int32_t batch, int32_t n_new, void* cache,
-                              int64_t num_pages, int32_t* dev_error, void* kv_out,
-                              void* workspace, size_t workspace_bytes, void* stream) {
+                              int64_t num_pages, int32_t* dev_error, void* kv_out, void* stream) {
   mla_status st = check_dims(dims);
   if (st != MLA_OK) return st;
   if (batch < 0 || n_new < 0 || hidden_dim <= 0 || hidden_dim % 8 != 0 ||
@@ -430,60 +415,49 @@ mla_status mla_down_kv_append(const mla_dims* dims, const void* hidden, int32_t 
     return MLA_ERR_INVALID_ARG;
   if (R > 128) return MLA_ERR_UNSUPPORTED;        // the rotary features share one tile
   const int64_t rows = int64_t(batch) * n_new;
-  if (rows > int64_t(65535) * 128) return MLA_ERR_UNSUPPORTED;
-  if (!workspace || !aligned(workspace, 256) || workspace_bytes < down_kv_ws(dims, rows))
-    return MLA_ERR_WORKSPACE;
+  if (rows > INT32_MAX) return MLA_ERR_UNSUPPORTED;
   const int D = row_width(dims);
-  WGemmParams p{};
-  {
-    const uint64_t dims3[3] = {uint64_t(hidden_dim), uint64_t(D), 1};
-    const uint64_t str[2] = {uint64_t(hidden_dim) * 2, uint64_t(D) * hidden_dim * 2};
-    const uint32_t box[3] = {64, 128, 1};
-    if (!encode_bf16_map(&p.tm_w, w_dkv, 3, dims3, str, box, CU_TENSOR_MAP_SWIZZLE_128B))
-      return MLA_ERR_CUDA;
-  }
   const int nr = pick_nr(rows);
+  DkvParams p{};
   {
-    const uint64_t dims3[3] = {uint64_t(hidden_dim), 1, uint64_t(rows)};
-    const uint64_t str[2] = {uint64_t(hidden_dim) * 2, uint64_t(hidden_dim) * 2};
-    const uint32_t box[3] = {64, 1, uint32_t(nr)};
-    if (!encode_bf16_map(&p.tm_x, hidden, 3, dims3, str, box, CU_TENSOR_MAP_SWIZZLE_128B))
+    const uint64_t d2[2] = {uint64_t(hidden_dim), uint64_t(D)};
+    const uint64_t s2[1] = {uint64_t(hidden_dim) * 2};
+    const uint32_t box[2] = {64, 128};
+    if (!encode_bf16_map(&p.tm_w, w_dkv, 2, d2, s2, box, CU_TENSOR_MAP_SWIZZLE_128B))
       return MLA_ERR_CUDA;
   }
-  p.out = nullptr;
-  p.bias = nullptr;
-  p.dev_error = dev_error;
-  p.M = D;
-  p.K = hidden_dim;
-  p.rows = int32_t(rows);
-  p.heads = 1;
-  p.a_mn = 0;
-  p.q_pe = nullptr;
-  p.rope_cos = rope_cos;
-  p.rope_sin = rope_sin;
-  p.groups = dims->num_kv_groups;
-  p.rope_dim = dims->rope_dim;
+  {
+    const uint64_t d2[2] = {uint64_t(hidden_dim), uint64_t(rows)};
+    const uint64_t s2[1] = {uint64_t(hidden_dim) * 2};
+    const uint32_t box[2] = {64, uint32_t(nr)};
+    if (!encode_bf16_map(&p.tm_x, hidden, 2, d2, s2, box, CU_TENSOR_MAP_SWIZZLE_128B))
+      return MLA_ERR_CUDA;
+  }
   p.cache = static_cast<uint16_t*>(cache);
   p.block_table = block_table;
   p.start_pos = start_pos;
+  p.rope_cos = rope_cos;
+  p.rope_sin = rope_sin;
   p.kv_out = static_cast<uint16_t*>(kv_out);
+  p.dev_error = dev_error;
   p.num_pages = num_pages;
   p.max_pages = max_pages_per_seq;
   p.n_new = n_new;
   p.page_size = dims->page_size;
-  p.lat_r = r;
+  p.r = r;
+  p.groups = dims->num_kv_groups;
+  p.rope_dim = dims->rope_dim;
+  p.rows = int32_t(rows);
+  p.K = hidden_dim;
   p.lat_tiles = (r + 127) / 128;
-  // K (the model width) split so that the (feature tile, split, row tile) items fill the GPU
-  const int n_mt = p.lat_tiles + (R > 0 ? 1 : 0);
-  const int64_t n_nt = (rows + nr - 1) / nr;
+  p.n_nt = int32_t((rows + nr - 1) / nr);
+  // the model width split across a cluster of up to 16 CTAs (the launcher lowers it to what
+  // the device can co-schedule), at least 2 K blocks of 64 each
   const int nk = (hidden_dim + 63) / 64;
-  // (at least 8 K blocks of 64 per split: fewer, longer items than one per SM)
-  p.splits = int(std::max<int64_t>(1, std::min<int64_t>(nk / 8, num_sms() / (n_mt * n_nt))));
-  const int64_t tiles = int64_t(n_mt) * n_nt;
-  p.tile_done = static_cast<int32_t*>(workspace);
-  p.acc = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) +
-                                   (size_t(tiles) * 4 + 255) / 256 * 256);
-  return launch_wgemm(p, nr, num_sms(), as_stream(stream)) == cudaSuccess ? MLA_OK : MLA_ERR_CUDA;
+  p.splits = std::max(1, std::min(16, nk / 2));
+  if (int64_t(p.lat_tiles + (R > 0 ? 1 : 0)) * p.n_nt * p.splits > (int64_t(1) << 31) - 1)
+    return MLA_ERR_UNSUPPORTED;
+  return launch_down_kv(p, nr, as_stream(stream)) == cudaSuccess ? MLA_OK : MLA_ERR_CUDA;
 }
 
 }  // extern "C"
@@ -712,6 +686,7 @@ mla_status launch_decode_plan(const DecodePlan& P, const DecodeParams& p, cudaSt
     c.col_groups = P.col_groups;
     c.units = P.units;
     c.vgrid = P.vgrid;
+    c.sms = num_sms();
     if (launch_combine(c, s) != cudaSuccess) return MLA_ERR_CUDA;
   }
   return MLA_OK;

@@ -1,5 +1,6 @@
 // decode.cu - mla_decode_attn on sm_100a for blocks of up to 64 query rows: paged,
-// split-KV absorbed attention over the latent cache, and the merge of the split pieces.
+// split-KV absorbed attention over the latent cache (the merge of split pieces is in
+// combine.cu).
 //
 // Formulation. Every query row (i, h) of a sequence scores the SAME cache rows, so the
 // CTA keeps a block of NCOL query rows resident and streams the cache pages once:
@@ -16,7 +17,7 @@
 // equal ranges, one per CTA, so ragged lengths balance. A CTA walks the units its range
 // touches; a unit it holds whole is written straight to o_latent / lse, a unit cut
 // between CTAs leaves one normalised partial per piece (o in bf16, lse in fp32), merged
-// afterwards by mla_combine_kernel with the log-sum-exp identity.
+// afterwards by the merge kernels of combine.cu with the log-sum-exp identity.
 //
 // Roles (224 threads): warp 0 TMA producer, warp 1 S^T issuer and TMEM owner, warps 2-5
 // softmax and epilogue, warp 6 PV issuer. (Issued by one lane of a softmax warp, the 16
@@ -29,6 +30,8 @@
 // it moves only when a score exceeds it by more than 8 (unnormalised weights stay <= 256);
 // then the tile max is reduced over the CTA and O^T and the running sums are rescaled.
 #include <math.h>
+
+#include <algorithm>
 
 #include "decode_sched.cuh"
 #include "kernels.h"
@@ -625,183 +628,6 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (warp == 1) tmem_dealloc(tmem, p.tmem_cols);
 }
 
-// ---- merge of cut units: lse = log sum_i e^{lse_i}, o = sum_i e^{lse_i - lse} o_i ------
-// One block per (unit, query row): warp 0 reduces the pieces' lse, then the 4 warps split
-// the pieces and every lane accumulates up to 16 latents (8 x lane + 256 k + 0..7: one
-// 16-byte load of a piece's bf16 row per k; two pieces' loads in flight per step); shared
-// memory adds the warps.
-__global__ void __launch_bounds__(128) mla_combine_kernel(const CombineParams p) {
-  __shared__ float part[4][512];
-  __shared__ float lse_s;
-  grid_dep_wait();
-  grid_dep_launch();
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int u = int(blockIdx.x / unsigned(p.ncol));
-  const int n = int(blockIdx.x % unsigned(p.ncol));
-  const int G = p.col_groups;
-  const int b = u / G, cg = u - b * G;
-  const int f = cg * p.ncol + n;
-  if (f >= p.qH) return;
-  int L = p.seq_lens[b];
-  const bool ok = L >= p.q_len && L <= p.max_seq_len && int64_t(L) <= int64_t(p.max_pages) * kDecodeTok;
-  if (!ok) L = 0;
-  const int tiles = L > 0 ? (L + kDecodeTok - 1) / kDecodeTok : 1;
-  const int per = *p.range_len;
-  const int s = p.unit_start[u];
-  const int i0 = s / per, i1 = (s + tiles - 1) / per;
-  if (i0 == i1) return;   // held whole by one CTA: already written
-  if (warp == 0) {
-    float mx = -INFINITY;
-    for (int i = i0 + lane; i <= i1; i += 32)
-      mx = fmaxf(mx, p.part_lse[int64_t(piece_slot(i, s, per, G, cg)) * p.ncol + n]);
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
-    float den = 0.0f;
-    for (int i = i0 + lane; i <= i1; i += 32) {
-      const float li = p.part_lse[int64_t(piece_slot(i, s, per, G, cg)) * p.ncol + n];
-      den += li == -INFINITY ? 0.0f : expf(li - mx);
-    }
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) den += __shfl_xor_sync(0xffffffffu, den, o);
-    if (lane == 0) lse_s = mx == -INFINITY ? -INFINITY : mx + logf(den);
-  }
-  __syncthreads();
-  const float lse = lse_s;
-  float acc[16];
-#pragma unroll
-  for (int j = 0; j < 16; ++j) acc[j] = 0.0f;
-  // latents 8 * lane + 256 * k + e of a piece's row: 16-byte aligned (r % 8 == 0)
-  auto add_piece = [&](int i) {
-    const int64_t sl = piece_slot(i, s, per, G, cg);
-    const float li = p.part_lse[sl * p.ncol + n];
-    const uint16_t* row = p.part_o + (sl * p.ncol + n) * p.r;
-    uint4 v[2];
-#pragma unroll
-    for (int k = 0; k < 2; ++k) {
-      const int lat = 8 * lane + 256 * k;
-      v[k] = (lat < p.r && li != -INFINITY) ? *reinterpret_cast<const uint4*>(row + lat)
-                                            : make_uint4(0u, 0u, 0u, 0u);
-    }
-    const float wgt = li == -INFINITY ? 0.0f : expf(li - lse);
-#pragma unroll
-    for (int k = 0; k < 2; ++k) {
-      const uint32_t w[4] = {v[k].x, v[k].y, v[k].z, v[k].w};
-#pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        acc[8 * k + 2 * e] += wgt * __uint_as_float(w[e] << 16);
-        acc[8 * k + 2 * e + 1] += wgt * __uint_as_float(w[e] & 0xFFFF0000u);
-      }
-    }
-  };
-  int i = i0 + warp;
-  for (; i + 4 <= i1; i += 8) {
-    add_piece(i);
-    add_piece(i + 4);
-  }
-  if (i <= i1) add_piece(i);
-#pragma unroll
-  for (int k = 0; k < 2; ++k) {
-    const int lat = 8 * lane + 256 * k;
-    if (lat < p.r) {
-#pragma unroll
-      for (int e = 0; e < 8; ++e) part[warp][lat + e] = acc[8 * k + e];
-    }
-  }
-  __syncthreads();
-  uint16_t* out = p.o_latent + (int64_t(b) * p.qH + f) * p.r;
-  for (int lat = threadIdx.x; lat < p.r; lat += 128)
-    out[lat] = f32_to_bf16_rne(part[0][lat] + part[1][lat] + part[2][lat] + part[3][lat]);
-  if (threadIdx.x == 0) p.lse[int64_t(b) * p.qH + f] = lse;
-}
-
-// The same merge with one warp per (unit, query row), four rows per block: for units cut
-// into a few pieces. Up to 32 pieces, lane i reads piece i0 + i's lse once and the maximum,
-// the sum and each piece's weight come from shuffles; more pieces take a loop over global
-// memory. Lanes own latents 4 * lane + 128 k + {0..3}: every load of a piece's bf16 row is
-// one 256-byte coalesced segment per warp.
-__global__ void __launch_bounds__(128) mla_combine_rows_kernel(const CombineParams p) {
-  grid_dep_wait();
-  grid_dep_launch();
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int64_t gw = int64_t(blockIdx.x) * 4 + warp;
-  if (gw >= int64_t(p.units) * p.ncol) return;
-  const int u = int(gw / p.ncol);
-  const int n = int(gw - int64_t(u) * p.ncol);
-  const int G = p.col_groups;
-  const int b = u / G, cg = u - b * G;
-  const int f = cg * p.ncol + n;
-  if (f >= p.qH) return;
-  int L = p.seq_lens[b];
-  const bool ok = L >= p.q_len && L <= p.max_seq_len && int64_t(L) <= int64_t(p.max_pages) * kDecodeTok;
-  if (!ok) L = 0;
-  const int tiles = L > 0 ? (L + kDecodeTok - 1) / kDecodeTok : 1;
-  const int per = *p.range_len;
-  const int s = p.unit_start[u];
-  const int i0 = s / per, i1 = (s + tiles - 1) / per;
-  if (i0 == i1) return;   // held whole by one range: already written
-  const int np = i1 - i0 + 1;
-  const bool few = np <= 32;
-  // this lane's piece (few pieces) and the row's max and log-sum-exp
-  const float my_l = (few && lane < np)
-                         ? p.part_lse[int64_t(piece_slot(i0 + lane, s, per, G, cg)) * p.ncol + n]
-                         : -INFINITY;
-  float mx = my_l;
-  if (!few)
-    for (int i = i0 + lane; i <= i1; i += 32)
-      mx = fmaxf(mx, p.part_lse[int64_t(piece_slot(i, s, per, G, cg)) * p.ncol + n]);
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
-  float den = my_l == -INFINITY ? 0.0f : expf(my_l - mx);
-  if (!few) {
-    den = 0.0f;
-    for (int i = i0 + lane; i <= i1; i += 32) {
-      const float li = p.part_lse[int64_t(piece_slot(i, s, per, G, cg)) * p.ncol + n];
-      den += li == -INFINITY ? 0.0f : expf(li - mx);
-    }
-  }
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) den += __shfl_xor_sync(0xffffffffu, den, o);
-  const float lse = mx == -INFINITY ? -INFINITY : mx + logf(den);
-  float4 acc[4];
-#pragma unroll
-  for (int k = 0; k < 4; ++k) acc[k] = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
-  for (int i = i0; i <= i1; ++i) {
-    const int64_t sl = piece_slot(i, s, per, G, cg);
-    const float li = few ? __shfl_sync(0xffffffffu, my_l, i - i0) : p.part_lse[sl * p.ncol + n];
-    if (li == -INFINITY) continue;
-    const float wgt = expf(li - lse);
-    const uint16_t* row = p.part_o + (sl * p.ncol + n) * p.r;
-#pragma unroll
-    for (int k = 0; k < 4; ++k) {
-      const int lat = 4 * lane + 128 * k;
-      if (lat < p.r) {
-        const uint2 v = *reinterpret_cast<const uint2*>(row + lat);   // r % 4 == 0: 8-byte aligned
-        acc[k].x += wgt * __uint_as_float(v.x << 16);
-        acc[k].y += wgt * __uint_as_float(v.x & 0xFFFF0000u);
-        acc[k].z += wgt * __uint_as_float(v.y << 16);
-        acc[k].w += wgt * __uint_as_float(v.y & 0xFFFF0000u);
-      }
-    }
-  }
-  uint16_t* out = p.o_latent + (int64_t(b) * p.qH + f) * p.r;
-  const bool vec = (reinterpret_cast<uintptr_t>(out) & 7u) == 0;
-#pragma unroll
-  for (int k = 0; k < 4; ++k) {
-    const int lat = 4 * lane + 128 * k;
-    if (lat >= p.r) continue;
-    if (vec) {
-      *reinterpret_cast<uint2*>(out + lat) =
-          make_uint2(cvt_bf16x2(acc[k].x, acc[k].y), cvt_bf16x2(acc[k].z, acc[k].w));
-    } else {
-      out[lat] = f32_to_bf16_rne(acc[k].x);
-      out[lat + 1] = f32_to_bf16_rne(acc[k].y);
-      out[lat + 2] = f32_to_bf16_rne(acc[k].z);
-      out[lat + 3] = f32_to_bf16_rne(acc[k].w);
-    }
-  }
-  if (lane == 0) p.lse[int64_t(b) * p.qH + f] = lse;
-}
-
 #ifdef MLA_TRACE
 extern "C" int mla_trace_read(unsigned long long* host, int n) {
   return int(cudaMemcpyFromSymbol(host, g_mla_trace, sizeof(unsigned long long) *
@@ -809,17 +635,6 @@ extern "C" int mla_trace_read(unsigned long long* host, int n) {
 }
 #endif
 
-cudaError_t launch_combine(const CombineParams& p, cudaStream_t stream) {
-  const int64_t rows = int64_t(p.units) * p.ncol;
-  if (rows <= 0 || rows > 0x7fffffffLL || p.r > 512 || p.r % 4 != 0) return cudaErrorInvalidValue;
-  if (int64_t(p.vgrid) <= 4 * int64_t(p.units)) {
-    // a few pieces per unit: one warp per row
-    return launch_pdl(mla_combine_rows_kernel, dim3(unsigned((rows + 3) / 4)), dim3(128), 0,
-                      stream, 1, p);
-  }
-  // many pieces per unit: the four warps of a block split one row's pieces
-  return launch_pdl(mla_combine_kernel, dim3(unsigned(rows)), dim3(128), 0, stream, 1, p);
-}
 
 template <int NCOL>
 static cudaError_t launch_decode_n(const DecodeParams& p, dim3 grid, size_t smem,

@@ -73,7 +73,7 @@ struct WGemmParams {
   CUtensorMap tm_w;          // 3D weight map, box 128 x 64 (see launcher)
   CUtensorMap tm_x;          // 3D activations {K, H, rows}, box {64, 1, NR}
   uint16_t* out;             // element (n, h, m) at n*out_row_stride + h*out_head_stride + m
-  CUtensorMap tm_out;        // 3D {M, H, rows} over out, box {min(128, M), 1, NR}
+  CUtensorMap tm_out;        // 3D {M, H, rows} over out, box {128, 1, NR} (clipped past M)
   int64_t out_row_stride, out_head_stride;
   const uint16_t* bias;      // [H, M] or null
   int32_t* dev_error;
@@ -86,28 +86,31 @@ struct WGemmParams {
   const float* rope_sin;
   int32_t groups, rope_dim;
   int32_t rope_vec;          // 1: q_pe 8-byte, cos/sin 16-byte aligned and d_r/2 % 4 == 0
-  // fused cache append (mla_down_kv_append; cache == nullptr otherwise): the outputs are the
-  // D = r + G*d_r features of each token's [c_kv ; k_r], written as cache rows. Features
-  // come in ceil(r/128) latent tiles [128 t, 128 t + 128) and one rotary tile [r, D).
-  uint16_t* cache;           // [num_pages, page_size, D]
-  const int32_t* block_table;   // [B, max_pages]
-  const int32_t* start_pos;     // [B]
-  uint16_t* kv_out;          // [rows, D] bf16 GEMM output before the rotation, or null
-  int64_t num_pages;
-  int32_t max_pages, n_new, page_size, lat_r, lat_tiles;
-  // K split across CTAs (fused append only; 1 elsewhere): split s of an output tile sums
-  // the K blocks [s nk / splits, (s + 1) nk / splits) into acc with fp32 reductions, and the
-  // last split to finish (tile_done) reads the sums back, clears them and writes the rows.
-  int32_t splits;
-  float* acc;                // [rows, D] fp32, zero between calls
-  int32_t* tile_done;        // [tiles], zero between calls
   // cache append folded into the absorption (the one-call decode step; batch == 0 when
   // unused): the epilogue warps write the new tokens' cache rows before their first item
   AppendParams app;
 };
-// max_ctas: the persistent grid's size limit (one CTA per SM). With p.cache set the
-// output goes into the paged cache (see WGemmParams) instead of p.out.
+// max_ctas: the persistent grid's size limit (one CTA per SM).
 cudaError_t launch_wgemm(const WGemmParams& p, int nr, int max_ctas, cudaStream_t stream);
+
+// ---- mla_down_kv_append: split-K GEMM on clusters, cache rows in the epilogue (down_kv.cu)
+struct DkvParams {
+  CUtensorMap tm_w;          // 2D {hidden, D} over w_dkv, box {64, 128}
+  CUtensorMap tm_x;          // 2D {hidden, rows} over the hidden states, box {64, NR}
+  uint16_t* cache;           // [num_pages, page_size, D]
+  const int32_t* block_table;   // [B, max_pages]
+  const int32_t* start_pos;     // [B]
+  const float* rope_cos;     // [rows, G, d_r/2]
+  const float* rope_sin;
+  uint16_t* kv_out;          // [rows, D] or null
+  int32_t* dev_error;
+  int64_t num_pages;
+  int32_t max_pages, n_new, page_size, r, groups, rope_dim, rows, K;
+  int32_t lat_tiles;         // ceil(r / 128) latent feature tiles (+ one rotary tile)
+  int32_t n_nt;              // row tiles of NR tokens
+  int32_t splits;            // CTAs per cluster splitting K (the cluster size)
+};
+cudaError_t launch_down_kv(const DkvParams& p, int nr, cudaStream_t stream);
 
 // ---- mla_out_proj: einsum (5) then einsum (6) in one cooperative kernel (oproj.cu) -------
 struct OProjParams {
@@ -182,6 +185,7 @@ struct CombineParams {
   float* lse;
   int32_t q_len, max_seq_len, max_pages, qH, r, ncol, col_groups, units;
   int32_t vgrid;             // work ranges the decode used (pieces per unit ~ vgrid / units)
+  int32_t sms;               // SMs of the device (sizes the row-merge grid)
 };
 cudaError_t launch_combine(const CombineParams& p, cudaStream_t stream);
 

@@ -1,14 +1,11 @@
-// wgemm.cu - per-head weight GEMM on tcgen05 for mla_absorb_q, mla_out_up and
-// mla_down_kv_append.
+// wgemm.cu - per-head weight GEMM on tcgen05 for mla_absorb_q and mla_out_up.
 //
-// All three steps are "one small weight matrix per head times a few activation rows":
+// Both steps are "one small weight matrix per head times a few activation rows":
 //   absorb:  q_c[n, h, :]  = W_UK[h]^T q_nope[n, h, :]   (W_UK[h] stored [d_n][r])
 //   out_up:  o[n, h, :]    = W_UV[h]   o_latent[n, h, :] (W_UV[h] stored [d_v][r])
-//   down_kv: [c_kv ; k_r][n, :] = W_DKV x[n, :]          (one "head", W_DKV stored [D][hidden])
-// and the last one writes its output straight into the paged cache (mla_down_kv_append).
 // The weights dominate the bytes, so the output features are the UMMA M dimension
 // (128 per work item) and the activation rows the N dimension; D[m, n] lives in TMEM with
-// one output feature per lane, so the epilogue writes consecutive features per warp.
+// one output feature per lane.
 //
 // The grid is persistent: one CTA per SM walks the work items (head, 128-feature tile,
 // row tile) with a stride of the grid size. Per item the weight tile is only 16-128 KB,
@@ -17,7 +14,8 @@
 // stages) can be in flight at once. Warp 0 issues the TMA loads, warp 1 the UMMAs into
 // one of two TMEM accumulators, and warps 2-5 (one per TMEM sub-partition) drain the
 // other accumulator, so an item's epilogue overlaps the next item's loads and UMMAs. For
-// the absorb step the epilogue warps first write q_ext's rotary slots.
+// the absorb step the epilogue warps first write q_ext's rotary slots (and, in the one-call
+// decode step, the new tokens' cache rows).
 #include "append.cuh"
 #include "decode_sched.cuh"
 #include "kernels.h"
@@ -31,60 +29,34 @@ constexpr int kWgEpiThreads = 128;
 constexpr int kWgABytes = 128 * 128;   // 128 x 64 bf16 weight tile (two 64x64 boxes for W_UK)
 
 // Shared memory: the TMA stages, 256 bytes of barriers, two epilogue staging tiles of
-// [NR rows][128 features] bf16, NR cache-row indices (fused append), 1 KB alignment slack.
+// [NR rows][128 features] bf16, 1 KB alignment slack.
 template <int NR>
 struct WgLayout {
   static constexpr int kB = NR * 128;                 // NR rows x 64 bf16
   static constexpr int kStage = kWgABytes + kB;
   static constexpr int kEpi = NR * 128 * 2;           // one staging tile
-  static constexpr int kFit = (227 * 1024 - 256 - 2 * kEpi - NR * 8 - 1024) / kStage;
+  static constexpr int kFit = (227 * 1024 - 256 - 2 * kEpi - 1024) / kStage;
   static constexpr int kStages = kFit < 8 ? kFit : 8;
   static constexpr int kBars = kStage * kStages;      // barriers after the stages
   static constexpr int kEpiOff = kBars + 256;
-  static constexpr int kSlotOff = kEpiOff + 2 * kEpi;
-  static constexpr int kTotal = kSlotOff + NR * 8 + 1024;
+  static constexpr int kTotal = kEpiOff + 2 * kEpi + 1024;
 };
 
 MLA_DEVICE uint8_t* align1024(uint8_t* p) {
   return reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(p) + 1023) & ~uintptr_t(1023));
 }
 
-// Work item `it` -> (head, first output feature, first activation row). For the fused
-// append the last feature tile is the rotary one and starts at feature r (all of a
-// group's rotation pairs then sit in one tile); the others are 128-aligned latent tiles.
-// With K split in `splits` parts, items are (head, feature tile, split, row tile) and an
-// item covers the K blocks [kb0, kb1).
+// Work item `it` -> (head, first output feature, first activation row).
 struct WgItem {
-  int h, m0, n0, mt, s, kb0, kb1, tile;
-  MLA_DEVICE WgItem(int it, int n_mt, int n_nt, int nr, int rope_tile_m0, int splits, int nk) {
+  int h, m0, n0;
+  MLA_DEVICE WgItem(int it, int n_mt, int n_nt, int nr) {
     const int nt = it % n_nt;
-    const int rest = it / n_nt;
-    s = rest % splits;
-    const int hm = rest / splits;
+    const int hm = it / n_nt;
     h = hm / n_mt;
-    mt = hm % n_mt;
-    m0 = (rope_tile_m0 >= 0 && mt == n_mt - 1) ? rope_tile_m0 : mt * 128;
+    m0 = (hm % n_mt) * 128;
     n0 = nt * nr;
-    kb0 = s * nk / splits;
-    kb1 = (s + 1) * nk / splits;
-    tile = mt * n_nt + nt;
   }
 };
-
-MLA_DEVICE bool warp_leader(int sp, int lane) { return sp == 2 && lane == 0; }
-
-// Physical cache row of activation row `row` (token t of sequence b) for the fused append,
-// or -1 when its position or page is out of range (the caller sets the error word).
-MLA_DEVICE int64_t append_slot(const WGemmParams& p, int row) {
-  const int b = row / p.n_new;
-  const int t = row - b * p.n_new;
-  const int64_t pos = int64_t(p.start_pos[b]) + t;
-  const int64_t lp = pos >= 0 ? pos / p.page_size : -1;
-  if (pos < 0 || lp >= p.max_pages) return -1;
-  const int32_t page = p.block_table[int64_t(b) * p.max_pages + lp];
-  if (page < 0 || page >= p.num_pages) return -1;
-  return int64_t(page) * p.page_size + pos % p.page_size;
-}
 
 // One rotary chunk: outputs j..j+3 and j+half..j+half+3 of the (n, h, group) slice `seg`
 // (c = j / 4). Split into an address/load step and a compute/store step so that a thread
@@ -197,133 +169,6 @@ MLA_DEVICE void write_rope_slots(const WGemmParams& p, int tid, int nthreads) {
 }
 }  // namespace
 
-// Epilogue of the fused down-projection + cache append, run by the four epilogue warps for
-// one item: the accumulator (feature m0 + lane of each TMEM lane, one column per token) is
-// rounded to bf16 into a [NR tokens][128 features] staging tile, the accumulator is handed
-// back, and the tile is written as cache rows: latent features as 16-byte copies, rotary
-// features rotated in fp32 (separately rounded products and sums, from the rounded bf16
-// values, exactly as mla_cache_append) and rounded to bf16 with ties to even.
-// All four warps pass both named barriers whatever their accumulator wait returned (`ok`);
-// a failed wait leaves the CTA's abort flag set, and then no warp writes the tile.
-// With the K split in several CTAs (p.splits > 1) each split first adds its fp32 sums into
-// p.acc; the last split of the tile to finish reads the totals back (clearing them for the
-// next call) and writes the rows. `last` is a shared-memory flag of the CTA.
-template <int NR>
-MLA_DEVICE void append_epilogue(const WGemmParams& p, const WgItem& w, int buf, uint32_t tmem,
-                                int sp, int lane, uint16_t* stage, int64_t* slot_s,
-                                uint64_t* acc_empty, bool ok, volatile int* abort_flag,
-                                volatile int* last) {
-  const int m_loc = sp * 32 + lane;
-  const int nrows = min(NR, p.rows - w.n0);
-  const int D = p.lat_r + p.groups * p.rope_dim;
-  const int f = w.m0 + m_loc;                     // feature of this thread's TMEM lane
-  // the latent tiles own features [m0, r), the rotary tile [r, D)
-  const bool own = w.m0 < p.lat_r ? f < p.lat_r : f < D;
-  const bool split = p.splits > 1;
-  if (ok) {
-#pragma unroll 1
-    for (int c0 = 0; c0 < NR; c0 += 16) {
-      float v[16];
-      tmem_ld16(tmem + (uint32_t(sp * 32) << 16) + uint32_t(buf * NR + c0), v);
-      tmem_wait_ld();
-      if (split) {
-        if (own) {
-#pragma unroll
-          for (int j = 0; j < 16; ++j)
-            if (c0 + j < nrows) atomicAdd(p.acc + int64_t(w.n0 + c0 + j) * D + f, v[j]);
-        }
-      } else {
-#pragma unroll
-        for (int j = 0; j < 16; ++j) stage[(c0 + j) * 128 + m_loc] = f32_to_bf16_rne(v[j]);
-      }
-    }
-    if (split) __threadfence();
-  }
-  tc_fence_before();
-  __syncwarp();
-  if (lane == 0) mbar_arrive(acc_empty);
-  named_bar_sync(1, kWgEpiThreads);
-  if (split) {
-    if (warp_leader(sp, lane) && *abort_flag == 0) {
-      const int old = atomicAdd(p.tile_done + w.tile, 1);
-      *last = (old == p.splits - 1) ? 1 : 0;
-    }
-    named_bar_sync(1, kWgEpiThreads);
-    if (*last != 0 && *abort_flag == 0) {
-      // read the totals back (4 features per thread and step, several rows' loads in
-      // flight), clear them for the next call and round them into the staging tile
-      __threadfence();
-      const int f_end = w.m0 < p.lat_r ? min(w.m0 + 128, p.lat_r) : D;   // multiple of 4
-#pragma unroll 4
-      for (int idx = m_loc; idx < nrows * 32; idx += kWgEpiThreads) {
-        const int n = idx >> 5, c = 4 * (idx & 31);
-        float4 v = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
-        if (w.m0 + c < f_end) {
-          float4* a = reinterpret_cast<float4*>(p.acc + int64_t(w.n0 + n) * D + w.m0 + c);
-          v = __ldcg(a);
-          __stcg(a, make_float4(0.0f, 0.0f, 0.0f, 0.0f));
-        }
-        *reinterpret_cast<uint2*>(stage + n * 128 + c) =
-            make_uint2(cvt_bf16x2(v.x, v.y), cvt_bf16x2(v.z, v.w));
-      }
-      if (warp_leader(sp, lane)) p.tile_done[w.tile] = 0;
-    }
-    named_bar_sync(1, kWgEpiThreads);             // the staging tile is complete
-    const bool write = *last != 0;
-    named_bar_sync(1, kWgEpiThreads);             // every thread has read `last`
-    if (warp_leader(sp, lane)) *last = 0;
-    if (!write) return;
-  }
-  if (*abort_flag != 0) {
-    named_bar_sync(1, kWgEpiThreads);
-    return;
-  }
-  const int tid = m_loc;                          // 0..127
-  // the cache row of every token of the tile, looked up once (two dependent loads each)
-  if (tid < nrows) {
-    const int64_t slot = append_slot(p, w.n0 + tid);
-    if (slot < 0 && p.dev_error) atomicOr(p.dev_error, MLA_DEVERR_BOUNDS);
-    slot_s[tid] = slot;
-  }
-  named_bar_sync(1, kWgEpiThreads);
-  if (w.m0 < p.lat_r) {
-    // latent tile: features [m0, min(m0 + 128, r)) of every token, 8 per 16-byte chunk
-    const int chunks = (min(128, p.lat_r - w.m0)) / 8;
-    for (int idx = tid; idx < nrows * chunks; idx += kWgEpiThreads) {
-      const int n = idx / chunks, c = idx - (idx / chunks) * chunks;
-      const int row = w.n0 + n;
-      const uint4 v = *reinterpret_cast<const uint4*>(stage + n * 128 + c * 8);
-      if (p.kv_out) *reinterpret_cast<uint4*>(p.kv_out + int64_t(row) * D + w.m0 + c * 8) = v;
-      const int64_t slot = slot_s[n];
-      if (slot >= 0) *reinterpret_cast<uint4*>(p.cache + slot * D + w.m0 + c * 8) = v;
-    }
-  } else {
-    // rotary tile: features [r, D), pair j of group g = (x_j, x_{j + d_r/2})
-    const int half = p.rope_dim / 2;
-    const int pairs = p.groups * half;
-    for (int idx = tid; idx < nrows * pairs; idx += kWgEpiThreads) {
-      const int n = idx / pairs, pi = idx - (idx / pairs) * pairs;
-      const int g = pi / half, j = pi - (pi / half) * half;
-      const int row = w.n0 + n;
-      const int f = g * p.rope_dim + j;           // feature within the rotary tile
-      const uint16_t b0 = stage[n * 128 + f], b1 = stage[n * 128 + f + half];
-      if (p.kv_out) {
-        p.kv_out[int64_t(row) * D + p.lat_r + f] = b0;
-        p.kv_out[int64_t(row) * D + p.lat_r + f + half] = b1;
-      }
-      const int64_t slot = slot_s[n];
-      if (slot < 0) continue;
-      const float x0 = bf16_bits_to_f32(b0), x1 = bf16_bits_to_f32(b1);
-      const int64_t ci = (int64_t(row) * p.groups + g) * half + j;
-      const float cj = p.rope_cos[ci], sj = p.rope_sin[ci];
-      uint16_t* dst = p.cache + slot * D + p.lat_r + f;
-      dst[0] = f32_to_bf16_rne(__fsub_rn(__fmul_rn(x0, cj), __fmul_rn(x1, sj)));
-      dst[half] = f32_to_bf16_rne(__fadd_rn(__fmul_rn(x1, cj), __fmul_rn(x0, sj)));
-    }
-  }
-  named_bar_sync(1, kWgEpiThreads);               // the staging tile may be reused
-}
-
 // Epilogue of absorb / out_up for one item, run by the four epilogue warps: the
 // accumulator (output feature m0 + lane of each TMEM lane, one column per activation row)
 // plus the bias is rounded to bf16 into a [NR rows][128 features] staging tile (two
@@ -397,17 +242,13 @@ __global__ void __launch_bounds__(kWgThreads, 1) wgemm_kernel(const __grid_const
   uint64_t* acc_empty = acc_full + 2;                                 // [2] accumulator drained
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(acc_empty + 2);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
-  volatile int* last_flag = abort_flag + 1;
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-  const bool append = p.cache != nullptr;
-  const int rope_m0 = (append && p.groups * p.rope_dim > 0) ? p.lat_r : -1;
-  const int n_mt = append ? p.lat_tiles + (rope_m0 >= 0 ? 1 : 0) : (p.M + 127) / 128;
+  const int n_mt = (p.M + 127) / 128;
   const int n_nt = (p.rows + NR - 1) / NR;
   const int nk = (p.K + 63) / 64;
-  const int splits = p.splits > 1 ? p.splits : 1;
-  const int items = n_mt * p.heads * splits * n_nt;
+  const int items = n_mt * p.heads * n_nt;
   constexpr uint32_t kCols = 2 * NR < 32 ? 32 : 2 * NR;   // two accumulators of NR columns
   const WaitCtx wc{abort_flag, p.dev_error};
 
@@ -421,7 +262,6 @@ __global__ void __launch_bounds__(kWgThreads, 1) wgemm_kernel(const __grid_const
       mbar_init(&acc_empty[i], 4);                    // the four epilogue warps
     }
     *abort_flag = 0;
-    *last_flag = 0;
     fence_mbar_init();
   }
   if (warp == 1) {
@@ -442,8 +282,8 @@ __global__ void __launch_bounds__(kWgThreads, 1) wgemm_kernel(const __grid_const
       // The weights are no kernel's output here: warm L2 with this CTA's weight tiles while
       // the previous kernel may still run (an L2 prefetch is coherent with any writer).
       for (int it = blockIdx.x; it < items; it += gridDim.x) {
-        const WgItem w(it, n_mt, n_nt, NR, rope_m0, splits, nk);
-        for (int kb = w.kb0; kb < w.kb1; ++kb) {
+        const WgItem w(it, n_mt, n_nt, NR);
+        for (int kb = 0; kb < nk; ++kb) {
           if (p.a_mn) {
             tma_prefetch_l2_3d(&p.tm_w, w.m0, kb * 64, w.h);
             tma_prefetch_l2_3d(&p.tm_w, w.m0 + 64, kb * 64, w.h);
@@ -461,8 +301,8 @@ __global__ void __launch_bounds__(kWgThreads, 1) wgemm_kernel(const __grid_const
       int g = 0;   // stages issued
       bool ok = true;
       for (int it = blockIdx.x; ok && it < items; it += gridDim.x) {
-        const WgItem w(it, n_mt, n_nt, NR, rope_m0, splits, nk);
-        for (int kb = w.kb0; kb < w.kb1; ++kb, ++g, ring.next()) {
+        const WgItem w(it, n_mt, n_nt, NR);
+        for (int kb = 0; kb < nk; ++kb, ++g, ring.next()) {
           if (g >= S && !mbar_wait(&empty[ring.slot], (ring.round - 1) & 1, wc)) {
             ok = false;
             break;
@@ -494,13 +334,13 @@ __global__ void __launch_bounds__(kWgThreads, 1) wgemm_kernel(const __grid_const
       bool ok = true;
       int li = 0;   // items of this CTA so far
       for (int it = blockIdx.x; ok && it < items; it += gridDim.x, ++li) {
-        const WgItem w(it, n_mt, n_nt, NR, rope_m0, splits, nk);
+        const WgItem w(it, n_mt, n_nt, NR);
         const int buf = li & 1;
         // the epilogue has drained this accumulator (item li - 2)
         if (li >= 2 && !mbar_wait(&acc_empty[buf], ((li >> 1) - 1) & 1, wc)) break;
         tc_fence_after();
         const uint32_t d = tmem + uint32_t(buf * NR);
-        for (int kb = w.kb0; kb < w.kb1; ++kb, ring.next()) {
+        for (int kb = 0; kb < nk; ++kb, ring.next()) {
           if (!mbar_wait(&full[ring.slot], ring.round & 1, wc)) {
             ok = false;
             break;
@@ -514,7 +354,7 @@ __global__ void __launch_bounds__(kWgThreads, 1) wgemm_kernel(const __grid_const
             const uint64_t ad = p.a_mn ? make_sdesc(a + kk * 2048, 8192, 1024, kSw128)
                                        : make_sdesc(a + kk * 32, 16, 1024, kSw128);
             const uint64_t bd = make_sdesc(b + kk * 32, 16, 1024, kSw128);
-            umma_bf16(d, ad, bd, idesc, (kb != w.kb0 || kk != 0) ? 1u : 0u);
+            umma_bf16(d, ad, bd, idesc, (kb != 0 || kk != 0) ? 1u : 0u);
           }
           umma_commit(&empty[ring.slot]);
         }
@@ -538,17 +378,10 @@ __global__ void __launch_bounds__(kWgThreads, 1) wgemm_kernel(const __grid_const
                        int(gridDim.x) * kWgEpiThreads);
     int li = 0;
     for (int it = blockIdx.x; it < items; it += gridDim.x, ++li) {
-      const WgItem w(it, n_mt, n_nt, NR, rope_m0, splits, nk);
+      const WgItem w(it, n_mt, n_nt, NR);
       const int buf = li & 1;
       const bool ok = __all_sync(0xffffffffu, mbar_wait(&acc_full[buf], (li >> 1) & 1, wc));
       tc_fence_after();
-      if (append) {
-        append_epilogue<NR>(p, w, buf, tmem, sp, lane,
-                            reinterpret_cast<uint16_t*>(base + Lay::kEpiOff),
-                            reinterpret_cast<int64_t*>(base + Lay::kSlotOff), &acc_empty[buf],
-                            ok, abort_flag, last_flag);
-        continue;
-      }
       plain_epilogue<NR>(p, w, buf, tmem, sp, lane,
                          reinterpret_cast<uint16_t*>(base + Lay::kEpiOff + (li & 1) * Lay::kEpi),
                          &acc_empty[buf], ok, abort_flag);
@@ -563,14 +396,11 @@ __global__ void __launch_bounds__(kWgThreads, 1) wgemm_kernel(const __grid_const
 
 template <int NR>
 static cudaError_t launch_wgemm_nr(const WGemmParams& p, int max_ctas, cudaStream_t stream) {
-  const bool append = p.cache != nullptr;
   const int smem = WgLayout<NR>::kTotal;
   cudaError_t e = cudaFuncSetAttribute(wgemm_kernel<NR>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
-  const int64_t n_mt = append ? p.lat_tiles + (p.groups * p.rope_dim > 0 ? 1 : 0)
-                              : (p.M + 127) / 128;
-  const int64_t items = n_mt * p.heads * (p.splits > 1 ? p.splits : 1) * ((p.rows + NR - 1) / NR);
+  const int64_t items = int64_t((p.M + 127) / 128) * p.heads * ((p.rows + NR - 1) / NR);
   const int grid = int(items < max_ctas ? items : max_ctas);
   return launch_pdl(wgemm_kernel<NR>, dim3(grid), dim3(kWgThreads), size_t(smem), stream, 1, p);
 }

@@ -118,24 +118,19 @@ mla_status mla_cache_append(const mla_dims* dims, const void* c_kv, const void* 
  *   rope_cos/sin, block_table, start_pos, cache, num_pages, dev_error: as mla_cache_append
  *   kv_out      bf16 [B, n_new, D] or NULL    if given, also receives the GEMM's bf16
  *                                             output [c_kv ; k_r] before the rotation
- *   workspace   >= mla_down_kv_workspace_size(dims, B, n_new) bytes, 256-byte aligned,
- *               zeroed once after allocation; each call leaves it zero again (it holds the
- *               fp32 sums of the model width split across CTAs and their counters), so it
- *               serves later calls on the same stream, not concurrent ones
  *
  * For each token: [c_kv ; k_r] = bf16_rne(fp32 sum over hidden of w_dkv * x), then exactly
  * what mla_cache_append writes for that c_kv and k_r (the same cache bytes). The sum over
- * the model width is split across CTAs and added with fp32 atomics, so its last bit may
- * differ from call to call. Requires
- * G*d_r <= 128 (MLA_ERR_UNSUPPORTED otherwise). Bounds faults as mla_cache_append.
+ * the model width is split across the CTAs of a cluster and added in a fixed order, so
+ * every call gives the same bits. Needs no workspace. Requires G*d_r <= 128
+ * (MLA_ERR_UNSUPPORTED otherwise). Bounds faults as mla_cache_append.
  */
-size_t mla_down_kv_workspace_size(const mla_dims* dims, int32_t batch, int32_t n_new);
 mla_status mla_down_kv_append(const mla_dims* dims, const void* hidden, int32_t hidden_dim,
                               const void* w_dkv, const float* rope_cos, const float* rope_sin,
                               const int32_t* block_table, int32_t max_pages_per_seq,
                               const int32_t* start_pos, int32_t batch, int32_t n_new,
                               void* cache, int64_t num_pages, int32_t* dev_error, void* kv_out,
-                              void* workspace, size_t workspace_bytes, void* stream);
+                              void* stream);
 
 /*
  * mla_absorb_q - fold W_UK into the query and rotate its RoPE part.

@@ -237,13 +237,9 @@ def test_down_kv_append_validation(mla_lib):
     L = mla.lib()
     d = _dims()
 
-    def call(dd=d, hidden=FAKE, hid=5120, w=FAKE, batch=2, n=1, cache=FAKE, kv_out=None,
-             ws=P(0x10000), wsb=1 << 20):
+    def call(dd=d, hidden=FAKE, hid=5120, w=FAKE, batch=2, n=1, cache=FAKE, kv_out=None):
         return L.mla_down_kv_append(ctypes.byref(dd), hidden, hid, w, FAKE, FAKE, FAKE, 4, FAKE,
-                                    batch, n, cache, 100, None, kv_out, ws, wsb, None)
-    assert call(ws=None) == mla.MLA_ERR_WORKSPACE
-    assert call(wsb=16) == mla.MLA_ERR_WORKSPACE
-    assert mla.mla_down_kv_workspace_size(d, 64, 1) >= 64 * 576 * 4
+                                    batch, n, cache, 100, None, kv_out, None)
     assert call(hid=100) == mla.MLA_ERR_INVALID_ARG              # not a multiple of 8
     assert call(hidden=None) == mla.MLA_ERR_INVALID_ARG
     assert call(w=P(0x10008)) == mla.MLA_ERR_INVALID_ARG          # misaligned weight

@@ -83,11 +83,21 @@ def test_traffic_is_keyed_to_the_kernel_source(tmp_path, monkeypatch):
     monkeypatch.setattr(b, "ROOT", str(tmp_path))
     csrc = tmp_path / "head_latent_attention_attn_b200" / "csrc"
     csrc.mkdir(parents=True)
-    for f in ("decode_pair.cu", "decode.cu", "decode_sched.cuh", "ptx.cuh", "kernels.h"):
+    for f in ("decode_pair.cu", "decode.cu", "decode_sched.cuh", "ptx.cuh"):
         (csrc / f).write_text(f"// {f}\n")
+    hdr = "struct WGemmParams {\n  int a;\n};\nstruct DecodeParams {\n  int b;\n};\n"
+    (csrc / "kernels.h").write_text(hdr)
     h = b._source_hash(cfg)
     (prof / "decode_traffic.json").write_text(json.dumps(
         {"deepseek_v2": {"source_hash": h, "dram_bytes_per_launch": 123}}))
+    assert b._traffic(cfg) == 123
+    # another kernel's parameters change: the record still holds
+    (csrc / "kernels.h").write_text(hdr.replace("int a;", "int a, c;"))
+    assert b._traffic(cfg) == 123
+    # the decode kernel's parameters or source change: it does not
+    (csrc / "kernels.h").write_text(hdr.replace("int b;", "int b, d;"))
+    assert b._traffic(cfg) is None
+    (csrc / "kernels.h").write_text(hdr)
     assert b._traffic(cfg) == 123
     (csrc / "decode_pair.cu").write_text("// changed\n")
     assert b._traffic(cfg) is None
