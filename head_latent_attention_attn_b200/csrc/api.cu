@@ -662,8 +662,10 @@ mla_status build_decode(const mla_dims* dims, const void* q_ext, const void* cac
   return MLA_OK;
 }
 
-// The decode kernel of a built plan and, when units may be cut between CTAs, the merge.
-mla_status launch_decode_plan(const DecodePlan& P, const DecodeParams& p, cudaStream_t s) {
+// The decode kernel of a built plan and, when units may be cut between CTAs, the merge (which
+// then also brings `pf_bytes` at `pf`, the next kernel's weights, into L2; may be null).
+mla_status launch_decode_plan(const DecodePlan& P, const DecodeParams& p, cudaStream_t s,
+                              const void* pf = nullptr, int64_t pf_bytes = 0) {
   const cudaError_t le = P.pair ? launch_decode_pair(p, dim3(P.grid), P.smem, s)
                                 : launch_decode(p, P.ncol, dim3(P.grid), P.smem, s);
   if (le != cudaSuccess) return MLA_ERR_CUDA;
@@ -687,6 +689,8 @@ mla_status launch_decode_plan(const DecodePlan& P, const DecodeParams& p, cudaSt
     c.units = P.units;
     c.vgrid = P.vgrid;
     c.sms = num_sms();
+    c.l2_prefetch = pf;
+    c.l2_prefetch_bytes = pf_bytes;
     if (launch_combine(c, s) != cudaSuccess) return MLA_ERR_CUDA;
   }
   return MLA_OK;
@@ -756,7 +760,8 @@ mla_status mla_decode_step(const mla_dims* dims, const void* c_kv_new, const voi
   cudaStream_t s = as_stream(stream);
   if (!ap_empty) ab.app = ap;     // the absorption's epilogue warps write the new rows
   if (launch_wgemm(ab, nr_ab, num_sms(), s) != cudaSuccess) return MLA_ERR_CUDA;
-  st = launch_decode_plan(P, dp, s);
+  // the merge kernel (if the plan has one) brings W_UV into L2 for the up-projection
+  st = launch_decode_plan(P, dp, s, w_uv, int64_t(dims->num_heads) * w_uv_head_stride * 2);
   if (st != MLA_OK) return st;
   return launch_wgemm(ou, nr_ou, num_sms(), s) == cudaSuccess ? MLA_OK : MLA_ERR_CUDA;
 }

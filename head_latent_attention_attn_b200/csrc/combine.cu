@@ -12,6 +12,23 @@
 
 namespace mla {
 
+// Bring `bytes` (a multiple of 16) at the 16-byte-aligned global address `src` into L2.
+MLA_DEVICE void bulk_prefetch_l2(const void* src, uint32_t bytes) {
+  asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(src), "r"(bytes) : "memory");
+}
+
+// Before its grid-dependency wait, block i of the merge brings slice i of p.l2_prefetch into
+// L2 (the blocks start as the decode's CTAs leave, so this overlaps the decode's last CTAs).
+MLA_DEVICE void prefetch_next_weights(const CombineParams& p) {
+  if (p.l2_prefetch == nullptr || threadIdx.x != 0) return;
+  const int64_t slice = ((p.l2_prefetch_bytes + gridDim.x - 1) / gridDim.x + 15) & ~int64_t(15);
+  const int64_t off = int64_t(blockIdx.x) * slice;
+  const int64_t n = min(slice, p.l2_prefetch_bytes - off) & ~int64_t(15);
+  for (int64_t o = 0; o < n; o += 65536)
+    bulk_prefetch_l2(static_cast<const uint8_t*>(p.l2_prefetch) + off + o,
+                     uint32_t(min(int64_t(65536), n - o)));
+}
+
 // ---- merge of cut units: lse = log sum_i e^{lse_i}, o = sum_i e^{lse_i - lse} o_i ------
 // One block per (unit, query row): warp 0 reduces the pieces' lse, then the 4 warps split
 // the pieces and every lane accumulates up to 16 latents (8 x lane + 256 k + 0..7: one
@@ -20,6 +37,7 @@ namespace mla {
 __global__ void __launch_bounds__(128) mla_combine_kernel(const CombineParams p) {
   __shared__ float part[4][512];
   __shared__ float lse_s;
+  prefetch_next_weights(p);
   grid_dep_wait();
   grid_dep_launch();
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -110,6 +128,7 @@ __global__ void __launch_bounds__(128) mla_combine_kernel(const CombineParams p)
 constexpr int kFewPieces = 4;
 
 __global__ void __launch_bounds__(256) mla_combine_rows_kernel(const CombineParams p) {
+  prefetch_next_weights(p);
   grid_dep_wait();
   grid_dep_launch();
   const int lane = threadIdx.x & 31;

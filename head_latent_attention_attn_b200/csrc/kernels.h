@@ -186,6 +186,10 @@ struct CombineParams {
   int32_t q_len, max_seq_len, max_pages, qH, r, ncol, col_groups, units;
   int32_t vgrid;             // work ranges the decode used (pieces per unit ~ vgrid / units)
   int32_t sms;               // SMs of the device (sizes the row-merge grid)
+  // optional: bytes the next kernel of the step reads (the up-projection's weights), brought
+  // into L2 by the merge blocks before they wait for the decode grid (null: none)
+  const void* l2_prefetch;
+  int64_t l2_prefetch_bytes;
 };
 cudaError_t launch_combine(const CombineParams& p, cudaStream_t stream);
 
