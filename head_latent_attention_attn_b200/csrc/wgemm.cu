@@ -368,9 +368,12 @@ __global__ void __launch_bounds__(kWgThreads, 1) wgemm_kernel(const __grid_const
     grid_dep_launch();
     const int sp = warp & 3;
     {
-      // new tokens' cache rows (one warp per token) while the first accumulator fills
+      // new tokens' cache rows (one warp per token) while the first accumulator fills; dealt
+      // from the last CTA down, since the items are dealt from the first CTA up and the last
+      // CTAs may hold one item fewer
       const int64_t ntok = int64_t(p.app.batch) * p.app.n_new;
-      for (int64_t gw = int64_t(blockIdx.x) * 4 + (warp - 2); gw < ntok; gw += int64_t(gridDim.x) * 4)
+      for (int64_t gw = int64_t(gridDim.x - 1 - blockIdx.x) * 4 + (warp - 2); gw < ntok;
+           gw += int64_t(gridDim.x) * 4)
         append_token(p.app, gw, lane);
     }
     if (p.q_pe != nullptr && p.rope_dim > 0)
