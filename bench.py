@@ -281,9 +281,12 @@ def max_over_ranks(values, dist, device):
     return [float(x) for x in vec.tolist()]
 
 
-def cpu_oracle_sample(cfg, wl, budget_s=12.0, max_seqs=None):
-    """Time the fp64 oracle on whole sequences of the workload until ``budget_s`` is spent."""
+def cpu_oracle_sample(cfg, wl, budget_s=12.0, max_seqs=None, absorbed=False):
+    """Time the fp64 oracle on whole sequences of the workload until ``budget_s`` is spent
+    (None: every sequence). ``absorbed``: the oracle's absorbed form (einsums 3-5 of the
+    DeepSeek-V2 page's matrix absorption) instead of the unabsorbed one."""
     import oracle.mla_oracle as O
+    fn = O.mla_decode_absorbed if absorbed else O.mla_decode_reference
     try:
         from threadpoolctl import threadpool_info
         cores = max([i.get("num_threads", 1) for i in threadpool_info()] + [1])
@@ -293,17 +296,19 @@ def cpu_oracle_sample(cfg, wl, budget_s=12.0, max_seqs=None):
     done, tok_ctx, t0 = [], 0, time.perf_counter()
     for b in order:
         c_kv, k_r = wl.context(int(b))
-        O.mla_decode_reference(wl.q_nope[b], wl.q_pe[b], c_kv, k_r, wl.w_uk, wl.w_uv, wl.bias,
-                               wl.theta, wl.query_positions()[b], cfg.softmax_scale, causal=cfg.causal)
+        fn(wl.q_nope[b], wl.q_pe[b], c_kv, k_r, wl.w_uk, wl.w_uv, wl.bias, wl.theta,
+           wl.query_positions()[b], cfg.softmax_scale, causal=cfg.causal)
         done.append(int(b))
         tok_ctx += int(wl.seq_lens[b])
-        if time.perf_counter() - t0 >= budget_s or (max_seqs and len(done) >= max_seqs):
+        if ((budget_s is not None and time.perf_counter() - t0 >= budget_s) or
+                (max_seqs and len(done) >= max_seqs)):
             break
     el = time.perf_counter() - t0
+    form = "absorbed" if absorbed else "unabsorbed"
     return {"value": len(done) * cfg.q_len / el, "unit": "tokens/s", "cores": int(cores),
-            "kind": "oracle",
+            "kind": "oracle_absorbed" if absorbed else "oracle",
             "sample": f"{len(done)} of {cfg.batch} sequences ({tok_ctx} cached tokens, all "
-                      f"{cfg.num_heads} heads), fp64 unabsorbed form, {el:.1f} s"}
+                      f"{cfg.num_heads} heads), fp64 {form} form, {el:.1f} s"}
 
 
 def run_reference(args, cfg, rank, world):
@@ -400,6 +405,7 @@ PER_CONFIG = ("tiny", "qwen25_7b", "qwen3_30b_a3b", "hybrid_1m_q1", "hybrid_1m_q
               "prefill_hybrid_q64", "prefill_hybrid_q256", "prefill_hybrid_q1024")
 DOWN_KV = ("deepseek_v2", "qwen3_30b_a3b")   # mla_down_kv_append at these decode batches
 OUT_PROJ = ("deepseek_v2",)                  # mla_out_proj at this decode batch
+CPU_FULL = ("tiny", "qwen25_7b")             # both fp64 CPU forms timed over every sequence
 DECODE_BLOCK = 60   # decode launches timed back to back for the roofline figure
 
 
@@ -459,6 +465,18 @@ def run_gpu(args, cfg, rank, world, dist):
             step_ms = time_calls(lambda st: one_step(), args.steps, stream, flush)
         # the decode alone, back to back: the roofline figure (median of DECODE_BLOCK launches)
         dec_block = time_decode(prob, cfg, DECODE_BLOCK, stream, flush)
+        # the same step as four library calls (append, absorb, decode + merge, out_up)
+        if flush is None:
+            t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            t0.record(stream)
+            for _ in range(args.steps):
+                prob.step_four_calls(stream)
+            t1.record(stream)
+            torch.cuda.synchronize()
+            step4_ms = [t0.elapsed_time(t1) / args.steps]
+        else:
+            step4_ms = time_calls(lambda st: prob.step_four_calls(stream), args.steps, stream,
+                                  flush)
         barrier()
         clk.mark_end()
     t_step = statistics.mean(step_ms)
@@ -549,7 +567,8 @@ def run_gpu(args, cfg, rank, world, dist):
         raise RuntimeError("end-to-end outputs differ from the device-resident step")
 
     # ---- max over ranks -------------------------------------------------------------------
-    t_step, t_dec, t_dec_mean, t_e2e = max_over_ranks([t_step, t_dec, t_dec_mean, t_e2e], dist, dev)
+    t_step, t_dec, t_dec_mean, t_e2e, t_step4 = max_over_ranks(
+        [t_step, t_dec, t_dec_mean, t_e2e, statistics.mean(step4_ms)], dist, dev)
     peaks = _peaks()
     tokens = cfg.batch * cfg.q_len
     value = world * tokens / (t_step * 1e-3)
@@ -557,7 +576,8 @@ def run_gpu(args, cfg, rank, world, dist):
     # absorb with the append folded in, decode, out_up (+ the split combine when the plan has
     # > 1 split; a one-split plan needs only the 256-byte error-word workspace)
     merge = 1 if plan_splits_ws > 256 else 0
-    launches = (3 + merge) * args.steps + (1 + merge) * DECODE_BLOCK
+    # the one-call steps, the decode block and the four-call steps
+    launches = (3 + merge) * args.steps + (1 + merge) * DECODE_BLOCK + (4 + merge) * args.steps
     line = {
         "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": t_step,
@@ -565,6 +585,7 @@ def run_gpu(args, cfg, rank, world, dist):
         "data": "synthetic",
         "config": dict(_config_json(cfg), l2=("cache > L2, no flush" if flush is None
                                               else "L2 flushed between launches (504 MB write)")),
+        "step_four_calls_ms": t_step4,
         "decode_us": 1e3 * t_dec, "decode_us_mean": 1e3 * t_dec_mean,
         "decode_launches_timed": DECODE_BLOCK,
         "step_timing": ("K steps back to back between two events" if flush is None
@@ -588,6 +609,9 @@ def run_gpu(args, cfg, rank, world, dist):
         return
     if world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_oracle_sample(cfg, wl, budget_s=args.cpu_budget)
+        # the absorbed fp64 form beside it: a second CPU baseline
+        line["cpu_baseline_absorbed"] = cpu_oracle_sample(cfg, wl, budget_s=args.cpu_budget / 2,
+                                                          absorbed=True)
     print(json.dumps(line), flush=True)
 
 
@@ -629,6 +653,11 @@ def per_config_block(args, head_cfg, dev, stream, dist, peaks):
                      "roofline": roofline_of(cfg, wl.seq_lens, t_med, peaks),
                      "l2": "cache > L2, no flush" if flush is None else "L2 flushed between launches",
                      "clocks": clk.summary()}
+        # the two smallest workloads: both fp64 CPU forms over every sequence (rank 0, N = 1)
+        if name in CPU_FULL and not args.no_cpu_baseline and dist is None:
+            out[name]["cpu_baseline"] = cpu_oracle_sample(cfg, wl, budget_s=None)
+            out[name]["cpu_baseline_absorbed"] = cpu_oracle_sample(cfg, wl, budget_s=None,
+                                                                   absorbed=True)
         del prob, flush, wl
         torch.cuda.empty_cache()
     # einsums (5) and (6) fused (mla_out_proj) at the DeepSeek-V2 decode batch

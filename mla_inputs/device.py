@@ -111,6 +111,19 @@ class DeviceProblem:
                             lse=self.lse, o=self.o, causal=self.cfg.causal,
                             num_splits=self.num_splits, stream=stream)
 
+    def step_four_calls(self, stream=None) -> None:
+        """The same decode step as four library calls: append, absorb, decode (+ merge),
+        up-projection."""
+        mla.mla_cache_append(self.dims, self.c_new, self.k_new, self.cos_q, self.sin_q,
+                             self.block_table, self.start_pos, self.cache,
+                             dev_error=self.workspace.view(torch.int32)[:1], stream=stream)
+        mla.mla_absorb_q(self.dims, self.q_nope, self.q_pe, self.cos_q, self.sin_q, self.w_uk,
+                         self.q_ext, stream=stream)
+        mla.mla_decode_attn(self.dims, self.q_ext, self.cache, self.block_table, self.seq_lens,
+                            self.max_seq_len, self.workspace, self.o_latent, self.lse,
+                            causal=self.cfg.causal, num_splits=self.num_splits, stream=stream)
+        mla.mla_out_up(self.dims, self.o_latent, self.w_uv, self.o, bias=self.bias, stream=stream)
+
     def decode_only(self, num_splits=None) -> None:
         ns = self.num_splits if num_splits is None else num_splits
         mla.mla_decode_attn(self.dims, self.q_ext, self.cache, self.block_table, self.seq_lens,
