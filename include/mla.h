@@ -15,8 +15,12 @@
  *
  * Conventions shared by every call
  *   - Every data pointer is DEVICE memory owned by the caller; the library allocates
- *     nothing and keeps no state between calls, so concurrent calls on different
- *     streams are safe as long as their output buffers differ.
+ *     nothing and keeps no state between calls that a result depends on, so concurrent
+ *     calls on different streams are safe as long as their output buffers differ. Two
+ *     exceptions: mla_decode_attn_noalloc's fixed scratch array (one call at a time, see
+ *     there), and a mutex-guarded, per-device memo of a hardware property (how many
+ *     two-CTA clusters of the decode fit on the device at once, which is constant for a
+ *     device and shared-memory size).
  *   - bf16 tensors are passed as void* (uint16 storage), contiguous, row-major, in the
  *     shapes given below; fp32 and int32 tensors likewise.
  *   - Calls are asynchronous on `stream` (a cudaStream_t / CUstream; NULL = the legacy
